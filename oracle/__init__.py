@@ -1,0 +1,163 @@
+"""Python access to the fp64 CPU oracle (``spec_verify_oracle.c``).
+
+TEST INFRASTRUCTURE ONLY: imported by tests/, ``__graft_entry__.smoke()`` and
+the CPU-baseline leg of ``bench.py``.  The CUDA library never imports it and
+it never imports the CUDA library.  Arguments are numpy arrays; bf16 logits
+are passed as their uint16 bit patterns.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+from typing import Optional
+
+import numpy as np
+
+from . import build as _build
+
+DTYPE_BF16 = 0
+DTYPE_F32 = 1
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        _lib = ctypes.CDLL(_build.build())
+        P, I, D = ctypes.c_void_p, ctypes.c_int, ctypes.c_double
+        _lib.oracle_process_row.argtypes = [P, I, I, D, I, P, P]
+        _lib.oracle_process_row.restype = I
+        _lib.oracle_argmax_row.argtypes = [P, I, I]
+        _lib.oracle_argmax_row.restype = I
+        _lib.oracle_inverse_cdf.argtypes = [P, I, D, P, P, P]
+        _lib.oracle_inverse_cdf.restype = I
+        _lib.oracle_verify.argtypes = [P, P, P, P, I, I, I, P, I, I, I, P, P, P, P, P, P, P]
+        _lib.oracle_verify.restype = I
+        _lib.oracle_sample_rows.argtypes = [P, I, I, I, P, I, I, P, P, P, P]
+        _lib.oracle_sample_rows.restype = I
+    return _lib
+
+
+def _ptr(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _dtype_code(a: np.ndarray) -> int:
+    if a.dtype == np.uint16:
+        return DTYPE_BF16
+    if a.dtype == np.float32:
+        return DTYPE_F32
+    raise TypeError(f"logits must be uint16 (bf16 bits) or float32, got {a.dtype}")
+
+
+def process_row(row: np.ndarray, temperature: float = 1.0, top_k: int = 0):
+    """Processed probabilities of one logit row (fp64), or None on a row error."""
+    row = np.ascontiguousarray(row)
+    V = row.shape[-1]
+    prob = np.zeros(V, dtype=np.float64)
+    work = np.zeros(V, dtype=np.float64)
+    rc = lib().oracle_process_row(_ptr(row), _dtype_code(row), V, float(temperature), int(top_k),
+                                  _ptr(prob), _ptr(work))
+    return None if rc else prob
+
+
+def argmax_row(row: np.ndarray) -> int:
+    row = np.ascontiguousarray(row)
+    return lib().oracle_argmax_row(_ptr(row), _dtype_code(row), row.shape[-1])
+
+
+def inverse_cdf(w: np.ndarray, u: float):
+    """(token, cdf_lo, cdf_hi) of the inverse-CDF draw, or None if the mass is 0."""
+    w = np.ascontiguousarray(w, dtype=np.float64)
+    tok = ctypes.c_int(-1)
+    lo = ctypes.c_double(0)
+    hi = ctypes.c_double(0)
+    rc = lib().oracle_inverse_cdf(_ptr(w), w.size, float(u), ctypes.byref(tok), ctypes.byref(lo),
+                                  ctypes.byref(hi))
+    return None if rc else (tok.value, lo.value, hi.value)
+
+
+@dataclasses.dataclass
+class VerifyResult:
+    tokens: np.ndarray      # [B, k+1] int32
+    n_accepted: np.ndarray  # [B] int32
+    p: np.ndarray           # [B, k] fp64 (NaN for greedy / error rows)
+    q: np.ndarray           # [B, k] fp64
+    ratio: np.ndarray       # [B, k] acceptance thresholds min(1, p/q)
+    cdf_lo: np.ndarray      # [B] CDF point below the final token
+    cdf_hi: np.ndarray      # [B] CDF point at the final token
+    errors: int
+
+
+def verify(target: np.ndarray, draft: Optional[np.ndarray], draft_tokens: np.ndarray,
+           uniforms: Optional[np.ndarray], temperature: Optional[np.ndarray] = None,
+           top_k: int = 0, greedy: bool = False) -> VerifyResult:
+    """Verify a batch: target [B,k+1,V], draft [B,k,V], draft_tokens [B,k],
+    uniforms [B,k+1], temperature [B]."""
+    target = np.ascontiguousarray(target)
+    B, k1, V = target.shape
+    k = k1 - 1
+    dt = _dtype_code(target)
+    if draft is not None:
+        draft = np.ascontiguousarray(draft)
+        assert draft.dtype == target.dtype and draft.shape == (B, k, V)
+    elif not greedy:
+        raise ValueError("stochastic verification needs draft logits")
+    draft_tokens = np.ascontiguousarray(draft_tokens, dtype=np.int32).reshape(B, k)
+    if uniforms is not None:
+        uniforms = np.ascontiguousarray(uniforms, dtype=np.float32).reshape(B, k + 1)
+    elif not greedy:
+        raise ValueError("stochastic verification needs uniforms")
+    if temperature is not None:
+        temperature = np.ascontiguousarray(temperature, dtype=np.float32).reshape(B)
+    tokens = np.empty((B, k + 1), dtype=np.int32)
+    n = np.empty(B, dtype=np.int32)
+    p = np.empty((B, max(k, 0)), dtype=np.float64)
+    q = np.empty_like(p)
+    ratio = np.empty_like(p)
+    lo = np.empty(B, dtype=np.float64)
+    hi = np.empty(B, dtype=np.float64)
+    errs = lib().oracle_verify(_ptr(target), _ptr(draft), _ptr(draft_tokens), _ptr(uniforms), B, k,
+                               V, _ptr(temperature), int(top_k), int(bool(greedy)), dt,
+                               _ptr(tokens), _ptr(n), _ptr(p), _ptr(q), _ptr(ratio), _ptr(lo),
+                               _ptr(hi))
+    if errs < 0:
+        raise MemoryError("oracle_verify could not allocate its work arrays")
+    return VerifyResult(tokens, n, p, q, ratio, lo, hi, errs)
+
+
+def sample_rows(logits: np.ndarray, u: Optional[np.ndarray], temperature: Optional[np.ndarray] = None,
+                top_k: int = 0, greedy: bool = False):
+    """One token per row of ``logits`` [..., V]; returns (tokens, cdf_lo, cdf_hi)."""
+    logits = np.ascontiguousarray(logits)
+    shape = logits.shape[:-1]
+    V = logits.shape[-1]
+    rows = int(np.prod(shape)) if shape else 1
+    if u is not None:
+        u = np.ascontiguousarray(u, dtype=np.float32).reshape(rows)
+    elif not greedy:
+        raise ValueError("stochastic sampling needs uniforms")
+    if temperature is not None:
+        temperature = np.ascontiguousarray(temperature, dtype=np.float32).reshape(rows)
+    out = np.empty(rows, dtype=np.int32)
+    lo = np.empty(rows, dtype=np.float64)
+    hi = np.empty(rows, dtype=np.float64)
+    errs = lib().oracle_sample_rows(_ptr(logits), _dtype_code(logits), rows, V, _ptr(temperature),
+                                    int(top_k), int(bool(greedy)), _ptr(u), _ptr(out), _ptr(lo),
+                                    _ptr(hi))
+    if errs < 0:
+        raise MemoryError("oracle_sample_rows could not allocate its work arrays")
+    return out.reshape(shape), lo.reshape(shape), hi.reshape(shape)
+
+
+def draft_tokens_for(case) -> np.ndarray:
+    """The proposer's tokens for a ``workloads.Case``: d_i ~ q_i processed with
+    the case's temperature and top-k (stochastic), or the argmax of the noisy
+    proxy (greedy)."""
+    if case.mode == "greedy":
+        tok, _, _ = sample_rows(case.draft_proxy, None, greedy=True)
+        return tok.astype(np.int32)
+    temp = np.repeat(case.temperature, case.k)
+    tok, _, _ = sample_rows(case.draft, case.draft_uniforms, temp, case.top_k)
+    return tok.astype(np.int32)

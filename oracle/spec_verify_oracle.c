@@ -1,0 +1,307 @@
+/*
+ * Plain fp64 CPU oracle for batched speculative-sampling verification.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may call, link or
+ * execute this file; only tests/, the smoke check and the benchmark's CPU
+ * baseline leg use it.  It shares no code, header or constant with the CUDA
+ * library: it restates the method from the pages in the plainest way, one
+ * sequence at a time, single threaded, every value held in double.
+ *
+ * Source of the method (speculative decoding encyclopedia entry "推测解码",
+ * glopedia.cn/401080):
+ *   - section "提议与核验的基本步骤", paragraph 2: the draft token x at
+ *     position i is accepted with probability min(1, p(x)/q(x)); p and q are
+ *     the conditional probabilities under the sampling settings actually in
+ *     use; acceptance stops at the first rejection; the rejected position is
+ *     redrawn from the normalised positive residual max(0, p - q); when every
+ *     candidate passes, one extra token is drawn from the target.
+ *   - same section, paragraph 3: the worked example (A/B/C, 0.6/0.3/0.1 vs
+ *     0.5/0.4/0.1) used as a pin in the tests.
+ *   - same section, paragraph 4: greedy verification compares the draft with
+ *     the target's most probable token and replaces it at the first
+ *     mismatch; temperature / top-k must be applied identically to p and q
+ *     and kept consistent in the correction step.
+ *
+ * Readings of what the pages leave open (each stated where it is used):
+ *   R1 accept iff u*q < p  (i.e. u < min(1, p/q) for u in [0,1));
+ *   R2 the final draw (correction or bonus) uses its own uniform u_k;
+ *   R3 inverse CDF: smallest v with C_v > u*W, C the running sum in index
+ *      order, W = C_{V-1}; if none (rounding) the largest v with w_v > 0;
+ *   R4 top-k keeps every logit >= tau, tau = K-th largest raw logit counted
+ *      with multiplicity (ties at tau are all kept);
+ *   R5 temperature divides the logits before the softmax; top-k is chosen on
+ *      the raw logits;
+ *   R6 greedy: lowest index among equal maxima, values compared as numbers
+ *      (-0.0 == +0.0); after a full match the target's argmax at position k
+ *      is emitted; temperature, top-k and uniforms are ignored;
+ *   R7 row errors: a NaN or +inf logit, no finite kept logit, a draft token
+ *      outside [0, V), a temperature that is not finite and > 0 (stochastic
+ *      only), a uniform outside [0, 1) (stochastic only).  The whole
+ *      sequence is then reported as n = -1 with every token -1;
+ *   R8 if the residual mass W is zero at a rejected position the
+ *      replacement is drawn from p at that position with the same rule.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define OR_DTYPE_BF16 0
+#define OR_DTYPE_F32 1
+
+/* ---- reading logits (bf16 widening is exact) ---------------------------- */
+
+static double or_logit(const void* row, int dtype, long v) {
+    if (dtype == OR_DTYPE_BF16) {
+        uint32_t bits = ((uint32_t)((const uint16_t*)row)[v]) << 16;
+        float f;
+        memcpy(&f, &bits, sizeof f);
+        return (double)f;
+    }
+    return (double)((const float*)row)[v];
+}
+
+static const void* or_row(const void* base, int dtype, long row, long V) {
+    size_t elt = dtype == OR_DTYPE_BF16 ? 2 : 4;
+    return (const char*)base + (size_t)row * (size_t)V * elt;
+}
+
+static int cmp_desc(const void* a, const void* b) {
+    double x = *(const double*)a, y = *(const double*)b;
+    return (x < y) - (x > y);
+}
+
+/*
+ * Logits processing of one row, the same for target and draft (section
+ * "提议与核验的基本步骤", paragraph 4: processing rules applied identically).
+ *   kept = all v, or {v : z_v >= tau} when 0 < top_k < V        (R4)
+ *   s_v = z_v / T, m = max_kept s, e_v = exp(s_v - m), S = sum_kept e_v
+ *   prob_v = e_v / S on kept entries, 0 elsewhere.
+ * Returns 0, or 1 for a row error (R7).  `work` holds V doubles.
+ */
+int oracle_process_row(const void* row, int dtype, int V, double T, int top_k,
+                       double* prob, double* work) {
+    long v;
+    double tau = -INFINITY, m = -INFINITY, S = 0.0;
+    if (!(T > 0.0) || isinf(T)) return 1;
+    for (v = 0; v < V; ++v) {
+        double z = or_logit(row, dtype, v);
+        if (isnan(z) || z == INFINITY) return 1;
+        work[v] = z;
+    }
+    if (top_k > 0 && top_k < V) {
+        qsort(work, (size_t)V, sizeof(double), cmp_desc);
+        tau = work[top_k - 1];
+    }
+    for (v = 0; v < V; ++v) {
+        double z = or_logit(row, dtype, v);
+        if (z >= tau && z / T > m) m = z / T;
+    }
+    if (m == -INFINITY) return 1;
+    for (v = 0; v < V; ++v) {
+        double z = or_logit(row, dtype, v);
+        prob[v] = (z >= tau) ? exp(z / T - m) : 0.0;
+        S += prob[v];
+    }
+    for (v = 0; v < V; ++v) prob[v] /= S;
+    return 0;
+}
+
+/* Lowest-index argmax of the raw row (R6).  Returns -1 on a row error. */
+int oracle_argmax_row(const void* row, int dtype, int V) {
+    long v;
+    int best = -1;
+    double bv = -INFINITY;
+    for (v = 0; v < V; ++v) {
+        double z = or_logit(row, dtype, v);
+        if (isnan(z) || z == INFINITY) return -1;
+        if (z > bv) {
+            bv = z;
+            best = (int)v;
+        }
+    }
+    return best; /* -1 when every entry is -inf */
+}
+
+/*
+ * Inverse-CDF draw from non-negative weights w (R3).  Writes the token and
+ * the two CDF points C_{y-1}/W and C_y/W around it.  Returns 1 if W == 0.
+ */
+int oracle_inverse_cdf(const double* w, int V, double u, int* token, double* cdf_lo,
+                       double* cdf_hi) {
+    long v;
+    double W = 0.0, C = 0.0, x;
+    int last_pos = -1;
+    for (v = 0; v < V; ++v) {
+        W += w[v];
+        if (w[v] > 0.0) last_pos = (int)v;
+    }
+    if (!(W > 0.0)) return 1;
+    x = u * W;
+    for (v = 0; v < V; ++v) {
+        double prev = C;
+        C += w[v];
+        if (C > x) {
+            *token = (int)v;
+            *cdf_lo = prev / W;
+            *cdf_hi = C / W;
+            return 0;
+        }
+    }
+    /* rounding left u*W at or above the running total: largest positive v */
+    C = 0.0;
+    for (v = 0; v < last_pos; ++v) C += w[v];
+    *token = last_pos;
+    *cdf_lo = C / W;
+    *cdf_hi = (C + w[last_pos]) / W;
+    return 0;
+}
+
+/*
+ * Batched verification, one sequence after another.
+ *   target        [B][k+1][V]   dtype
+ *   draft         [B][k][V]     dtype (ignored when greedy != 0)
+ *   draft_tokens  [B][k]
+ *   uniforms      [B][k+1]      u_0..u_{k-1} acceptance, u_k final draw (R2)
+ *   temperature   [B] or NULL (all 1.0)
+ * Outputs: out_tokens [B][k+1], out_n [B]; optional (NULL to skip)
+ *   out_p, out_q  [B][k]   p_i(d_i), q_i(d_i) at every position i < k
+ *   out_ratio     [B][k]   acceptance threshold min(1, p/q) (q = 0: 1 if p>0 else 0)
+ *   out_lo, out_hi [B]     CDF points around the final token
+ * Returns the number of sequences reported as row errors.
+ */
+int oracle_verify(const void* target, const void* draft, const int32_t* draft_tokens,
+                  const float* uniforms, int B, int k, int V, const float* temperature,
+                  int top_k, int greedy, int dtype, int32_t* out_tokens, int32_t* out_n,
+                  double* out_p, double* out_q, double* out_ratio, double* out_lo,
+                  double* out_hi) {
+    int b, i, errors = 0;
+    double* pt = (double*)malloc(sizeof(double) * (size_t)(k + 1) * (size_t)V);
+    double* pd = (double*)malloc(sizeof(double) * (size_t)(k > 0 ? k : 1) * (size_t)V);
+    double* w = (double*)malloc(sizeof(double) * (size_t)V);
+    double* work = (double*)malloc(sizeof(double) * (size_t)V);
+    if (!pt || !pd || !w || !work) {
+        free(pt); free(pd); free(w); free(work);
+        return -1;
+    }
+    for (b = 0; b < B; ++b) {
+        int32_t* tok = out_tokens + (size_t)b * (k + 1);
+        const int32_t* d = draft_tokens + (size_t)b * k;
+        const float* u = uniforms ? uniforms + (size_t)b * (k + 1) : NULL;
+        double T = temperature ? (double)temperature[b] : 1.0;
+        int err = 0, j = k, y = -1;
+        double lo = NAN, hi = NAN;
+        for (i = 0; i < k; ++i)
+            if (d[i] < 0 || d[i] >= V) err = 1;
+        for (i = 0; i <= k; ++i) tok[i] = -1;
+        if (out_p) for (i = 0; i < k; ++i) out_p[(size_t)b * k + i] = NAN;
+        if (out_q) for (i = 0; i < k; ++i) out_q[(size_t)b * k + i] = NAN;
+        if (out_ratio) for (i = 0; i < k; ++i) out_ratio[(size_t)b * k + i] = NAN;
+
+        if (greedy) {
+            /* R6: g_i = argmax of target row i; the first mismatch emits g_j.
+             * Every row is examined so that a bad row anywhere is reported. */
+            for (i = 0; i <= k && !err; ++i) {
+                int g = oracle_argmax_row(or_row(target, dtype, (long)b * (k + 1) + i, V), dtype, V);
+                if (g < 0) {
+                    err = 1;
+                } else if (i < k && j == k && d[i] != g) {
+                    j = i;
+                    y = g;
+                } else if (i == k && j == k) {
+                    y = g;
+                }
+            }
+        } else {
+            if (!(T > 0.0) || isinf(T) || isnan(T)) err = 1;
+            for (i = 0; i <= k && !err; ++i)
+                if (!(u[i] >= 0.0f && u[i] < 1.0f)) err = 1;
+            for (i = 0; i <= k && !err; ++i)
+                err |= oracle_process_row(or_row(target, dtype, (long)b * (k + 1) + i, V), dtype,
+                                          V, T, top_k, pt + (size_t)i * V, work);
+            for (i = 0; i < k && !err; ++i)
+                err |= oracle_process_row(or_row(draft, dtype, (long)b * k + i, V), dtype, V, T,
+                                          top_k, pd + (size_t)i * V, work);
+            if (!err) {
+                long v;
+                int found = 0;
+                /* p_i(d_i), q_i(d_i) at every position; R1 for the decisions */
+                for (i = 0; i < k; ++i) {
+                    double p = pt[(size_t)i * V + d[i]], q = pd[(size_t)i * V + d[i]];
+                    if (out_p) out_p[(size_t)b * k + i] = p;
+                    if (out_q) out_q[(size_t)b * k + i] = q;
+                    if (out_ratio)
+                        out_ratio[(size_t)b * k + i] = q > 0.0 ? (p / q < 1.0 ? p / q : 1.0)
+                                                               : (p > 0.0 ? 1.0 : 0.0);
+                    if (!found && !((double)u[i] * q < p)) {
+                        j = i;
+                        found = 1;
+                    }
+                }
+                if (j < k) {
+                    /* residual max(0, p_j - q_j), R8 if it has no mass */
+                    for (v = 0; v < V; ++v) {
+                        double r = pt[(size_t)j * V + v] - pd[(size_t)j * V + v];
+                        w[v] = r > 0.0 ? r : 0.0;
+                    }
+                    if (oracle_inverse_cdf(w, V, (double)u[k], &y, &lo, &hi))
+                        oracle_inverse_cdf(pt + (size_t)j * V, V, (double)u[k], &y, &lo, &hi);
+                } else {
+                    /* bonus token from the processed target at position k */
+                    oracle_inverse_cdf(pt + (size_t)k * V, V, (double)u[k], &y, &lo, &hi);
+                }
+            }
+        }
+        if (err) {
+            out_n[b] = -1;
+            errors++;
+        } else {
+            for (i = 0; i < j; ++i) tok[i] = d[i];
+            tok[j] = y;
+            out_n[b] = j;
+        }
+        if (out_lo) out_lo[b] = lo;
+        if (out_hi) out_hi[b] = hi;
+    }
+    free(pt); free(pd); free(w); free(work);
+    return errors;
+}
+
+/*
+ * Proposer sampling step, one token per row (the draft side of a round):
+ * stochastic rows draw from the processed row with the inverse CDF (R3, R4,
+ * R5) and their own uniform; greedy rows take the lowest-index argmax (R6).
+ *   logits [rows][V], temperature [rows] or NULL, u [rows] (stochastic)
+ * out_tokens[r] = -1 on a row error.  out_lo/out_hi optional.
+ */
+int oracle_sample_rows(const void* logits, int dtype, int rows, int V, const float* temperature,
+                       int top_k, int greedy, const float* u, int32_t* out_tokens,
+                       double* out_lo, double* out_hi) {
+    int r, errors = 0;
+    double* prob = (double*)malloc(sizeof(double) * (size_t)V);
+    double* work = (double*)malloc(sizeof(double) * (size_t)V);
+    if (!prob || !work) {
+        free(prob); free(work);
+        return -1;
+    }
+    for (r = 0; r < rows; ++r) {
+        const void* row = or_row(logits, dtype, r, V);
+        int y = -1;
+        double lo = NAN, hi = NAN;
+        if (greedy) {
+            y = oracle_argmax_row(row, dtype, V);
+        } else {
+            double T = temperature ? (double)temperature[r] : 1.0;
+            if ((u[r] >= 0.0f && u[r] < 1.0f) &&
+                oracle_process_row(row, dtype, V, T, top_k, prob, work) == 0) {
+                if (oracle_inverse_cdf(prob, V, (double)u[r], &y, &lo, &hi)) y = -1;
+            }
+        }
+        if (y < 0) errors++;
+        out_tokens[r] = y;
+        if (out_lo) out_lo[r] = lo;
+        if (out_hi) out_hi[r] = hi;
+    }
+    free(prob); free(work);
+    return errors;
+}
