@@ -1,0 +1,432 @@
+"""Benchmark: batched speculative-sampling verification on B200.
+
+One step = one ``spec_verify`` call over one batch of synthetic inputs (every
+row of the workload read once: target [B,k+1,V], draft [B,k,V]).  Metric:
+verified draft positions per second (B*k per step) and logit GB/s, with the
+verify kernel's achieved HBM bandwidth against the measured copy peak.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...   # the fp64 CPU oracle on host cores
+
+Multi-GPU (torchrun, one process per GPU): every rank verifies its own
+batch (independent replicas, no data-path collective); the JSON line reports
+the units of all ranks over the slowest rank's device time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+PROFILE_DIR = os.path.join(ROOT, "profiles")
+KERNEL_SOURCES = [os.path.join(ROOT, "draft_token_verification_verify_b200", "csrc", f)
+                  for f in ("sv_kernels.cuh", "sv_ptx.cuh", "spec_verify.cu")]
+
+DESCR = {
+    "tiny": "tiny stochastic verify B=1 k=4 V=32 fp32 T=1",
+    "single": "single-sequence stochastic verify B=1 k=8 V=151936 bf16 T=1",
+    "batched": "batched stochastic verify B=64 k=4 V=151936 bf16 T=0.7 top-k 50",
+    "greedy": "batched greedy verify B=256 k=8 V=151936 bf16",
+    "large": "large-batch stochastic verify B=512 k=3 V=128256 fp32 T in {0.5,1,1.5}",
+}
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def measured_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel source (else None)."""
+    path = os.path.join(PROFILE_DIR, f"sv_unit_kernel_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    for line in open(path):
+        if line.startswith("- ") and ":" in line:
+            k, v = line[2:].split(":", 1)
+            vals[k.strip()] = v.strip().strip("`")
+    if vals.get("kernel_source_sha256_16") != kernel_source_hash():
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling while the GPU is busy."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for name, val in zip(("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                                  "sw_power_cap"), f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+def to_dev(a, device):
+    import torch
+
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:
+        return torch.from_numpy(a.view(np.int16)).to(device).view(torch.bfloat16)
+    return torch.from_numpy(a).to(device)
+
+
+def to_pinned(a):
+    import torch
+
+    a = np.ascontiguousarray(a)
+    t = torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a)
+    t = t.pin_memory()
+    return t.view(torch.bfloat16) if a.dtype == np.uint16 else t
+
+
+def cpu_baseline(name: str, case, drafts, budget_s: float):
+    """The fp64 oracle, as it stands, on a bounded sample of the same batch:
+    sequences one after another until the time budget is spent."""
+    import oracle
+
+    greedy = case.mode == "greedy"
+    done, t0 = 0, time.perf_counter()
+    while done < case.B:
+        s = slice(done, done + 1)
+        oracle.verify(case.target[s], None if greedy else case.draft[s], drafts[s],
+                      None if greedy else case.uniforms[s], case.temperature[s], case.top_k, greedy)
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": done * case.k / dt, "unit": "positions/s", "cores": 1, "kind": "oracle",
+            "sample": f"{done} of {workloads.WORKLOADS[name].B} sequences of the {name} workload "
+                      f"({DESCR[name]}), single thread, {dt:.1f} s"}
+
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+
+    name = args.workload
+    w = workloads.WORKLOADS[name]
+    case = workloads.make_case(name, seed=0, B=min(4, w.B))
+    drafts = oracle.draft_tokens_for(case)
+    greedy = case.mode == "greedy"
+    per_step = 1 if name in ("single", "batched", "greedy", "large") else case.B
+
+    def step(i):
+        b = i % case.B
+        s = slice(b, b + per_step)
+        oracle.verify(case.target[s], None if greedy else case.draft[s], drafts[s],
+                      None if greedy else case.uniforms[s], case.temperature[s], case.top_k, greedy)
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(i)
+    dt = time.perf_counter() - t0
+    value = args.steps * per_step * case.k / dt
+    line = {
+        "impl": "reference", "metric": "verified draft positions/sec", "value": value,
+        "unit": "positions/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000 * dt / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": DESCR[name], "sample_per_step": f"{per_step} sequence(s)"},
+        "cpu_baseline": {"value": value, "unit": "positions/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{per_step} sequence(s) of the {name} workload per step, single thread"},
+        "e2e": {"value": value, "unit": "positions/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import torch
+
+    import draft_token_verification_verify_b200 as sv
+
+    world, rank, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    sv.lib()
+
+    name = args.workload
+    w = workloads.WORKLOADS[name]
+    case = workloads.make_case(name, seed=1000 + rank)
+    B, k, V = case.B, case.k, case.V
+    greedy = case.mode == "greedy"
+    mode = (sv.SV_MODE_GREEDY if greedy else sv.SV_MODE_STOCHASTIC) | (
+        sv.SV_DTYPE_BF16 if case.dtype == "bf16" else sv.SV_DTYPE_F32)
+    logit_bytes = case.logit_bytes()
+
+    target0 = to_dev(case.target, dev)
+    draft0 = None if greedy else to_dev(case.draft, dev)
+    unif = None if greedy else to_dev(case.uniforms, dev)
+    temp = to_dev(case.temperature, dev)
+    # the proposer's tokens, drawn on the GPU by the library's sampler (untimed)
+    if greedy:
+        drafts = sv.sample(to_dev(case.draft_proxy, dev), greedy=True)
+    else:
+        drafts = sv.sample(draft0, to_dev(case.draft_uniforms, dev), temp.repeat_interleave(k), case.top_k)
+    torch.cuda.synchronize()
+
+    # rotate input sets so that consecutive steps never hit in L2
+    nsets = max(2, -(-4 * L2_BYTES // logit_bytes)) if logit_bytes < 4 * L2_BYTES else 1
+    nsets = min(nsets, 64)
+    targets = [target0] + [target0.clone() for _ in range(nsets - 1)]
+    drafts_l = [draft0] + ([draft0.clone() for _ in range(nsets - 1)] if draft0 is not None else [None] * (nsets - 1))
+    out_tok = torch.empty((B, k + 1), dtype=torch.int32, device=dev)
+    out_n = torch.empty((B,), dtype=torch.int32, device=dev)
+    status = torch.zeros((1,), dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(i, ev0=None, ev1=None):
+        opts = sv.make_options(event_start=ev0, event_stop=ev1) if ev0 is not None else None
+        st = sv.spec_verify_ex(targets[i % nsets], drafts_l[i % nsets], drafts, unif, B, k, V, temp,
+                               case.top_k, mode, out_tok, out_n, None, None, status, opts, stream)
+        if st != sv.SV_OK:
+            raise sv.SpecVerifyError(st, "spec_verify_ex")
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if int(status.item()) != 0:
+        raise SystemExit(f"device status {int(status.item())} during warm-up")
+
+    # clock window: the same work back to back while nvidia-smi samples
+    sampler = ClockSampler(local)
+    sampler.start()
+    t_end = time.perf_counter() + args.clock_window
+    i = 0
+    while time.perf_counter() < t_end:
+        for _ in range(64):
+            step(i)
+            i += 1
+        torch.cuda.synchronize()
+
+    # ---- timed region: exactly K steps --------------------------------------------
+    evk = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_stop = torch.cuda.Event(enable_timing=True)
+    for a, b in evk:  # torch creates the CUDA event on first record
+        a.record(stream)
+        b.record(stream)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t_start.record(stream)
+    for s in range(args.steps):
+        step(s, evk[s][0], evk[s][1])
+    t_stop.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop()
+    elapsed_ms = t_start.elapsed_time(t_stop)
+    kern_ms = [a.elapsed_time(b) for a, b in evk]
+    if world > 1:
+        t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    if int(status.item()) != 0:
+        raise SystemExit(f"device status {int(status.item())} in the timed region")
+
+    units = B * k * args.steps * world
+    value = units / (elapsed_ms / 1000.0)
+    gbs = logit_bytes * args.steps * world / (elapsed_ms / 1000.0) / 1e9
+    kmean = sum(kern_ms) / len(kern_ms)
+    peak, peak_src = measured_peak()
+    achieved = logit_bytes / (kmean / 1000.0) / 1e9
+    traffic = profiled_traffic(name)
+
+    # ---- end to end through the public API, host (pinned) buffers -------------------
+    e2e = None
+    if not args.no_e2e:
+        h_target = to_pinned(case.target)
+        h_draft = None if greedy else to_pinned(case.draft)
+        h_tok = drafts.cpu().pin_memory()
+        h_unif = None if greedy else to_pinned(case.uniforms)
+        h_temp = to_pinned(case.temperature)
+        o_tok = torch.empty((B, k + 1), dtype=torch.int32).pin_memory()
+        o_n = torch.empty((B,), dtype=torch.int32).pin_memory()
+        d_target, d_draft = targets[0], drafts_l[0]
+        d_tok = torch.empty_like(drafts)
+        d_unif = None if greedy else torch.empty_like(unif)
+        d_temp = torch.empty_like(temp)
+        h2d = sum(x.numel() * x.element_size() for x in (h_target, h_draft, h_tok, h_unif, h_temp)
+                  if x is not None)
+        d2h = o_tok.numel() * 4 + o_n.numel() * 4
+
+        def e2e_step():
+            d_target.copy_(h_target, non_blocking=True)
+            if h_draft is not None:
+                d_draft.copy_(h_draft, non_blocking=True)
+                d_unif.copy_(h_unif, non_blocking=True)
+            d_tok.copy_(h_tok, non_blocking=True)
+            d_temp.copy_(h_temp, non_blocking=True)
+            st = sv.spec_verify(d_target, d_draft, d_tok, d_unif, B, k, V, d_temp, case.top_k, mode,
+                                out_tok, out_n, stream)
+            if st != sv.SV_OK:
+                raise sv.SpecVerifyError(st, "spec_verify")
+            o_tok.copy_(out_tok, non_blocking=True)
+            o_n.copy_(out_n, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        n_e2e = max(3, min(args.steps, 20))
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        a.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = a.elapsed_time(b)
+        if world > 1:
+            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": B * k * n_e2e * world / (e_ms / 1000.0), "unit": "positions/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": n_e2e}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(name, case, drafts.cpu().numpy(), args.cpu_budget)
+
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": "verified draft positions/sec", "value": value, "unit": "positions/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": case.dtype, "data": "synthetic",
+        "config": {"workload": DESCR[name], "B": B, "k": k, "V": V, "top_k": case.top_k,
+                   "mode": case.mode, "per_rank_batch": B, "parallelism": f"replicas x{world}",
+                   "l2": f"{nsets} rotating input sets of {logit_bytes / 1e6:.1f} MB (> 126 MB L2)",
+                   "clocks_window": f"sampled over a {args.clock_window:.1f} s window of the same "
+                                    "steps right before the timed region"},
+        "logit_gbs": gbs,
+        "logit_bytes_per_step": logit_bytes,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
+                     "kernel": "sv_unit_kernel", "kernel_ms_mean": kmean,
+                     "kernel_ms_median": statistics.median(kern_ms)},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(workloads.WORKLOADS), default="batched")
+    ap.add_argument("--clock-window", type=float, default=1.5)
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,209 @@
+"""Batched speculative-sampling verification on B200: Python binding.
+
+Argument marshalling only.  Every entry point forwards to the C ABI of
+``libspec_verify.so`` (declared in ``include/spec_verify.h``), whose CUDA
+kernels do all of the work; there is no Python or CPU fallback, and a
+missing library raises ``ImportError``-style errors on first use.
+
+Pointers may be given as torch tensors (their ``data_ptr()`` is passed), as
+integers, or as ``None`` (NULL).  Streams may be a ``torch.cuda.Stream``, a
+raw ``cudaStream_t`` integer, or ``None`` for torch's current stream.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+from . import _build
+
+SV_OK = 0
+SV_ERR_INVALID_ARG = -1
+SV_ERR_UNSUPPORTED = -2
+SV_ERR_CUDA = -3
+SV_ERR_DEVICE_TIMEOUT = -4
+
+SV_MODE_STOCHASTIC = 0
+SV_MODE_GREEDY = 1
+SV_DTYPE_BF16 = 0 << 8
+SV_DTYPE_F32 = 1 << 8
+
+LIB_PATH = _build.LIB
+
+__all__ = [
+    "SV_OK", "SV_ERR_INVALID_ARG", "SV_ERR_UNSUPPORTED", "SV_ERR_CUDA", "SV_ERR_DEVICE_TIMEOUT",
+    "SV_MODE_STOCHASTIC", "SV_MODE_GREEDY", "SV_DTYPE_BF16", "SV_DTYPE_F32", "SvOptions",
+    "SpecVerifyError", "lib", "spec_verify", "spec_verify_ex", "spec_sample", "spec_sample_ex",
+    "spec_verify_status_string", "spec_verify_version", "verify", "sample",
+]
+
+
+class SvOptions(ctypes.Structure):
+    """Mirror of ``sv_options_t``."""
+    _fields_ = [
+        ("cluster_size", ctypes.c_int),
+        ("threads", ctypes.c_int),
+        ("topk_path", ctypes.c_int),
+        ("event_start", ctypes.c_void_p),
+        ("event_stop", ctypes.c_void_p),
+        ("wait_timeout_ns", ctypes.c_uint64),
+        ("test_extra_tx", ctypes.c_uint32),
+    ]
+
+
+class SpecVerifyError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what} failed: {spec_verify_status_string(status)} ({status})")
+        self.status = status
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load the C-ABI library (built in-tree by ``__graft_entry__.build()``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: run __graft_entry__.build() first")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I = ctypes.c_void_p, ctypes.c_int
+        L.spec_verify.argtypes = [P, P, P, P, I, I, I, P, I, I, P, P, P]
+        L.spec_verify.restype = I
+        L.spec_verify_ex.argtypes = [P, P, P, P, I, I, I, P, I, I, P, P, P, P, P,
+                                     ctypes.POINTER(SvOptions), P]
+        L.spec_verify_ex.restype = I
+        L.spec_sample.argtypes = [P, P, I, I, P, I, I, P, P]
+        L.spec_sample.restype = I
+        L.spec_sample_ex.argtypes = [P, P, I, I, P, I, I, P, ctypes.POINTER(SvOptions), P]
+        L.spec_sample_ex.restype = I
+        L.spec_verify_status_string.argtypes = [I]
+        L.spec_verify_status_string.restype = ctypes.c_char_p
+        L.spec_verify_version.argtypes = []
+        L.spec_verify_version.restype = I
+        _lib = L
+    return _lib
+
+
+def _p(x):
+    if x is None:
+        return None
+    if hasattr(x, "data_ptr"):
+        return ctypes.c_void_p(x.data_ptr())
+    return ctypes.c_void_p(int(x))
+
+
+def _stream(s):
+    if s is None:
+        import torch
+
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if hasattr(s, "cuda_stream"):
+        return ctypes.c_void_p(s.cuda_stream)
+    return ctypes.c_void_p(int(s))
+
+
+def _event(e):
+    if e is None:
+        return None
+    if hasattr(e, "cuda_event"):
+        return e.cuda_event
+    return int(e)
+
+
+def _opts(opts: Optional[SvOptions]):
+    return None if opts is None else ctypes.byref(opts)
+
+
+def spec_verify_status_string(status: int) -> str:
+    return lib().spec_verify_status_string(int(status)).decode()
+
+
+def spec_verify_version() -> int:
+    return lib().spec_verify_version()
+
+
+def spec_verify(target_logits, draft_logits, draft_tokens, uniforms, B, k, V, temperature, top_k,
+                mode, out_tokens, out_n_accepted, stream=None) -> int:
+    return lib().spec_verify(_p(target_logits), _p(draft_logits), _p(draft_tokens), _p(uniforms),
+                             int(B), int(k), int(V), _p(temperature), int(top_k), int(mode),
+                             _p(out_tokens), _p(out_n_accepted), _stream(stream))
+
+
+def spec_verify_ex(target_logits, draft_logits, draft_tokens, uniforms, B, k, V, temperature, top_k,
+                   mode, out_tokens, out_n_accepted, out_p=None, out_q=None, out_status=None,
+                   opts: Optional[SvOptions] = None, stream=None) -> int:
+    return lib().spec_verify_ex(_p(target_logits), _p(draft_logits), _p(draft_tokens), _p(uniforms),
+                                int(B), int(k), int(V), _p(temperature), int(top_k), int(mode),
+                                _p(out_tokens), _p(out_n_accepted), _p(out_p), _p(out_q),
+                                _p(out_status), _opts(opts), _stream(stream))
+
+
+def spec_sample(logits, uniforms, rows, V, temperature, top_k, mode, out_tokens, stream=None) -> int:
+    return lib().spec_sample(_p(logits), _p(uniforms), int(rows), int(V), _p(temperature), int(top_k),
+                             int(mode), _p(out_tokens), _stream(stream))
+
+
+def spec_sample_ex(logits, uniforms, rows, V, temperature, top_k, mode, out_tokens,
+                   opts: Optional[SvOptions] = None, stream=None) -> int:
+    return lib().spec_sample_ex(_p(logits), _p(uniforms), int(rows), int(V), _p(temperature),
+                                int(top_k), int(mode), _p(out_tokens), _opts(opts), _stream(stream))
+
+
+def make_options(cluster_size=0, threads=0, topk_path=0, event_start=None, event_stop=None,
+                 wait_timeout_ns=0, test_extra_tx=0) -> SvOptions:
+    return SvOptions(cluster_size, threads, topk_path, _event(event_start), _event(event_stop),
+                     wait_timeout_ns, test_extra_tx)
+
+
+def _dtype_code(t) -> int:
+    import torch
+
+    if t.dtype == torch.bfloat16:
+        return SV_DTYPE_BF16
+    if t.dtype == torch.float32:
+        return SV_DTYPE_F32
+    raise TypeError(f"logits must be bfloat16 or float32, got {t.dtype}")
+
+
+def verify(target, draft, draft_tokens, uniforms=None, temperature=None, top_k: int = 0,
+           greedy: bool = False, out_tokens=None, out_n_accepted=None, out_p=None, out_q=None,
+           out_status=None, opts: Optional[SvOptions] = None, stream=None):
+    """Tensor convenience wrapper around ``spec_verify_ex``.
+
+    target [B, k+1, V], draft [B, k, V] (bf16 or fp32, contiguous, on the
+    GPU), draft_tokens [B, k] int32, uniforms [B, k+1] fp32, temperature [B]
+    fp32 or None.  Output tensors are allocated with torch when not given.
+    Returns (out_tokens [B, k+1], out_n_accepted [B]).
+    """
+    import torch
+
+    B, k1, V = target.shape
+    k = k1 - 1
+    dev = target.device
+    if out_tokens is None:
+        out_tokens = torch.empty((B, k + 1), dtype=torch.int32, device=dev)
+    if out_n_accepted is None:
+        out_n_accepted = torch.empty((B,), dtype=torch.int32, device=dev)
+    mode = (SV_MODE_GREEDY if greedy else SV_MODE_STOCHASTIC) | _dtype_code(target)
+    st = spec_verify_ex(target, draft, draft_tokens, uniforms, B, k, V, temperature, top_k, mode,
+                        out_tokens, out_n_accepted, out_p, out_q, out_status, opts, stream)
+    if st != SV_OK:
+        raise SpecVerifyError(st, "spec_verify_ex")
+    return out_tokens, out_n_accepted
+
+
+def sample(logits, uniforms=None, temperature=None, top_k: int = 0, greedy: bool = False,
+           out_tokens=None, opts: Optional[SvOptions] = None, stream=None):
+    """Tensor convenience wrapper around ``spec_sample_ex``: logits [..., V]."""
+    import torch
+
+    V = logits.shape[-1]
+    rows = logits.numel() // V
+    if out_tokens is None:
+        out_tokens = torch.empty(logits.shape[:-1], dtype=torch.int32, device=logits.device)
+    mode = (SV_MODE_GREEDY if greedy else SV_MODE_STOCHASTIC) | _dtype_code(logits)
+    st = spec_sample_ex(logits, uniforms, rows, V, temperature, top_k, mode, out_tokens, opts, stream)
+    if st != SV_OK:
+        raise SpecVerifyError(st, "spec_sample_ex")
+    return out_tokens

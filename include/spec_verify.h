@@ -1,0 +1,165 @@
+/*
+ * spec_verify — batched speculative-sampling verification on NVIDIA B200
+ * (sm_100a).  C ABI; every entry point is asynchronous on the caller's
+ * CUDA stream.
+ *
+ * What is computed (speculative decoding entry "推测解码", glopedia.cn/401080,
+ * section "提议与核验的基本步骤"):
+ *   For each sequence b the caller supplies target logits at k+1 positions,
+ *   draft logits at k positions, the k draft tokens d_0..d_{k-1} and k+1
+ *   uniforms.  Both sides are processed identically (temperature, top-k,
+ *   full-vocabulary softmax; paragraph 4).  Position i accepts d_i iff
+ *   u_i * q_i(d_i) < p_i(d_i), i.e. with probability min(1, p/q)
+ *   (paragraph 2); acceptance stops at the first rejection j, whose token is
+ *   redrawn from the normalised residual max(0, p_j - q_j); if all k pass,
+ *   a bonus token is drawn from p_k.  Both draws use u_k and the inverse
+ *   CDF in index order (smallest v with C_v > u_k * W).  Greedy mode instead
+ *   compares d_i with the lowest-index argmax of the target row
+ *   (paragraph 4) and emits the target token at the first mismatch, or the
+ *   argmax of row k after a full match.
+ *
+ * Conventions fixed by this library where the method leaves them open:
+ *   - top-k keeps every logit >= tau, tau = the K-th largest raw logit
+ *     counted with multiplicity, so ties at tau are all kept;
+ *   - temperature divides the logits before the softmax; top-k is chosen on
+ *     the raw logits; -inf logits have probability 0;
+ *   - q(d) = 0 accepts iff p(d) > 0; a zero residual mass (only possible
+ *     through rounding or when p(d) = q(d) = 0) redraws from p_j;
+ *   - argmax ties go to the lowest index; -0.0 equals +0.0.
+ *
+ * Memory: every pointer is DEVICE memory owned by the caller and must stay
+ * valid until the stream work completes.  The library allocates nothing and
+ * keeps no state between calls.  Logits are contiguous row-major; bf16 rows
+ * need 2-byte and fp32 rows 4-byte alignment (16-byte-aligned rows take the
+ * fastest path).  Integer and float arrays need 4-byte alignment.
+ *
+ * Errors:
+ *   - argument problems found on the host return SV_ERR_INVALID_ARG with no
+ *     launch (B <= 0, k < 1, V < 1, top_k < 0, unknown mode or dtype bits,
+ *     a required pointer NULL or misaligned, sizes that overflow);
+ *   - SV_ERR_UNSUPPORTED: no usable CUDA device of compute capability >= 9.0,
+ *     or a vocabulary whose rows do not fit the per-cluster shared memory
+ *     (2 * V * element size > 16 * ~200 KB for verification);
+ *   - SV_ERR_CUDA: a CUDA call failed while launching;
+ *   - per-sequence data errors do not fail the call: out_n_accepted[b] = -1
+ *     and out_tokens[b, :] = -1.  They are a draft token outside [0, V), a
+ *     temperature that is not finite and > 0, a uniform outside [0, 1), a
+ *     NaN or +inf logit, or a row with no finite kept logit.  In greedy mode
+ *     temperature, top-k and uniforms are ignored;
+ *   - a device-side wait that runs out (bounded at about one second) marks
+ *     its sequence as an error and writes SV_ERR_DEVICE_TIMEOUT to
+ *     *out_status (spec_verify_ex).
+ */
+#ifndef SPEC_VERIFY_H
+#define SPEC_VERIFY_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SV_API __attribute__((visibility("default")))
+#else
+#define SV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum sv_status {
+    SV_OK = 0,
+    SV_ERR_INVALID_ARG = -1,
+    SV_ERR_UNSUPPORTED = -2,
+    SV_ERR_CUDA = -3,
+    SV_ERR_DEVICE_TIMEOUT = -4
+} sv_status_t;
+
+/* mode = one SV_MODE_* (low byte) OR-ed with one SV_DTYPE_* */
+enum {
+    SV_MODE_STOCHASTIC = 0,
+    SV_MODE_GREEDY = 1,
+    SV_DTYPE_BF16 = 0 << 8,
+    SV_DTYPE_F32 = 1 << 8
+};
+
+/* Tuning and instrumentation for spec_verify_ex / spec_sample_ex.  Zero
+ * every field for the library's own choices. */
+typedef struct sv_options {
+    int cluster_size;          /* CTAs per row pair: 0 = auto, else 1, 2, 4, 8 or 16 */
+    int threads;               /* threads per CTA: 0 = auto (256), else 128, 256 or 512 */
+    int topk_path;             /* 0 = auto, 1 = candidate threshold path, 2 = radix select */
+    void* event_start;         /* cudaEvent_t or NULL, recorded before the verify kernel */
+    void* event_stop;          /* cudaEvent_t or NULL, recorded right after it */
+    uint64_t wait_timeout_ns;  /* bound of every device-side wait: 0 = 1e9 ns */
+    uint32_t test_extra_tx;    /* test hook: bytes added to each bulk-copy wait so that
+                                  the bounded wait runs out (0 in normal use) */
+} sv_options_t;
+
+/*
+ * spec_verify — verify one speculative round for B sequences.
+ *   target_logits  [B][k+1][V]  bf16 or fp32 (per `mode`)
+ *   draft_logits   [B][k][V]    same dtype; may be NULL in greedy mode
+ *   draft_tokens   [B][k]       int32
+ *   uniforms       [B][k+1]     fp32: u_0..u_{k-1} decide acceptance, u_k
+ *                               drives the correction or bonus draw; may be
+ *                               NULL in greedy mode
+ *   B, k, V        sequences, draft length (>= 1), vocabulary size
+ *   temperature    [B] fp32 per-sequence temperature, or NULL for 1.0
+ *   top_k          0 or >= V disables top-k; else applied to p and q alike
+ *   mode           SV_MODE_* | SV_DTYPE_*
+ *   out_tokens     [B][k+1] int32: d_0..d_{j-1}, the corrected/bonus token at
+ *                  j, then -1 (also used as scratch during the call)
+ *   out_n_accepted [B] int32: j, the number of accepted draft tokens
+ *   stream         cudaStream_t (NULL = legacy default stream)
+ */
+SV_API sv_status_t spec_verify(const void* target_logits, const void* draft_logits,
+                        const int32_t* draft_tokens, const float* uniforms, int B, int k,
+                        int V, const float* temperature, int top_k, int mode,
+                        int32_t* out_tokens, int32_t* out_n_accepted, void* stream);
+
+/*
+ * spec_verify_ex — spec_verify plus optional outputs and options.
+ *   out_p, out_q  [B][k] fp32 or NULL: p_i(d_i) and q_i(d_i) at EVERY
+ *                 position (also past the first rejection); stochastic mode
+ *   out_status    1 int32 or NULL: SV_OK, or SV_ERR_DEVICE_TIMEOUT if a
+ *                 device wait ran out (written by the call's kernels)
+ *   opts          NULL or options (see sv_options_t)
+ */
+SV_API sv_status_t spec_verify_ex(const void* target_logits, const void* draft_logits,
+                           const int32_t* draft_tokens, const float* uniforms, int B, int k,
+                           int V, const float* temperature, int top_k, int mode,
+                           int32_t* out_tokens, int32_t* out_n_accepted, float* out_p,
+                           float* out_q, int32_t* out_status, const sv_options_t* opts,
+                           void* stream);
+
+/*
+ * spec_sample — the proposer's sampling step (section "提议与核验的基本步骤",
+ * paragraph 1: the proposer draws each candidate from its own
+ * distribution): one token per logit row, drawn with the same processing
+ * and inverse-CDF rule as the verification's bonus draw (stochastic), or
+ * the lowest-index argmax (greedy).
+ *   logits       [rows][V] bf16 or fp32
+ *   uniforms     [rows] fp32 in [0, 1); NULL in greedy mode
+ *   temperature  [rows] fp32 or NULL for 1.0
+ *   top_k, mode  as for spec_verify
+ *   out_tokens   [rows] int32; -1 for a row with a data error
+ */
+SV_API sv_status_t spec_sample(const void* logits, const float* uniforms, int rows, int V,
+                        const float* temperature, int top_k, int mode, int32_t* out_tokens,
+                        void* stream);
+
+/* spec_sample with options (opts may be NULL). */
+SV_API sv_status_t spec_sample_ex(const void* logits, const float* uniforms, int rows, int V,
+                           const float* temperature, int top_k, int mode, int32_t* out_tokens,
+                           const sv_options_t* opts, void* stream);
+
+/* Static description of a status code. */
+SV_API const char* spec_verify_status_string(sv_status_t status);
+
+/* Library version as MAJOR * 10000 + MINOR * 100 + PATCH. */
+SV_API int spec_verify_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPEC_VERIFY_H */

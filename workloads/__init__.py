@@ -286,11 +286,13 @@ def _rows_f64(w: Workload, seed: int, B: int, k: int, V: int, chunk_rows: int = 
 
 def make_case(name: str, seed: int = 0, B: Optional[int] = None, k: Optional[int] = None,
               V: Optional[int] = None, top_k: Optional[int] = None,
-              temperature: Optional[tuple] = None) -> Case:
+              temperature: Optional[tuple] = None, dtype: Optional[str] = None) -> Case:
     """Build the inputs of workload ``name``; ``B``/``k``/``V``/``top_k`` /
-    ``temperature`` override the workload's own sizes (for reduced test
-    cases of the same value model)."""
+    ``temperature`` / ``dtype`` override the workload's own settings (for
+    reduced or edge-shape test cases of the same value model)."""
     w = WORKLOADS[name]
+    if dtype is not None:
+        w = dataclasses.replace(w, dtype=dtype)
     B = w.B if B is None else B
     k = w.k if k is None else k
     V = w.V if V is None else V
