@@ -35,7 +35,7 @@ L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
 PROFILE_DIR = os.path.join(ROOT, "profiles")
 KERNEL_SOURCES = [os.path.join(ROOT, "draft_token_verification_verify_b200", "csrc", f)
-                  for f in ("sv_kernels.cuh", "sv_ptx.cuh", "spec_verify.cu")]
+                  for f in ("sv_common.cuh", "sv_rows.cuh", "sv_seq.cuh", "sv_ptx.cuh", "spec_verify.cu")]
 
 DESCR = {
     "tiny": "tiny stochastic verify B=1 k=4 V=32 fp32 T=1",
@@ -72,7 +72,7 @@ def kernel_source_hash() -> str:
 def profiled_traffic(workload: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken
     on the current kernel source (else None)."""
-    path = os.path.join(PROFILE_DIR, f"sv_unit_kernel_{workload}.md")
+    path = os.path.join(PROFILE_DIR, f"sv_rows_kernel_{workload}.md")
     if not os.path.exists(path):
         return None
     vals = {}
@@ -262,11 +262,14 @@ def run_ours(args):
     out_n = torch.empty((B,), dtype=torch.int32, device=dev)
     status = torch.zeros((1,), dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream()
+    wbytes = sv.spec_verify_workspace_size(B, k, V, case.top_k, mode)
+    wsp = torch.empty((max(wbytes, 1),), dtype=torch.uint8, device=dev)
 
     def step(i, ev0=None, ev1=None):
         opts = sv.make_options(event_start=ev0, event_stop=ev1) if ev0 is not None else None
         st = sv.spec_verify_ex(targets[i % nsets], drafts_l[i % nsets], drafts, unif, B, k, V, temp,
-                               case.top_k, mode, out_tok, out_n, None, None, status, opts, stream)
+                               case.top_k, mode, out_tok, out_n, None, None, status, wsp, wbytes, opts,
+                               stream)
         if st != sv.SV_OK:
             raise sv.SpecVerifyError(st, "spec_verify_ex")
 
@@ -398,7 +401,7 @@ def run_ours(args):
         "logit_bytes_per_step": logit_bytes,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
-                     "kernel": "sv_unit_kernel", "kernel_ms_mean": kmean,
+                     "kernel": "sv_rows_kernel", "kernel_ms_mean": kmean,
                      "kernel_ms_median": statistics.median(kern_ms)},
         "gpu_launches": 2 * args.steps,
         "clocks": clocks,

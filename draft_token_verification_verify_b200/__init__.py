@@ -33,7 +33,8 @@ LIB_PATH = _build.LIB
 __all__ = [
     "SV_OK", "SV_ERR_INVALID_ARG", "SV_ERR_UNSUPPORTED", "SV_ERR_CUDA", "SV_ERR_DEVICE_TIMEOUT",
     "SV_MODE_STOCHASTIC", "SV_MODE_GREEDY", "SV_DTYPE_BF16", "SV_DTYPE_F32", "SvOptions",
-    "SpecVerifyError", "lib", "spec_verify", "spec_verify_ex", "spec_sample", "spec_sample_ex",
+    "SpecVerifyError", "lib", "spec_verify", "spec_verify_ex", "spec_verify_workspace_size",
+    "spec_sample", "spec_sample_ex", "spec_sample_workspace_size", "make_options",
     "spec_verify_status_string", "spec_verify_version", "verify", "sample",
 ]
 
@@ -41,7 +42,7 @@ __all__ = [
 class SvOptions(ctypes.Structure):
     """Mirror of ``sv_options_t``."""
     _fields_ = [
-        ("cluster_size", ctypes.c_int),
+        ("chunks_per_row", ctypes.c_int),
         ("threads", ctypes.c_int),
         ("topk_path", ctypes.c_int),
         ("event_start", ctypes.c_void_p),
@@ -70,13 +71,18 @@ def lib() -> ctypes.CDLL:
         P, I = ctypes.c_void_p, ctypes.c_int
         L.spec_verify.argtypes = [P, P, P, P, I, I, I, P, I, I, P, P, P]
         L.spec_verify.restype = I
-        L.spec_verify_ex.argtypes = [P, P, P, P, I, I, I, P, I, I, P, P, P, P, P,
-                                     ctypes.POINTER(SvOptions), P]
+        Z = ctypes.c_size_t
+        OP = ctypes.POINTER(SvOptions)
+        L.spec_verify_ex.argtypes = [P, P, P, P, I, I, I, P, I, I, P, P, P, P, P, P, Z, OP, P]
         L.spec_verify_ex.restype = I
+        L.spec_verify_workspace_size.argtypes = [I, I, I, I, I, OP]
+        L.spec_verify_workspace_size.restype = Z
         L.spec_sample.argtypes = [P, P, I, I, P, I, I, P, P]
         L.spec_sample.restype = I
-        L.spec_sample_ex.argtypes = [P, P, I, I, P, I, I, P, ctypes.POINTER(SvOptions), P]
+        L.spec_sample_ex.argtypes = [P, P, I, I, P, I, I, P, P, Z, OP, P]
         L.spec_sample_ex.restype = I
+        L.spec_sample_workspace_size.argtypes = [I, I, I, I, OP]
+        L.spec_sample_workspace_size.restype = Z
         L.spec_verify_status_string.argtypes = [I]
         L.spec_verify_status_string.restype = ctypes.c_char_p
         L.spec_verify_version.argtypes = []
@@ -132,11 +138,21 @@ def spec_verify(target_logits, draft_logits, draft_tokens, uniforms, B, k, V, te
 
 def spec_verify_ex(target_logits, draft_logits, draft_tokens, uniforms, B, k, V, temperature, top_k,
                    mode, out_tokens, out_n_accepted, out_p=None, out_q=None, out_status=None,
-                   opts: Optional[SvOptions] = None, stream=None) -> int:
+                   workspace=None, workspace_bytes=0, opts: Optional[SvOptions] = None,
+                   stream=None) -> int:
     return lib().spec_verify_ex(_p(target_logits), _p(draft_logits), _p(draft_tokens), _p(uniforms),
                                 int(B), int(k), int(V), _p(temperature), int(top_k), int(mode),
                                 _p(out_tokens), _p(out_n_accepted), _p(out_p), _p(out_q),
-                                _p(out_status), _opts(opts), _stream(stream))
+                                _p(out_status), _p(workspace), int(workspace_bytes), _opts(opts),
+                                _stream(stream))
+
+
+def spec_verify_workspace_size(B, k, V, top_k, mode, opts: Optional[SvOptions] = None) -> int:
+    return lib().spec_verify_workspace_size(int(B), int(k), int(V), int(top_k), int(mode), _opts(opts))
+
+
+def spec_sample_workspace_size(rows, V, top_k, mode, opts: Optional[SvOptions] = None) -> int:
+    return lib().spec_sample_workspace_size(int(rows), int(V), int(top_k), int(mode), _opts(opts))
 
 
 def spec_sample(logits, uniforms, rows, V, temperature, top_k, mode, out_tokens, stream=None) -> int:
@@ -144,15 +160,16 @@ def spec_sample(logits, uniforms, rows, V, temperature, top_k, mode, out_tokens,
                              int(mode), _p(out_tokens), _stream(stream))
 
 
-def spec_sample_ex(logits, uniforms, rows, V, temperature, top_k, mode, out_tokens,
-                   opts: Optional[SvOptions] = None, stream=None) -> int:
+def spec_sample_ex(logits, uniforms, rows, V, temperature, top_k, mode, out_tokens, workspace=None,
+                   workspace_bytes=0, opts: Optional[SvOptions] = None, stream=None) -> int:
     return lib().spec_sample_ex(_p(logits), _p(uniforms), int(rows), int(V), _p(temperature),
-                                int(top_k), int(mode), _p(out_tokens), _opts(opts), _stream(stream))
+                                int(top_k), int(mode), _p(out_tokens), _p(workspace),
+                                int(workspace_bytes), _opts(opts), _stream(stream))
 
 
-def make_options(cluster_size=0, threads=0, topk_path=0, event_start=None, event_stop=None,
+def make_options(chunks_per_row=0, threads=0, topk_path=0, event_start=None, event_stop=None,
                  wait_timeout_ns=0, test_extra_tx=0) -> SvOptions:
-    return SvOptions(cluster_size, threads, topk_path, _event(event_start), _event(event_stop),
+    return SvOptions(chunks_per_row, threads, topk_path, _event(event_start), _event(event_stop),
                      wait_timeout_ns, test_extra_tx)
 
 
@@ -168,12 +185,13 @@ def _dtype_code(t) -> int:
 
 def verify(target, draft, draft_tokens, uniforms=None, temperature=None, top_k: int = 0,
            greedy: bool = False, out_tokens=None, out_n_accepted=None, out_p=None, out_q=None,
-           out_status=None, opts: Optional[SvOptions] = None, stream=None):
+           out_status=None, workspace=None, opts: Optional[SvOptions] = None, stream=None):
     """Tensor convenience wrapper around ``spec_verify_ex``.
 
     target [B, k+1, V], draft [B, k, V] (bf16 or fp32, contiguous, on the
     GPU), draft_tokens [B, k] int32, uniforms [B, k+1] fp32, temperature [B]
-    fp32 or None.  Output tensors are allocated with torch when not given.
+    fp32 or None.  Output tensors are allocated with torch when not given; the
+    workspace (a uint8 tensor) is taken from the library pool when None.
     Returns (out_tokens [B, k+1], out_n_accepted [B]).
     """
     import torch
@@ -186,8 +204,10 @@ def verify(target, draft, draft_tokens, uniforms=None, temperature=None, top_k: 
     if out_n_accepted is None:
         out_n_accepted = torch.empty((B,), dtype=torch.int32, device=dev)
     mode = (SV_MODE_GREEDY if greedy else SV_MODE_STOCHASTIC) | _dtype_code(target)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = spec_verify_ex(target, draft, draft_tokens, uniforms, B, k, V, temperature, top_k, mode,
-                        out_tokens, out_n_accepted, out_p, out_q, out_status, opts, stream)
+                        out_tokens, out_n_accepted, out_p, out_q, out_status, workspace, wbytes, opts,
+                        stream)
     if st != SV_OK:
         raise SpecVerifyError(st, "spec_verify_ex")
     return out_tokens, out_n_accepted
@@ -203,7 +223,8 @@ def sample(logits, uniforms=None, temperature=None, top_k: int = 0, greedy: bool
     if out_tokens is None:
         out_tokens = torch.empty(logits.shape[:-1], dtype=torch.int32, device=logits.device)
     mode = (SV_MODE_GREEDY if greedy else SV_MODE_STOCHASTIC) | _dtype_code(logits)
-    st = spec_sample_ex(logits, uniforms, rows, V, temperature, top_k, mode, out_tokens, opts, stream)
+    st = spec_sample_ex(logits, uniforms, rows, V, temperature, top_k, mode, out_tokens, None, 0, opts,
+                        stream)
     if st != SV_OK:
         raise SpecVerifyError(st, "spec_sample_ex")
     return out_tokens

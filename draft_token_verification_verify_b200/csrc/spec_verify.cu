@@ -1,32 +1,40 @@
-// Host side of the spec_verify C ABI: argument checks, launch planning and
-// the launches themselves.  Nothing here allocates device memory or
+// Host side of the spec_verify C ABI: argument checks, launch planning,
+// workspace handling and the two launches (the streaming pass, then the
+// per-sequence kernel as a programmatic dependent launch).  Nothing here
 // synchronises the caller's stream.
 #include <cuda_runtime.h>
 
-#include <atomic>
 #include <climits>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
 
 #include "../../include/spec_verify.h"
-#include "sv_kernels.cuh"
+#include "sv_rows.cuh"
+#include "sv_seq.cuh"
 
 namespace {
 
-constexpr int kVersion = 10000;  // 1.0.0
+constexpr int kVersion = 20000;  // 2.0.0
 constexpr int kMaxDevices = 64;
 constexpr uint64_t kDefaultTimeoutNs = 1000000000ull;
+constexpr int kSegBytes = sv::TILE_BYTES;  // bytes per segment (one ring stage)
+constexpr int kStages = 2;                 // ring stages of the streaming kernel
+constexpr int kTopkMax = 256;         // largest K on the kept-list path (<= threads)
+constexpr int kListCap = 1024;        // shared candidate list of a streaming CTA
 
 struct DeviceInfo {
     int ok = 0;
     int sms = 0;
     int smem_optin = 0;
+    int smem_per_sm = 0;
+    cudaMemPool_t pool = nullptr;
 };
 
 DeviceInfo g_dev[kMaxDevices];
 std::once_flag g_dev_once[kMaxDevices];
-std::once_flag g_attr_once[kMaxDevices][6];
+std::once_flag g_pool_once[kMaxDevices];
+std::once_flag g_attr_once[kMaxDevices][26];
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -41,7 +49,8 @@ const DeviceInfo* device_info(int* dev_out) {
         int major = 0;
         if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+            cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.smem_per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) !=
                 cudaSuccess) {
             cudaGetLastError();
             d.ok = 0;
@@ -53,145 +62,320 @@ const DeviceInfo* device_info(int* dev_out) {
     return g_dev[dev].ok ? &g_dev[dev] : nullptr;
 }
 
-using KernelFn = void (*)(sv::Params);
-
-KernelFn pick_kernel(int dt, int nt, int* slot) {
-    if (dt == 0) {
-        if (nt == 128) { *slot = 0; return sv::sv_unit_kernel<0, 128>; }
-        if (nt == 512) { *slot = 2; return sv::sv_unit_kernel<0, 512>; }
-        *slot = 1;
-        return sv::sv_unit_kernel<0, 256>;
-    }
-    if (nt == 128) { *slot = 3; return sv::sv_unit_kernel<1, 128>; }
-    if (nt == 512) { *slot = 5; return sv::sv_unit_kernel<1, 512>; }
-    *slot = 4;
-    return sv::sv_unit_kernel<1, 256>;
+// The library's own stream-ordered pool of one device: memory released with
+// cudaFreeAsync is kept for the next call instead of being unmapped.
+cudaMemPool_t device_pool(int dev) {
+    std::call_once(g_pool_once[dev], [dev] {
+        cudaMemPoolProps props;
+        std::memset(&props, 0, sizeof props);
+        props.allocType = cudaMemAllocationTypePinned;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = dev;
+        cudaMemPool_t pool = nullptr;
+        if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) {
+            cudaGetLastError();
+            return;
+        }
+        uint64_t keep = UINT64_MAX;
+        cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+        cudaGetLastError();
+        g_dev[dev].pool = pool;
+    });
+    return g_dev[dev].pool;
 }
 
+long long ceil_div(long long a, long long b) { return (a + b - 1) / b; }
+long long round_up(long long a, long long b) { return ceil_div(a, b) * b; }
+
 struct Plan {
-    int C = 1, NT = 256, L = 0, piece_bytes = 0, buf_bytes = 0, group_lanes = 32, use_cand = 0;
-    size_t smem = 0;
+    int mode = 0, elt = 2, seg = 0, nseg = 0, nch = 1, spc = 1, nt1 = 256, stages = kStages;
+    int stage_bytes = 0, lcap = 0, kcap = 0, mg = 0;
+    long long R = 0, tasks = 0;
+    size_t smem1 = 0, smem2 = 0;
+    size_t off_chunks = 0, off_cands = 0, ws_bytes = 0;
 };
 
-int ceil_div(long long a, long long b) { return static_cast<int>((a + b - 1) / b); }
-int round_up(long long a, long long b) { return static_cast<int>((a + b - 1) / b * b); }
-
-// Choose cluster size, slice length and shared-memory layout for a launch of
-// `units` units of `rows_per_unit` rows of V elements.
-sv_status_t make_plan(const DeviceInfo& dev, long long units, int rows_per_unit, int V, int elt,
-                      int top_k, const sv_options_t* opts, Plan* out) {
+// Plan the launches for `seqs` sequences of draft length k (rows = k+1 target
+// rows per sequence, plus k draft rows when stochastic).
+sv_status_t make_plan(const DeviceInfo& dev, long long seqs, int k, int V, int dt, bool greedy, int top_k,
+                      const sv_options_t* opts, Plan* out) {
     Plan p;
-    const int vec = 16 / elt;
-    p.NT = (opts && opts->threads) ? opts->threads : 256;
-    const long long unit_bytes = static_cast<long long>(rows_per_unit) * V * elt;
-    const int smem_budget = dev.smem_optin - sv::CTL_BYTES - 256;
-    int C;
-    if (opts && opts->cluster_size) {
-        C = opts->cluster_size;
-    } else {
-        // about 40 KB of logits per CTA, more CTAs for small batches
-        C = 1;
-        while (C < 16 && unit_bytes > static_cast<long long>(C) * 40 * 1024) C *= 2;
-        while (C < 16 && units * C < 2LL * dev.sms) C *= 2;
-        // no CTA should get an empty slice
-        while (C > 1 && static_cast<long long>(C - 1) * round_up(ceil_div(V, C), vec) >= V) C /= 2;
-    }
-    for (;;) {
-        p.C = C;
-        p.L = round_up(ceil_div(V, C), vec);
-        p.buf_bytes = round_up(static_cast<long long>(p.L) * elt + 32, 128);
-        if (static_cast<long long>(p.buf_bytes) * rows_per_unit <= smem_budget) break;
-        if (opts && opts->cluster_size) return SV_ERR_UNSUPPORTED;
-        if (C >= 16) return SV_ERR_UNSUPPORTED;
-        C *= 2;
-    }
-    p.piece_bytes = round_up(ceil_div(p.buf_bytes, sv::MAX_PIECES), 16);
-    if (p.piece_bytes < 8192) p.piece_bytes = 8192;
-    p.smem = static_cast<size_t>(sv::CTL_BYTES) + static_cast<size_t>(p.buf_bytes) * rows_per_unit;
-    // top-k lower bound groups: enough groups for a tight bound, within GMAX
-    p.use_cand = 0;
-    p.group_lanes = 32;
-    if (top_k > 0 && !(opts && opts->topk_path == 2)) {
-        int best = 0;
-        for (int g = 32; g >= 1; g >>= 1) {
-            const long long Gt = static_cast<long long>(C) * (p.NT / g);
-            if (Gt > sv::GMAX) break;
-            if (Gt >= top_k) {
-                best = g;
-                if (Gt >= 2LL * top_k) break;
+    p.elt = dt ? 4 : 2;
+    const int vec = 16 / p.elt;
+    p.nt1 = (opts && opts->threads) ? opts->threads : 128;
+    p.seg = kSegBytes / p.elt;
+    p.nseg = static_cast<int>(ceil_div(V, p.seg));
+    p.R = seqs * (k + 1) + (greedy ? 0 : seqs * k);
+    const bool radix = opts && opts->topk_path == 2;
+    if (greedy)
+        p.mode = sv::MODE_GREEDY;
+    else if (top_k == 0)
+        p.mode = sv::MODE_SOFTMAX;
+    else if (top_k <= kTopkMax && !radix)
+        p.mode = sv::MODE_TOPK;
+    else
+        p.mode = sv::MODE_MAXONLY;
+    if (opts && opts->topk_path == 1 && top_k > 0 && p.mode != sv::MODE_TOPK) return SV_ERR_UNSUPPORTED;
+    p.stage_bytes = static_cast<int>(round_up(kSegBytes + 32, 128));
+    if (p.mode == sv::MODE_TOPK) {
+        // the running bound needs K <= threads (each warp contributes <= 32 ranks)
+        if (top_k > p.nt1) {
+            if (opts && opts->threads) {
+                if (opts->topk_path == 1) return SV_ERR_UNSUPPORTED;
+                p.mode = sv::MODE_MAXONLY;
+            } else {
+                p.nt1 = 256;
             }
         }
-        if (best && top_k <= sv::CAND_CAP / 2) {
-            p.group_lanes = best;
-            p.use_cand = 1;
-        }
+        if (p.mode == sv::MODE_TOPK) p.lcap = kListCap;
     }
-    if (opts && opts->topk_path == 1 && top_k > 0 && !p.use_cand) return SV_ERR_UNSUPPORTED;
-    if (static_cast<long long>(p.buf_bytes) / 16 > static_cast<long long>(sv::MAX_TILES) * p.NT)
+    p.smem1 = static_cast<size_t>(sv::ROWS_CTL_BYTES) + static_cast<size_t>(p.stages) * p.stage_bytes +
+              static_cast<size_t>(3) * sv::MAX_TILES_K1 * (p.nt1 / 32) * 4;
+    if (p.mode == sv::MODE_TOPK) p.smem1 += static_cast<size_t>(p.lcap) * 8;
+    // chunks per row: one when there are enough rows to fill the device
+    const long long per_sm_smem = dev.smem_per_sm > 0 ? dev.smem_per_sm : 233472;
+    long long occ = per_sm_smem / static_cast<long long>(p.smem1 + 1024);
+    if (occ > 2048 / p.nt1) occ = 2048 / p.nt1;
+    if (occ < 1) occ = 1;
+    const long long slots = occ * dev.sms;
+    int nch;
+    if (opts && opts->chunks_per_row) {
+        nch = opts->chunks_per_row;
+    } else if (p.R * 2 >= slots) {
+        nch = 1;
+    } else {
+        nch = static_cast<int>(ceil_div(slots, p.R));
+    }
+    if (nch > p.nseg) nch = p.nseg;
+    if (nch < ceil_div(p.nseg, sv::MAX_TILES_K1)) nch = static_cast<int>(ceil_div(p.nseg, sv::MAX_TILES_K1));
+    if (nch < 1) nch = 1;
+    p.spc = static_cast<int>(ceil_div(p.nseg, nch));
+    p.nch = static_cast<int>(ceil_div(p.nseg, p.spc));
+    p.tasks = p.R * p.nch;
+    if (p.tasks > INT_MAX || seqs > INT_MAX) return SV_ERR_INVALID_ARG;
+    if (p.mode == sv::MODE_TOPK) {
+        int kc = 64;
+        while (kc < 2 * top_k) kc <<= 1;
+        p.kcap = kc > 1024 ? 1024 : kc;
+        p.mg = p.nch == 1 ? p.kcap : (4 * p.kcap > 1024 ? 1024 : 4 * p.kcap);
+    } else {
+        p.kcap = 0;
+        p.mg = 64;  // also holds the two draw lists of the top-k path
+    }
+    // workspace: segment partials, chunk headers, kept lists
+    const size_t segs = static_cast<size_t>(p.R) * p.nseg * sizeof(sv::SegRec);
+    p.off_chunks = round_up(segs, 256);
+    size_t chunks = 0, cands = 0;
+    if (p.mode == sv::MODE_TOPK) {
+        chunks = static_cast<size_t>(p.R) * p.nch * sizeof(sv::ChunkRec);
+        cands = static_cast<size_t>(p.R) * p.nch * p.kcap * sizeof(sv::Cand);
+    }
+    p.off_cands = round_up(p.off_chunks + chunks, 256);
+    p.ws_bytes = round_up(p.off_cands + cands, 256);
+    // per-sequence kernel: control, row stats, gather buffers, segment masses
+    const int nrows = greedy ? k + 1 : 2 * k + 1;
+    size_t head = static_cast<size_t>(nrows) * sizeof(sv::RowStat) + static_cast<size_t>(k + 1) * 8 + 8;
+    head = round_up(head, 128);
+    p.smem2 = sv::SEQ_CTL_BYTES + head + static_cast<size_t>(sv::SEQ_NW) * p.mg * sizeof(sv::Cand) +
+              static_cast<size_t>(p.nseg) * (sv::SEQ_NW + 1) * sizeof(float);
+    if (p.smem1 > static_cast<size_t>(dev.smem_optin) || p.smem2 > static_cast<size_t>(dev.smem_optin))
         return SV_ERR_UNSUPPORTED;
-    if (units > INT_MAX / C) return SV_ERR_INVALID_ARG;
+    (void)vec;
     *out = p;
     return SV_OK;
 }
 
-sv_status_t launch_units(const sv::Params& prm, const Plan& plan, int dt, int dev, cudaStream_t stream) {
-    int slot = 0;
-    KernelFn fn = pick_kernel(dt, plan.NT, &slot);
-    cudaError_t aerr = cudaSuccess;
-    std::call_once(g_attr_once[dev][slot], [&] {
-        aerr = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, g_dev[dev].smem_optin);
-        if (aerr == cudaSuccess)
-            aerr = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    });
-    if (aerr != cudaSuccess) {
-        cudaGetLastError();
-        return SV_ERR_CUDA;
+using RowsFn = void (*)(sv::RowsParams);
+using SeqFn = void (*)(sv::SeqParams);
+
+template <int DT, int NT>
+RowsFn rows_for_mode(int mode) {
+    switch (mode) {
+        case sv::MODE_GREEDY: return sv::sv_rows_kernel<DT, NT, sv::MODE_GREEDY>;
+        case sv::MODE_SOFTMAX: return sv::sv_rows_kernel<DT, NT, sv::MODE_SOFTMAX>;
+        case sv::MODE_TOPK: return sv::sv_rows_kernel<DT, NT, sv::MODE_TOPK>;
+        default: return sv::sv_rows_kernel<DT, NT, sv::MODE_MAXONLY>;
     }
-    const long long grid = (prm.sample_only ? prm.B : prm.B * (prm.k + 1)) * plan.C;
-    cudaLaunchConfig_t cfg;
-    std::memset(&cfg, 0, sizeof cfg);
-    cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
-    cfg.blockDim = dim3(plan.NT, 1, 1);
-    cfg.dynamicSmemBytes = plan.smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = plan.C;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, fn, prm) != cudaSuccess) {
+}
+
+// slot = dtype * 12 + threads-class * 4 + mode (24 instantiations)
+RowsFn pick_rows(int dt, int nt, int mode, int* slot) {
+    const int ntc = nt == 128 ? 0 : (nt == 512 ? 2 : 1);
+    *slot = dt * 12 + ntc * 4 + mode;
+    if (dt == 0) {
+        if (nt == 128) return rows_for_mode<0, 128>(mode);
+        if (nt == 512) return rows_for_mode<0, 512>(mode);
+        return rows_for_mode<0, 256>(mode);
+    }
+    if (nt == 128) return rows_for_mode<1, 128>(mode);
+    if (nt == 512) return rows_for_mode<1, 512>(mode);
+    return rows_for_mode<1, 256>(mode);
+}
+
+sv_status_t set_attrs(int dev, int dt, int nt, int mode) {
+    int slot = 0;
+    RowsFn f1 = pick_rows(dt, nt, mode, &slot);
+    SeqFn f2 = dt ? sv::sv_seq_kernel<1> : sv::sv_seq_kernel<0>;
+    cudaError_t e = cudaSuccess;
+    std::call_once(g_attr_once[dev][slot], [&] {
+        e = cudaFuncSetAttribute(f1, cudaFuncAttributeMaxDynamicSharedMemorySize, g_dev[dev].smem_optin);
+    });
+    std::call_once(g_attr_once[dev][24 + dt], [&] {
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(f2, cudaFuncAttributeMaxDynamicSharedMemorySize, g_dev[dev].smem_optin);
+    });
+    if (e != cudaSuccess) {
         cudaGetLastError();
         return SV_ERR_CUDA;
     }
     return SV_OK;
 }
 
-sv_status_t launch_finalize(int32_t* tokens, const int32_t* draft_tokens, int32_t* n_accepted,
-                            int32_t* status, long long B, int k, cudaStream_t stream) {
-    cudaLaunchConfig_t cfg;
-    std::memset(&cfg, 0, sizeof cfg);
-    cfg.gridDim = dim3(static_cast<unsigned>((B + 255) / 256), 1, 1);
-    cfg.blockDim = dim3(256, 1, 1);
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, sv::sv_finalize_kernel, tokens, draft_tokens, n_accepted, status, B, k) !=
-        cudaSuccess) {
-        cudaGetLastError();
-        return SV_ERR_CUDA;
+struct Call {
+    const void* target = nullptr;
+    const void* draft = nullptr;
+    const int32_t* draft_tokens = nullptr;
+    const float* uniforms = nullptr;
+    const float* temperature = nullptr;
+    long long seqs = 0;
+    int k = 0, V = 0, top_k = 0, dt = 0;
+    bool greedy = false, sample = false;
+    int32_t* out_tokens = nullptr;
+    int32_t* out_n = nullptr;
+    float* out_p = nullptr;
+    float* out_q = nullptr;
+    int32_t* out_status = nullptr;
+};
+
+sv_status_t run(const Call& cl, void* workspace, size_t workspace_bytes, const sv_options_t* opts,
+                cudaStream_t st) {
+    int dev = 0;
+    const DeviceInfo* info = device_info(&dev);
+    if (!info) return SV_ERR_UNSUPPORTED;
+    Plan p;
+    sv_status_t s = make_plan(*info, cl.seqs, cl.k, cl.V, cl.dt, cl.greedy, cl.top_k, opts, &p);
+    if (s != SV_OK) return s;
+    if (workspace && (workspace_bytes < p.ws_bytes || !aligned(workspace, 16))) return SV_ERR_INVALID_ARG;
+    if ((s = set_attrs(dev, cl.dt, p.nt1, p.mode)) != SV_OK) return s;
+
+    void* ws = workspace;
+    bool owned = false;
+    if (!ws) {
+        cudaMemPool_t pool = device_pool(dev);
+        if (!pool || cudaMallocFromPoolAsync(&ws, p.ws_bytes, pool, st) != cudaSuccess) {
+            cudaGetLastError();
+            return SV_ERR_CUDA;
+        }
+        owned = true;
     }
-    return SV_OK;
+    auto* base = static_cast<unsigned char*>(ws);
+
+    sv::RowsParams r;
+    std::memset(&r, 0, sizeof r);
+    r.target = cl.target;
+    r.draft = cl.draft;
+    r.draft_tokens = cl.draft_tokens;
+    r.B = cl.seqs;
+    r.k = cl.k;
+    r.V = cl.V;
+    r.mode = p.mode;
+    r.top_k = cl.top_k;
+    r.temperature = cl.temperature;
+    r.seg = p.seg;
+    r.nseg = p.nseg;
+    r.spc = p.spc;
+    r.nch = p.nch;
+    r.stages = p.stages;
+    r.stage_bytes = p.stage_bytes;
+    r.lcap = p.lcap;
+    r.kcap = p.kcap;
+    r.segs = reinterpret_cast<sv::SegRec*>(base);
+    r.chunks = reinterpret_cast<sv::ChunkRec*>(base + p.off_chunks);
+    r.cands = reinterpret_cast<sv::Cand*>(base + p.off_cands);
+    r.out_status = cl.sample ? nullptr : cl.out_status;
+    r.timeout_ns = (opts && opts->wait_timeout_ns) ? opts->wait_timeout_ns : kDefaultTimeoutNs;
+    r.test_extra_tx = opts ? opts->test_extra_tx : 0u;
+
+    sv::SeqParams q;
+    std::memset(&q, 0, sizeof q);
+    q.target = cl.target;
+    q.draft = cl.draft;
+    q.draft_tokens = cl.draft_tokens;
+    q.uniforms = cl.uniforms;
+    q.temperature = cl.temperature;
+    q.B = cl.seqs;
+    q.k = cl.k;
+    q.V = cl.V;
+    q.mode = p.mode;
+    q.top_k = cl.top_k;
+    q.sample_only = cl.sample ? 1 : 0;
+    q.seg = p.seg;
+    q.nseg = p.nseg;
+    q.spc = p.spc;
+    q.nch = p.nch;
+    q.kcap = p.kcap;
+    q.mg = p.mg;
+    q.segs = r.segs;
+    q.chunks = r.chunks;
+    q.cands = r.cands;
+    q.out_tokens = cl.out_tokens;
+    q.out_n = cl.out_n;
+    q.out_p = cl.out_p;
+    q.out_q = cl.out_q;
+    q.out_status = cl.sample ? nullptr : cl.out_status;
+
+    sv_status_t result = SV_OK;
+    do {
+        if (opts && opts->event_start &&
+            cudaEventRecord(static_cast<cudaEvent_t>(opts->event_start), st) != cudaSuccess) {
+            result = SV_ERR_CUDA;
+            break;
+        }
+        int slot = 0;
+        RowsFn f1 = pick_rows(cl.dt, p.nt1, p.mode, &slot);
+        cudaLaunchConfig_t c1;
+        std::memset(&c1, 0, sizeof c1);
+        c1.gridDim = dim3(static_cast<unsigned>(p.tasks), 1, 1);
+        c1.blockDim = dim3(p.nt1, 1, 1);
+        c1.dynamicSmemBytes = p.smem1;
+        c1.stream = st;
+        if (cudaLaunchKernelEx(&c1, f1, r) != cudaSuccess) {
+            result = SV_ERR_CUDA;
+            break;
+        }
+        if (opts && opts->event_stop &&
+            cudaEventRecord(static_cast<cudaEvent_t>(opts->event_stop), st) != cudaSuccess) {
+            result = SV_ERR_CUDA;
+            break;
+        }
+        cudaLaunchConfig_t c2;
+        std::memset(&c2, 0, sizeof c2);
+        c2.gridDim = dim3(static_cast<unsigned>(cl.seqs), 1, 1);
+        c2.blockDim = dim3(sv::SEQ_NT, 1, 1);
+        c2.dynamicSmemBytes = p.smem2;
+        c2.stream = st;
+        cudaLaunchAttribute a2[1];
+        a2[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        a2[0].val.programmaticStreamSerializationAllowed = 1;
+        c2.attrs = a2;
+        c2.numAttrs = 1;
+        SeqFn f2 = cl.dt ? sv::sv_seq_kernel<1> : sv::sv_seq_kernel<0>;
+        if (cudaLaunchKernelEx(&c2, f2, q) != cudaSuccess) {
+            result = SV_ERR_CUDA;
+            break;
+        }
+    } while (false);
+    if (result != SV_OK) cudaGetLastError();
+    if (owned && cudaFreeAsync(ws, st) != cudaSuccess) {
+        cudaGetLastError();
+        if (result == SV_OK) result = SV_ERR_CUDA;
+    }
+    return result;
 }
 
 sv_status_t check_options(const sv_options_t* o) {
     if (!o) return SV_OK;
-    const int c = o->cluster_size;
-    if (!(c == 0 || c == 1 || c == 2 || c == 4 || c == 8 || c == 16)) return SV_ERR_INVALID_ARG;
+    if (o->chunks_per_row < 0) return SV_ERR_INVALID_ARG;
     if (!(o->threads == 0 || o->threads == 128 || o->threads == 256 || o->threads == 512))
         return SV_ERR_INVALID_ARG;
     if (o->topk_path < 0 || o->topk_path > 2) return SV_ERR_INVALID_ARG;
@@ -207,6 +391,91 @@ bool decode_mode(int mode, bool* greedy, int* dt) {
     return true;
 }
 
+// Argument checks shared by the verify entry points; fills `cl`.
+sv_status_t verify_args(const void* target_logits, const void* draft_logits, const int32_t* draft_tokens,
+                        const float* uniforms, int B, int k, int V, const float* temperature, int top_k,
+                        int mode, int32_t* out_tokens, int32_t* out_n_accepted, float* out_p, float* out_q,
+                        int32_t* out_status, const sv_options_t* opts, bool check_ptrs, Call* cl) {
+    bool greedy = false;
+    int dt = 0;
+    if (B <= 0 || k < 1 || V < 1 || top_k < 0) return SV_ERR_INVALID_ARG;
+    if (!decode_mode(mode, &greedy, &dt)) return SV_ERR_INVALID_ARG;
+    if (check_options(opts) != SV_OK) return SV_ERR_INVALID_ARG;
+    const int elt = dt ? 4 : 2;
+    if (static_cast<unsigned long long>(B) * static_cast<unsigned long long>(2 * k + 1) >
+        (1ULL << 62) / (static_cast<unsigned long long>(V) * 4ULL))
+        return SV_ERR_INVALID_ARG;
+    if (check_ptrs) {
+        if (!target_logits || !draft_tokens || !out_tokens || !out_n_accepted) return SV_ERR_INVALID_ARG;
+        if (!greedy && (!draft_logits || !uniforms)) return SV_ERR_INVALID_ARG;
+        if (!aligned(target_logits, elt) || (draft_logits && !aligned(draft_logits, elt))) return SV_ERR_INVALID_ARG;
+        if (!aligned(draft_tokens, 4) || !aligned(out_tokens, 4) || !aligned(out_n_accepted, 4) ||
+            (uniforms && !aligned(uniforms, 4)) || (temperature && !aligned(temperature, 4)) ||
+            (out_p && !aligned(out_p, 4)) || (out_q && !aligned(out_q, 4)) ||
+            (out_status && !aligned(out_status, 4)))
+            return SV_ERR_INVALID_ARG;
+    }
+    cl->target = target_logits;
+    cl->draft = greedy ? nullptr : draft_logits;
+    cl->draft_tokens = draft_tokens;
+    cl->uniforms = greedy ? nullptr : uniforms;
+    cl->temperature = greedy ? nullptr : temperature;
+    cl->seqs = B;
+    cl->k = k;
+    cl->V = V;
+    cl->top_k = (top_k > 0 && top_k < V && !greedy) ? top_k : 0;
+    cl->dt = dt;
+    cl->greedy = greedy;
+    cl->sample = false;
+    cl->out_tokens = out_tokens;
+    cl->out_n = out_n_accepted;
+    cl->out_p = greedy ? nullptr : out_p;
+    cl->out_q = greedy ? nullptr : out_q;
+    cl->out_status = out_status;
+    return SV_OK;
+}
+
+sv_status_t sample_args(const void* logits, const float* uniforms, int rows, int V, const float* temperature,
+                        int top_k, int mode, int32_t* out_tokens, const sv_options_t* opts, bool check_ptrs,
+                        Call* cl) {
+    bool greedy = false;
+    int dt = 0;
+    if (rows <= 0 || V < 1 || top_k < 0) return SV_ERR_INVALID_ARG;
+    if (!decode_mode(mode, &greedy, &dt)) return SV_ERR_INVALID_ARG;
+    if (check_options(opts) != SV_OK) return SV_ERR_INVALID_ARG;
+    const int elt = dt ? 4 : 2;
+    if (static_cast<unsigned long long>(rows) > (1ULL << 62) / (static_cast<unsigned long long>(V) * 4ULL))
+        return SV_ERR_INVALID_ARG;
+    if (check_ptrs) {
+        if (!logits || !out_tokens) return SV_ERR_INVALID_ARG;
+        if (!greedy && !uniforms) return SV_ERR_INVALID_ARG;
+        if (!aligned(logits, elt) || !aligned(out_tokens, 4) || (uniforms && !aligned(uniforms, 4)) ||
+            (temperature && !aligned(temperature, 4)))
+            return SV_ERR_INVALID_ARG;
+    }
+    cl->target = logits;
+    cl->uniforms = greedy ? nullptr : uniforms;
+    cl->temperature = greedy ? nullptr : temperature;
+    cl->seqs = rows;
+    cl->k = 0;
+    cl->V = V;
+    cl->top_k = (top_k > 0 && top_k < V && !greedy) ? top_k : 0;
+    cl->dt = dt;
+    cl->greedy = greedy;
+    cl->sample = true;
+    cl->out_tokens = out_tokens;
+    return SV_OK;
+}
+
+size_t workspace_for(const Call& cl, const sv_options_t* opts) {
+    int dev = 0;
+    const DeviceInfo* info = device_info(&dev);
+    if (!info) return 0;
+    Plan p;
+    if (make_plan(*info, cl.seqs, cl.k, cl.V, cl.dt, cl.greedy, cl.top_k, opts, &p) != SV_OK) return 0;
+    return p.ws_bytes;
+}
+
 }  // namespace
 
 extern "C" {
@@ -214,147 +483,52 @@ extern "C" {
 sv_status_t spec_verify_ex(const void* target_logits, const void* draft_logits, const int32_t* draft_tokens,
                            const float* uniforms, int B, int k, int V, const float* temperature, int top_k,
                            int mode, int32_t* out_tokens, int32_t* out_n_accepted, float* out_p, float* out_q,
-                           int32_t* out_status, const sv_options_t* opts, void* stream) {
-    bool greedy = false;
-    int dt = 0;
-    if (B <= 0 || k < 1 || V < 1 || top_k < 0) return SV_ERR_INVALID_ARG;
-    if (!decode_mode(mode, &greedy, &dt)) return SV_ERR_INVALID_ARG;
-    if (check_options(opts) != SV_OK) return SV_ERR_INVALID_ARG;
-    const int elt = dt ? 4 : 2;
-    if (!target_logits || !draft_tokens || !out_tokens || !out_n_accepted) return SV_ERR_INVALID_ARG;
-    if (!greedy && (!draft_logits || !uniforms)) return SV_ERR_INVALID_ARG;
-    if (!aligned(target_logits, elt) || (draft_logits && !aligned(draft_logits, elt))) return SV_ERR_INVALID_ARG;
-    if (!aligned(draft_tokens, 4) || !aligned(out_tokens, 4) || !aligned(out_n_accepted, 4) ||
-        (uniforms && !aligned(uniforms, 4)) || (temperature && !aligned(temperature, 4)) ||
-        (out_p && !aligned(out_p, 4)) || (out_q && !aligned(out_q, 4)) ||
-        (out_status && !aligned(out_status, 4)))
-        return SV_ERR_INVALID_ARG;
-    // element counts must fit in 64-bit byte offsets
-    if (static_cast<unsigned long long>(B) * static_cast<unsigned long long>(k + 1) >
-        (1ULL << 62) / (static_cast<unsigned long long>(V) * 4ULL))
-        return SV_ERR_INVALID_ARG;
-    const int eff_topk = (top_k > 0 && top_k < V && !greedy) ? top_k : 0;
-
-    int dev = 0;
-    const DeviceInfo* info = device_info(&dev);
-    if (!info) return SV_ERR_UNSUPPORTED;
-    const long long units = static_cast<long long>(B) * (k + 1);
-    Plan plan;
-    const sv_status_t ps = make_plan(*info, units, greedy ? 1 : 2, V, elt, eff_topk, opts, &plan);
-    if (ps != SV_OK) return ps;
-
-    sv::Params prm;
-    std::memset(&prm, 0, sizeof prm);
-    prm.target = target_logits;
-    prm.draft = draft_logits;
-    prm.draft_tokens = draft_tokens;
-    prm.uniforms = uniforms;
-    prm.temperature = temperature;
-    prm.out_codes = out_tokens;
-    prm.out_p = greedy ? nullptr : out_p;
-    prm.out_q = greedy ? nullptr : out_q;
-    prm.out_status = out_status;
-    prm.B = B;
-    prm.k = k;
-    prm.V = V;
-    prm.top_k = eff_topk;
-    prm.greedy = greedy ? 1 : 0;
-    prm.sample_only = 0;
-    prm.C = plan.C;
-    prm.L = plan.L;
-    prm.piece_bytes = plan.piece_bytes;
-    prm.buf_bytes = plan.buf_bytes;
-    prm.group_lanes = plan.group_lanes;
-    prm.use_cand = plan.use_cand;
-    prm.timeout_ns = (opts && opts->wait_timeout_ns) ? opts->wait_timeout_ns : kDefaultTimeoutNs;
-    prm.test_extra_tx = opts ? opts->test_extra_tx : 0u;
-
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (opts && opts->event_start &&
-        cudaEventRecord(static_cast<cudaEvent_t>(opts->event_start), st) != cudaSuccess) {
-        cudaGetLastError();
-        return SV_ERR_CUDA;
-    }
-    sv_status_t s = launch_units(prm, plan, dt, dev, st);
+                           int32_t* out_status, void* workspace, size_t workspace_bytes,
+                           const sv_options_t* opts, void* stream) {
+    Call cl;
+    const sv_status_t s = verify_args(target_logits, draft_logits, draft_tokens, uniforms, B, k, V, temperature,
+                                      top_k, mode, out_tokens, out_n_accepted, out_p, out_q, out_status, opts,
+                                      true, &cl);
     if (s != SV_OK) return s;
-    if (opts && opts->event_stop &&
-        cudaEventRecord(static_cast<cudaEvent_t>(opts->event_stop), st) != cudaSuccess) {
-        cudaGetLastError();
-        return SV_ERR_CUDA;
-    }
-    return launch_finalize(out_tokens, draft_tokens, out_n_accepted, out_status, B, k, st);
+    return run(cl, workspace, workspace_bytes, opts, static_cast<cudaStream_t>(stream));
 }
 
 sv_status_t spec_verify(const void* target_logits, const void* draft_logits, const int32_t* draft_tokens,
                         const float* uniforms, int B, int k, int V, const float* temperature, int top_k,
                         int mode, int32_t* out_tokens, int32_t* out_n_accepted, void* stream) {
     return spec_verify_ex(target_logits, draft_logits, draft_tokens, uniforms, B, k, V, temperature, top_k,
-                          mode, out_tokens, out_n_accepted, nullptr, nullptr, nullptr, nullptr, stream);
+                          mode, out_tokens, out_n_accepted, nullptr, nullptr, nullptr, nullptr, 0, nullptr,
+                          stream);
+}
+
+size_t spec_verify_workspace_size(int B, int k, int V, int top_k, int mode, const sv_options_t* opts) {
+    Call cl;
+    if (verify_args(nullptr, nullptr, nullptr, nullptr, B, k, V, nullptr, top_k, mode, nullptr, nullptr,
+                    nullptr, nullptr, nullptr, opts, false, &cl) != SV_OK)
+        return 0;
+    return workspace_for(cl, opts);
 }
 
 sv_status_t spec_sample_ex(const void* logits, const float* uniforms, int rows, int V, const float* temperature,
-                           int top_k, int mode, int32_t* out_tokens, const sv_options_t* opts, void* stream) {
-    bool greedy = false;
-    int dt = 0;
-    if (rows <= 0 || V < 1 || top_k < 0) return SV_ERR_INVALID_ARG;
-    if (!decode_mode(mode, &greedy, &dt)) return SV_ERR_INVALID_ARG;
-    if (check_options(opts) != SV_OK) return SV_ERR_INVALID_ARG;
-    const int elt = dt ? 4 : 2;
-    if (!logits || !out_tokens) return SV_ERR_INVALID_ARG;
-    if (!greedy && !uniforms) return SV_ERR_INVALID_ARG;
-    if (!aligned(logits, elt) || !aligned(out_tokens, 4) || (uniforms && !aligned(uniforms, 4)) ||
-        (temperature && !aligned(temperature, 4)))
-        return SV_ERR_INVALID_ARG;
-    if (static_cast<unsigned long long>(rows) > (1ULL << 62) / (static_cast<unsigned long long>(V) * 4ULL))
-        return SV_ERR_INVALID_ARG;
-    const int eff_topk = (top_k > 0 && top_k < V && !greedy) ? top_k : 0;
-
-    int dev = 0;
-    const DeviceInfo* info = device_info(&dev);
-    if (!info) return SV_ERR_UNSUPPORTED;
-    Plan plan;
-    const sv_status_t ps = make_plan(*info, rows, 1, V, elt, eff_topk, opts, &plan);
-    if (ps != SV_OK) return ps;
-
-    sv::Params prm;
-    std::memset(&prm, 0, sizeof prm);
-    prm.target = logits;
-    prm.uniforms = uniforms;
-    prm.temperature = temperature;
-    prm.out_codes = out_tokens;
-    prm.B = rows;
-    prm.k = 0;
-    prm.V = V;
-    prm.top_k = eff_topk;
-    prm.greedy = greedy ? 1 : 0;
-    prm.sample_only = 1;
-    prm.C = plan.C;
-    prm.L = plan.L;
-    prm.piece_bytes = plan.piece_bytes;
-    prm.buf_bytes = plan.buf_bytes;
-    prm.group_lanes = plan.group_lanes;
-    prm.use_cand = plan.use_cand;
-    prm.timeout_ns = (opts && opts->wait_timeout_ns) ? opts->wait_timeout_ns : kDefaultTimeoutNs;
-    prm.test_extra_tx = opts ? opts->test_extra_tx : 0u;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (opts && opts->event_start &&
-        cudaEventRecord(static_cast<cudaEvent_t>(opts->event_start), st) != cudaSuccess) {
-        cudaGetLastError();
-        return SV_ERR_CUDA;
-    }
-    sv_status_t s = launch_units(prm, plan, dt, dev, st);
+                           int top_k, int mode, int32_t* out_tokens, void* workspace, size_t workspace_bytes,
+                           const sv_options_t* opts, void* stream) {
+    Call cl;
+    const sv_status_t s =
+        sample_args(logits, uniforms, rows, V, temperature, top_k, mode, out_tokens, opts, true, &cl);
     if (s != SV_OK) return s;
-    if (opts && opts->event_stop &&
-        cudaEventRecord(static_cast<cudaEvent_t>(opts->event_stop), st) != cudaSuccess) {
-        cudaGetLastError();
-        return SV_ERR_CUDA;
-    }
-    return SV_OK;
+    return run(cl, workspace, workspace_bytes, opts, static_cast<cudaStream_t>(stream));
 }
 
 sv_status_t spec_sample(const void* logits, const float* uniforms, int rows, int V, const float* temperature,
                         int top_k, int mode, int32_t* out_tokens, void* stream) {
-    return spec_sample_ex(logits, uniforms, rows, V, temperature, top_k, mode, out_tokens, nullptr, stream);
+    return spec_sample_ex(logits, uniforms, rows, V, temperature, top_k, mode, out_tokens, nullptr, 0, nullptr,
+                          stream);
+}
+
+size_t spec_sample_workspace_size(int rows, int V, int top_k, int mode, const sv_options_t* opts) {
+    Call cl;
+    if (sample_args(nullptr, nullptr, rows, V, nullptr, top_k, mode, nullptr, opts, false, &cl) != SV_OK) return 0;
+    return workspace_for(cl, opts);
 }
 
 const char* spec_verify_status_string(sv_status_t status) {

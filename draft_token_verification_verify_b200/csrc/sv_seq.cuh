@@ -1,0 +1,670 @@
+// K2 — one CTA per sequence: merge the streaming partials of the sequence's
+// rows, take the acceptance decisions and draw the final token.
+//
+// Method (speculative decoding entry "推测解码", section "提议与核验的基本步骤"):
+// with p and q the processed target and draft distributions, position i
+// accepts d_i iff u_i * q_i(d_i) < p_i(d_i) (probability min(1, p/q)); the
+// first rejected position j is redrawn from max(0, p_j - q_j), normalised;
+// after k acceptances the bonus token is drawn from p_k; both draws take u_k
+// through the inverse CDF in index order.  Greedy mode compares d_i with the
+// lowest-index argmax of the target row.
+//
+// Draws: with top-k, from the kept lists gathered by the streaming pass (no
+// logit is read again); without top-k, the bonus draw locates its segment
+// from the streaming partials and rescans that segment only, while a
+// residual draw streams the rejected (target, draft) pair once to get
+// per-segment masses and rescans the segment that holds u * W.  Rows whose
+// kept list did not fit (massive ties) or top-k above the list capacity fall
+// back to an exact radix select over the row in global memory.
+#pragma once
+
+#include <climits>
+
+#include "sv_common.cuh"
+
+namespace sv {
+
+constexpr int SEQ_NT = 256;
+constexpr int SEQ_NW = SEQ_NT / 32;
+
+struct SeqParams {
+    const void* target;          // [B][k+1][V]
+    const void* draft;           // [B][k][V] or null
+    const int32_t* draft_tokens; // [B][k] or null (sampler)
+    const float* uniforms;       // [B][k+1] or null (greedy)
+    const float* temperature;    // [B] or null
+    long long B;
+    int k;
+    int V;
+    int mode;                    // MODE_* used by the streaming pass
+    int top_k;
+    int sample_only;             // proposer sampler: write one token per row
+    int seg, nseg, spc, nch, kcap;
+    int mg;                      // gather capacity per warp (power of two)
+    const SegRec* segs;
+    const ChunkRec* chunks;
+    const Cand* cands;
+    int32_t* out_tokens;         // [B][k+1] (sampler: [B])
+    int32_t* out_n;              // [B] or null (sampler)
+    float* out_p;                // [B][k] or null
+    float* out_q;                // [B][k] or null
+    int32_t* out_status;         // or null
+};
+
+struct RowStat {
+    float msc;   // maximum in log2 units (z*c)
+    float invS;  // 1 / normaliser
+    float tau;   // kept threshold (-inf: every finite logit)
+    float zd;    // logit at the draft token of the row's position (NaN if none)
+    int arg;     // greedy argmax
+    int err;     // 1 data error, 2 timeout
+    int slow;    // top-k threshold must be resolved by radix select
+    int pad;
+};
+
+struct __align__(16) SeqCtl {
+    float red_f[SEQ_NW][2];
+    int red_i[SEQ_NW];
+    int hist[256];
+    int j;
+    int err;
+    int token;
+    int tok_cross;
+    int tok_last;
+    int seg_sel;
+    int last_mode;
+    int retry;
+    int radix_digit;
+    int radix_k;
+    uint32_t radix_prefix;
+    float x;
+    float base;
+    float W;
+    float c;
+};
+
+constexpr int SEQ_CTL_BYTES = (int)((sizeof(SeqCtl) + 127) / 128 * 128);
+
+// vector q of a row: elements [q*VEC, q*VEC + VEC) clipped to [0, V)
+template <int DT>
+__device__ __forceinline__ void load_vec(const void* row, bool aligned, int q, int V, float* v) {
+    constexpr int VEC = VT<DT>::VEC;
+    const long long e = static_cast<long long>(q) * VEC;
+    if (aligned && e + VEC <= V) {
+        const uint4 raw = __ldg(reinterpret_cast<const uint4*>(row) + q);
+        unpack<DT>(raw, v);
+    } else {
+#pragma unroll
+        for (int t = 0; t < VEC; ++t) v[t] = (e + t < V) ? load_elem<DT>(row, e + t) : NEG_INF;
+    }
+}
+
+template <int DT>
+__global__ void __launch_bounds__(SEQ_NT, 2) sv_seq_kernel(const SeqParams P) {
+    constexpr int VEC = VT<DT>::VEC;
+    constexpr int ELT = VT<DT>::ELT;
+    constexpr int NT = SEQ_NT, NW = SEQ_NW;
+    extern __shared__ __align__(128) unsigned char smem[];
+    SeqCtl& S = *reinterpret_cast<SeqCtl*>(smem);
+    const int k = P.k, V = P.V;
+    const bool greedy = P.mode == MODE_GREEDY;
+    const int nrows = greedy || P.sample_only ? k + 1 : 2 * k + 1;
+    RowStat* rs = reinterpret_cast<RowStat*>(smem + SEQ_CTL_BYTES);
+    int* dtok = reinterpret_cast<int*>(rs + nrows);
+    float* uu = reinterpret_cast<float*>(dtok + (k > 0 ? k : 1));
+    Cand* gbuf = reinterpret_cast<Cand*>(
+        smem + SEQ_CTL_BYTES +
+        (((static_cast<size_t>(nrows) * sizeof(RowStat) + (k + 1) * 8 + 8) + 127) / 128 * 128));
+    float* part = reinterpret_cast<float*>(gbuf + static_cast<size_t>(NW) * P.mg);  // [nseg][NW]
+    float* mass = part + static_cast<size_t>(P.nseg) * NW;                            // [nseg]
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const long long b = blockIdx.x;
+    const long long Rt = P.B * (k + 1);
+    const int K = P.top_k;
+
+    // ---- inputs that do not depend on the streaming pass -----------------------
+    float T = 1.f;
+    if (!greedy && P.temperature) T = P.temperature[b];
+    const float c = (T > 0.f && T != POS_INF) ? LOG2E / T : 1.f;
+    for (int i = tid; i < k; i += NT) dtok[i] = P.draft_tokens[b * k + i];
+    if (!greedy)
+        for (int i = tid; i <= k; i += NT) uu[i] = P.uniforms[b * (k + 1) + i];
+    if (tid == 0) {
+        S.err = 0;
+        S.c = c;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        int bad = 0;
+        for (int i = 0; i < k; ++i)
+            if (dtok[i] < 0 || dtok[i] >= V) bad = 1;
+        if (!greedy) {
+            if (!(T > 0.f) || T == POS_INF) bad = 1;
+            for (int i = 0; i <= k; ++i)
+                if (!(uu[i] >= 0.f && uu[i] < 1.f)) bad = 1;
+        }
+        S.err = bad;
+    }
+    pdl_wait_primary();  // the streaming pass is complete from here on
+
+    auto row_ptr = [&](int rr) -> const void* {
+        if (rr <= k)
+            return static_cast<const char*>(P.target) + (static_cast<size_t>(b) * (k + 1) + rr) * static_cast<size_t>(V) * ELT;
+        return static_cast<const char*>(P.draft) + (static_cast<size_t>(b) * k + (rr - k - 1)) * static_cast<size_t>(V) * ELT;
+    };
+    auto row_index = [&](int rr) -> long long { return rr <= k ? b * (k + 1) + rr : Rt + b * k + (rr - k - 1); };
+    auto row_dtok = [&](int rr) -> int {
+        const int pos = rr <= k ? rr : rr - k - 1;
+        return pos < k ? dtok[pos] : -1;
+    };
+
+    // gather the entries >= thr of the row's chunk lists into dst (index order)
+    auto gather = [&](long long r, float thr, Cand* dst, int cap) -> int {
+        int base = 0;
+        for (int ch = 0; ch < P.nch; ++ch) {
+            const ChunkRec cr = P.chunks[r * P.nch + ch];
+            const Cand* src = P.cands + (r * P.nch + ch) * static_cast<long long>(P.kcap);
+            for (int e0 = 0; e0 < cr.n; e0 += 32) {
+                const int e = e0 + lane;
+                Cand cd = {NEG_INF, -1};
+                if (e < cr.n) cd = src[e];
+                const bool pred = e < cr.n && cd.v >= thr;
+                const unsigned m = __ballot_sync(0xffffffffu, pred);
+                const int pos = base + __popc(m & ((1u << lane) - 1u));
+                if (pred && pos < cap) dst[pos] = cd;
+                base += __popc(m);
+            }
+        }
+        return base;
+    };
+
+    // ---- phase 1: per-row statistics (one warp per row) ----------------------------
+    for (int rr = warp; rr < nrows; rr += NW) {
+        const long long r = row_index(rr);
+        const int d = row_dtok(rr);
+        RowStat st;
+        st.tau = NEG_INF;
+        st.zd = __int_as_float(0x7fc00000);
+        st.arg = -1;
+        st.err = 0;
+        st.slow = 0;
+        st.pad = 0;
+        st.invS = 0.f;
+        int tmo = 0;
+        if (greedy) {
+            float best = NEG_INF, mx = NEG_INF;
+            int bi = -1;
+            for (int s = lane; s < P.nch; s += 32) {  // one record per chunk
+                const SegRec g = P.segs[r * P.nseg + s];
+                tmo |= g.flags & REC_TIMEOUT;
+                mx = fmax_nan(mx, g.m);
+                if (arg_better(g.m, g.arg, best, bi)) {
+                    best = g.m;
+                    bi = g.arg;
+                }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const float ob = __shfl_xor_sync(0xffffffffu, best, o);
+                const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+                if (arg_better(ob, oi, best, bi)) {
+                    best = ob;
+                    bi = oi;
+                }
+                mx = fmax_nan(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            }
+            st.msc = mx;
+            st.arg = bi;
+            if (mx != mx || mx == POS_INF || bi < 0) st.err = 1;
+        } else if (P.mode == MODE_SOFTMAX) {
+            float m = NEG_INF, s = 0.f;
+            for (int q = lane; q < P.nseg; q += 32) {
+                const SegRec g = P.segs[r * P.nseg + q];
+                tmo |= g.flags & REC_TIMEOUT;
+                ms_combine(m, s, g.m, g.s);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+                ms_combine(m, s, __shfl_xor_sync(0xffffffffu, m, o), __shfl_xor_sync(0xffffffffu, s, o));
+            st.msc = m;
+            st.invS = 1.f / s;
+            if (m != m || m == POS_INF || m == NEG_INF || s != s) st.err = 1;
+            if (d >= 0 && d < V) st.zd = load_elem<DT>(row_ptr(rr), d);
+        } else {
+            // top-k: raw maximum over the chunks, then the kept set
+            float mx = NEG_INF;
+            for (int q = lane; q < P.nch; q += 32) {
+                if (P.mode == MODE_TOPK) {
+                    const ChunkRec g = P.chunks[r * P.nch + q];
+                    tmo |= g.flags & REC_TIMEOUT;
+                    mx = fmax_nan(mx, g.m);
+                } else {
+                    const SegRec g = P.segs[r * P.nseg + q];
+                    tmo |= g.flags & REC_TIMEOUT;
+                    mx = fmax_nan(mx, g.m);
+                }
+            }
+            mx = warp_max_nan(mx);
+            st.msc = mx * c;
+            if (mx != mx || mx == POS_INF || mx == NEG_INF) st.err = 1;
+            if (P.mode == MODE_MAXONLY) {
+                st.slow = 1;
+            } else if (!st.err) {
+                float G = NEG_INF;
+                int ovf = 0;
+                for (int ch = lane; ch < P.nch; ch += 32) {
+                    const ChunkRec cr = P.chunks[r * P.nch + ch];
+                    G = fmaxf(G, cr.tau);
+                    tmo |= cr.flags & REC_TIMEOUT;
+                    ovf |= cr.flags & REC_OVERFLOW;
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) G = fmaxf(G, __shfl_xor_sync(0xffffffffu, G, o));
+                ovf = __any_sync(0xffffffffu, ovf);
+                Cand* buf = gbuf + static_cast<size_t>(warp) * P.mg;
+                int ng = 0;
+                if (P.nch == 1 && !ovf) {
+                    // one chunk: its header already holds tau, the sum and the draft logit
+                    const ChunkRec cr = P.chunks[r];
+                    st.tau = cr.tau;
+                    st.invS = 1.f / cr.s;
+                    st.zd = cr.zd;
+                } else if (!ovf) {
+                    ng = gather(r, G, buf, P.mg);
+                }
+                if (P.nch == 1 && !ovf) {
+                    // done
+                } else if (ovf || ng > P.mg) {
+                    st.slow = 1;
+                } else {
+                    __syncwarp();
+                    float tau = G;
+                    if (P.nch > 1) {
+                        float cand = NEG_INF;
+                        for (int e = lane; e < ng; e += 32) {
+                            const float x = buf[e].v;
+                            int gt = 0, ge = 0;
+                            for (int q = 0; q < ng; ++q) {
+                                const float y = buf[q].v;
+                                gt += (y > x);
+                                ge += (y >= x);
+                            }
+                            if (gt < K && K <= ge) cand = x;
+                        }
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1) cand = fmaxf(cand, __shfl_xor_sync(0xffffffffu, cand, o));
+                        tau = cand;
+                    }
+                    float acc = 0.f, zd = NEG_INF;
+                    for (int e = lane; e < ng; e += 32) {
+                        const Cand cd = buf[e];
+                        if (cd.v >= tau) {
+                            acc += ex2(fmaf(cd.v, c, -st.msc));
+                            if (cd.i == d) zd = cd.v;
+                        }
+                    }
+                    acc = warp_sum(acc);
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) zd = fmaxf(zd, __shfl_xor_sync(0xffffffffu, zd, o));
+                    st.tau = tau;
+                    st.invS = 1.f / acc;
+                    st.zd = zd;  // -inf: the draft token is not kept (probability 0)
+                }
+            }
+        }
+        tmo = __any_sync(0xffffffffu, tmo);
+        if (tmo) st.err = 2;
+        if (lane == 0) rs[rr] = st;
+    }
+    __syncthreads();
+
+    // ---- phase 1b: exact top-k threshold of rows that need it (rare) --------------
+    if (!greedy && P.mode != MODE_SOFTMAX) {
+        for (int rr = 0; rr < nrows; ++rr) {
+            if (!rs[rr].slow || rs[rr].err) continue;  // uniform: read after a barrier
+            const void* row = row_ptr(rr);
+            constexpr int ROUNDS = (DT == 0) ? 2 : 4;
+            if (tid == 0) {
+                S.radix_prefix = 0u;
+                S.radix_k = K;
+            }
+            for (int round = 0; round < ROUNDS; ++round) {
+                const int shift = 24 - 8 * round;
+                for (int q = tid; q < 256; q += NT) S.hist[q] = 0;
+                __syncthreads();
+                const uint32_t pre = S.radix_prefix;
+                for (int e = tid; e < V; e += NT) {
+                    const uint32_t key = okey(load_elem<DT>(row, e));
+                    if (round == 0 || (key >> (shift + 8)) == pre) atomicAdd(&S.hist[(key >> shift) & 255u], 1);
+                }
+                __syncthreads();
+                if (tid == 0) {
+                    int kr = S.radix_k, cum = 0, digit = 0;
+                    for (int bin = 255; bin >= 0; --bin) {
+                        const int cnt = S.hist[bin];
+                        if (cum + cnt >= kr) {
+                            digit = bin;
+                            kr -= cum;
+                            break;
+                        }
+                        cum += cnt;
+                    }
+                    S.radix_prefix = (S.radix_prefix << 8) | static_cast<uint32_t>(digit);
+                    S.radix_k = kr;
+                }
+                __syncthreads();
+            }
+            float tau;
+            if constexpr (DT == 0)
+                tau = okey_inv(S.radix_prefix << 16 | ((S.radix_prefix & 0x8000u) ? 0u : 0xffffu));
+            else
+                tau = okey_inv(S.radix_prefix);
+            const float msc = rs[rr].msc;
+            float acc = 0.f;
+            for (int e = tid; e < V; e += NT) {
+                const float z = load_elem<DT>(row, e);
+                if (z >= tau) acc += ex2(fmaf(z, c, -msc));
+            }
+            acc = warp_sum(acc);
+            if (lane == 0) S.red_f[warp][0] = acc;
+            __syncthreads();
+            if (tid == 0) {
+                float s = 0.f;
+                for (int w = 0; w < NW; ++w) s += S.red_f[w][0];
+                rs[rr].tau = tau;
+                rs[rr].invS = 1.f / s;
+                const int d = row_dtok(rr);
+                rs[rr].zd = (d >= 0 && d < V) ? load_elem<DT>(row, d) : __int_as_float(0x7fc00000);
+            }
+            __syncthreads();
+        }
+    }
+
+    // ---- phase 2: decisions ----------------------------------------------------------
+    if (tid == 0) {
+        int err = S.err, tmo = 0;
+        for (int rr = 0; rr < nrows; ++rr) {
+            if (rs[rr].err) err = 1;
+            if (rs[rr].err == 2) tmo = 1;
+        }
+        int j = k;
+        if (!err) {
+            if (greedy) {
+                for (int i = 0; i < k; ++i)
+                    if (dtok[i] != rs[i].arg) {
+                        j = i;
+                        break;
+                    }
+                S.token = rs[j].arg;
+            } else {
+                bool found = false;
+                for (int i = 0; i < k; ++i) {
+                    const RowStat& t = rs[i];
+                    const RowStat& dd = rs[k + 1 + i];
+                    const float p = (t.zd >= t.tau) ? ex2(fmaf(t.zd, c, -t.msc)) * t.invS : 0.f;
+                    const float q = (dd.zd >= dd.tau) ? ex2(fmaf(dd.zd, c, -dd.msc)) * dd.invS : 0.f;
+                    if (P.out_p) P.out_p[b * k + i] = p;
+                    if (P.out_q) P.out_q[b * k + i] = q;
+                    if (!found && !(uu[i] * q < p)) {
+                        j = i;
+                        found = true;
+                    }
+                }
+            }
+        } else if (!greedy) {
+            for (int i = 0; i < k; ++i) {
+                if (P.out_p) P.out_p[b * k + i] = __int_as_float(0x7fc00000);
+                if (P.out_q) P.out_q[b * k + i] = __int_as_float(0x7fc00000);
+            }
+        }
+        if (tmo && P.out_status) atomicExch(P.out_status, -4);
+        S.err = err;
+        S.j = j;
+    }
+    __syncthreads();
+
+    // ---- phase 3: the draw -------------------------------------------------------------
+    if (!greedy && !S.err) {
+        const int j = S.j;
+        const RowStat tst = rs[j];
+        const bool use_q0 = j < k;
+        const RowStat dst = use_q0 ? rs[k + 1 + j] : tst;
+        const float u = uu[k];
+        const bool list_draw = P.mode == MODE_TOPK && !tst.slow && !(use_q0 && dst.slow);
+        if (list_draw) {
+            Cand* lt = gbuf;
+            Cand* ld = gbuf + P.mg;
+            int nt = 0, nd = 0;
+            if (warp == 0) nt = gather(row_index(j), tst.tau, lt, P.mg);
+            if (warp == 1 && use_q0) nd = gather(row_index(k + 1 + j), dst.tau, ld, P.mg);
+            if (warp == 1 && lane == 0) S.red_i[1] = nd;
+            __syncthreads();
+            nd = S.red_i[1];
+            if (warp == 0) {
+                auto find = [&](int v) {
+                    int a = 0, z = nd - 1;
+                    while (a <= z) {
+                        const int mid = (a + z) >> 1;
+                        const int x = ld[mid].i;
+                        if (x == v) return mid;
+                        if (x < v) a = mid + 1; else z = mid - 1;
+                    }
+                    return -1;
+                };
+                bool use_q = use_q0;
+                auto weight = [&](int e) {
+                    const float pt = ex2(fmaf(lt[e].v, c, -tst.msc)) * tst.invS;
+                    if (!use_q) return pt;
+                    const int pd = find(lt[e].i);
+                    const float q = pd >= 0 ? ex2(fmaf(ld[pd].v, c, -dst.msc)) * dst.invS : 0.f;
+                    return fmaxf(pt - q, 0.f);
+                };
+                float W = 0.f;
+                for (int attempt = 0; attempt < 2; ++attempt) {
+                    W = 0.f;
+                    for (int base = 0; base < nt; base += 32) {
+                        const float w = (base + lane < nt) ? weight(base + lane) : 0.f;
+                        const float incl = warp_incl_scan(w, lane);
+                        W += __shfl_sync(0xffffffffu, incl, 31);
+                    }
+                    if (W > 0.f || !use_q) break;
+                    use_q = false;  // zero residual mass: redraw from p at this position
+                }
+                const float x = u * W;
+                float carry = 0.f;
+                int token = -1;
+                for (int base = 0; base < nt; base += 32) {
+                    const float w = (base + lane < nt) ? weight(base + lane) : 0.f;
+                    const float incl = warp_incl_scan(w, lane);
+                    const unsigned hit = __ballot_sync(0xffffffffu, base + lane < nt && carry + incl > x);
+                    if (hit) {
+                        token = lt[base + __ffs(hit) - 1].i;
+                        break;
+                    }
+                    carry += __shfl_sync(0xffffffffu, incl, 31);
+                }
+                if (token < 0) {  // rounding: the last entry with positive weight
+                    int lastp = -1;
+                    for (int base = 0; base < nt; base += 32) {
+                        const float w = (base + lane < nt) ? weight(base + lane) : 0.f;
+                        const unsigned pos = __ballot_sync(0xffffffffu, w > 0.f);
+                        if (pos) lastp = base + 31 - __clz(pos);
+                    }
+                    token = lastp >= 0 ? lt[lastp].i : -1;
+                }
+                if (lane == 0) S.token = token;
+            }
+            __syncthreads();
+        } else {
+            // streaming draw over the row(s): per-segment masses, then one segment
+            const void* rowt = row_ptr(j);
+            const void* rowd = use_q0 ? row_ptr(k + 1 + j) : nullptr;
+            const bool alt = (reinterpret_cast<uintptr_t>(rowt) & 15u) == 0;
+            const bool ald = rowd && (reinterpret_cast<uintptr_t>(rowd) & 15u) == 0;
+            const int vps = P.seg / VEC;                      // vectors per segment
+            const int nvec = (V + VEC - 1) / VEC;
+            bool use_q = use_q0;
+            auto wt = [&](float zt, float zdv) {
+                const float pt = (zt >= tst.tau) ? ex2(fmaf(zt, c, -tst.msc)) * tst.invS : 0.f;
+                if (!use_q) return pt;
+                const float qd = (zdv >= dst.tau) ? ex2(fmaf(zdv, c, -dst.msc)) * dst.invS : 0.f;
+                return fmaxf(pt - qd, 0.f);
+            };
+            auto vec_w = [&](int q, float* w) {
+                float vt[VEC], vd[VEC];
+                load_vec<DT>(rowt, alt, q, V, vt);
+                if (use_q) load_vec<DT>(rowd, ald, q, V, vd);
+#pragma unroll
+                for (int t = 0; t < VEC; ++t) w[t] = wt(vt[t], use_q ? vd[t] : NEG_INF);
+            };
+            // masses known from the streaming pass: a plain (unmasked) bonus draw
+            const bool known = P.mode == MODE_SOFTMAX && !use_q0;
+            for (int attempt = 0; attempt < 2; ++attempt) {
+                if (known) {
+                    for (int s = tid; s < P.nseg; s += NT) {
+                        const SegRec g = P.segs[row_index(j) * P.nseg + s];
+                        mass[s] = g.s * ex2(g.m - tst.msc) * tst.invS;
+                    }
+                } else {
+                    for (int s = 0; s < P.nseg; ++s) {
+                        float acc = 0.f;
+                        for (int q = s * vps + tid; q < min(nvec, (s + 1) * vps); q += NT) {
+                            float w[VEC];
+                            vec_w(q, w);
+#pragma unroll
+                            for (int t = 0; t < VEC; ++t) acc += w[t];
+                        }
+                        acc = warp_sum(acc);
+                        if (lane == 0) part[s * NW + warp] = acc;
+                    }
+                    __syncthreads();
+                    for (int s = tid; s < P.nseg; s += NT) {
+                        float a = 0.f;
+                        for (int w = 0; w < NW; ++w) a += part[s * NW + w];
+                        mass[s] = a;
+                    }
+                }
+                __syncthreads();
+                if (tid == 0) {
+                    float W = 0.f;
+                    for (int s = 0; s < P.nseg; ++s) W += mass[s];
+                    S.retry = (!(W > 0.f) && use_q) ? 1 : 0;
+                    const float x = u * W;
+                    int sel = -1, lastm = 0;
+                    float a = 0.f, base = 0.f;
+                    for (int s = 0; s < P.nseg; ++s) {
+                        const float nxt = a + mass[s];
+                        if (nxt > x) {
+                            sel = s;
+                            base = a;
+                            break;
+                        }
+                        a = nxt;
+                    }
+                    if (sel < 0) {
+                        lastm = 1;
+                        for (int s = P.nseg - 1; s >= 0; --s)
+                            if (mass[s] > 0.f) {
+                                sel = s;
+                                break;
+                            }
+                    }
+                    S.W = W;
+                    S.x = x;
+                    S.base = base;
+                    S.seg_sel = sel;
+                    S.last_mode = lastm;
+                    S.tok_cross = -1;
+                    S.tok_last = -1;
+                }
+                __syncthreads();
+                if (!S.retry) break;
+                use_q = false;  // zero residual mass: redraw from p at this position
+                __syncthreads();
+            }
+            const int sel = S.seg_sel;
+            if (sel >= 0) {
+                const float x = S.x;
+                float base = S.base;
+                const bool lastm = S.last_mode != 0;
+                const int q0 = sel * vps, q1 = min(nvec, (sel + 1) * vps);
+                for (int tq = q0; tq < q1; tq += NT) {  // tiles of NT vectors, in index order
+                    const int q = tq + tid;
+                    float w[VEC];
+                    float vs = 0.f;
+                    if (q < q1) {
+                        vec_w(q, w);
+#pragma unroll
+                        for (int t = 0; t < VEC; ++t) vs += w[t];
+                    } else {
+#pragma unroll
+                        for (int t = 0; t < VEC; ++t) w[t] = 0.f;
+                    }
+                    int lastpos = -1;
+#pragma unroll
+                    for (int t = 0; t < VEC; ++t)
+                        if (w[t] > 0.f) lastpos = q * VEC + t;
+                    if (lastpos >= 0) atomicMax(&S.tok_last, lastpos);
+                    const float inw = warp_incl_scan(vs, lane);
+                    float exw = __shfl_up_sync(0xffffffffu, inw, 1);
+                    if (lane == 0) exw = 0.f;
+                    if (lane == 31) S.red_f[warp][0] = inw;
+                    __syncthreads();
+                    if (tid == 0) {
+                        float a = 0.f;
+                        for (int w2 = 0; w2 < NW; ++w2) {
+                            S.red_f[w2][1] = a;
+                            a += S.red_f[w2][0];
+                        }
+                    }
+                    __syncthreads();
+                    const float wp = S.red_f[warp][1];
+                    const float tile_tot = S.red_f[NW - 1][1] + S.red_f[NW - 1][0];
+                    if (!lastm && S.tok_cross < 0) {
+                        const float incl = base + (wp + inw);
+                        const float excl = base + (wp + exw);
+                        if (excl <= x && x < incl) {
+                            float acc = excl;
+                            int tok = -1;
+#pragma unroll
+                            for (int t = 0; t < VEC; ++t) {
+                                if (tok < 0 && w[t] > 0.f) {
+                                    const float nacc = acc + w[t];
+                                    if (nacc > x) tok = q * VEC + t;
+                                    acc = nacc;
+                                }
+                            }
+                            if (tok < 0) tok = lastpos;
+                            S.tok_cross = tok;
+                        }
+                    }
+                    base = base + tile_tot;
+                    __syncthreads();
+                }
+                if (tid == 0) S.token = S.tok_cross >= 0 ? S.tok_cross : S.tok_last;
+            } else if (tid == 0) {
+                S.token = -1;
+            }
+            __syncthreads();
+        }
+    }
+
+    // ---- phase 4: outputs --------------------------------------------------------------
+    if (tid == 0) {
+        int err = S.err;
+        const int j = S.j;
+        const int y = err ? -1 : S.token;
+        if (y < 0) err = 1;
+        if (P.sample_only) {
+            P.out_tokens[b] = err ? -1 : y;
+        } else {
+            int32_t* out = P.out_tokens + b * (k + 1);
+            for (int i = 0; i <= k; ++i) out[i] = (!err && i < j) ? dtok[i] : -1;
+            if (!err) out[j] = y;
+            P.out_n[b] = err ? -1 : j;
+        }
+    }
+}
+
+}  // namespace sv

@@ -28,18 +28,25 @@
  *   - argmax ties go to the lowest index; -0.0 equals +0.0.
  *
  * Memory: every pointer is DEVICE memory owned by the caller and must stay
- * valid until the stream work completes.  The library allocates nothing and
- * keeps no state between calls.  Logits are contiguous row-major; bf16 rows
- * need 2-byte and fp32 rows 4-byte alignment (16-byte-aligned rows take the
- * fastest path).  Integer and float arrays need 4-byte alignment.
+ * valid until the stream work completes.  Logits are contiguous row-major;
+ * bf16 rows need 2-byte and fp32 rows 4-byte alignment (16-byte-aligned rows
+ * take the fastest path).  Integer and float arrays need 4-byte alignment.
+ * The kernels exchange per-row partial results through a device WORKSPACE
+ * (spec_verify_workspace_size bytes, 16-byte aligned): the _ex entry points
+ * take it from the caller; with workspace = NULL, and always for
+ * spec_verify / spec_sample, the library takes it from its own
+ * stream-ordered memory pool on the call's stream and releases it on the
+ * same stream (memory the pool keeps for reuse).  Nothing else is allocated
+ * and no state is kept between calls.
  *
  * Errors:
  *   - argument problems found on the host return SV_ERR_INVALID_ARG with no
  *     launch (B <= 0, k < 1, V < 1, top_k < 0, unknown mode or dtype bits,
- *     a required pointer NULL or misaligned, sizes that overflow);
+ *     a required pointer NULL or misaligned, sizes that overflow, a
+ *     workspace that is too small or misaligned);
  *   - SV_ERR_UNSUPPORTED: no usable CUDA device of compute capability >= 9.0,
- *     or a vocabulary whose rows do not fit the per-cluster shared memory
- *     (2 * V * element size > 16 * ~200 KB for verification);
+ *     or sizes whose per-sequence shared-memory needs exceed the device
+ *     (about k > 1000);
  *   - SV_ERR_CUDA: a CUDA call failed while launching;
  *   - per-sequence data errors do not fail the call: out_n_accepted[b] = -1
  *     and out_tokens[b, :] = -1.  They are a draft token outside [0, V), a
@@ -53,6 +60,7 @@
 #ifndef SPEC_VERIFY_H
 #define SPEC_VERIFY_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #if defined(__GNUC__)
@@ -81,13 +89,13 @@ enum {
     SV_DTYPE_F32 = 1 << 8
 };
 
-/* Tuning and instrumentation for spec_verify_ex / spec_sample_ex.  Zero
- * every field for the library's own choices. */
+/* Tuning and instrumentation for the _ex entry points.  Zero every field for
+ * the library's own choices. */
 typedef struct sv_options {
-    int cluster_size;          /* CTAs per row pair: 0 = auto, else 1, 2, 4, 8 or 16 */
-    int threads;               /* threads per CTA: 0 = auto (256), else 128, 256 or 512 */
-    int topk_path;             /* 0 = auto, 1 = candidate threshold path, 2 = radix select */
-    void* event_start;         /* cudaEvent_t or NULL, recorded before the verify kernel */
+    int chunks_per_row;        /* streaming tasks per logit row: 0 = auto, else >= 1 */
+    int threads;               /* threads per streaming CTA: 0 = auto (256), else 128, 256 or 512 */
+    int topk_path;             /* 0 = auto, 1 = kept lists, 2 = radix select */
+    void* event_start;         /* cudaEvent_t or NULL, recorded before the streaming kernel */
     void* event_stop;          /* cudaEvent_t or NULL, recorded right after it */
     uint64_t wait_timeout_ns;  /* bound of every device-side wait: 0 = 1e9 ns */
     uint32_t test_extra_tx;    /* test hook: bytes added to each bulk-copy wait so that
@@ -117,19 +125,30 @@ SV_API sv_status_t spec_verify(const void* target_logits, const void* draft_logi
                         int32_t* out_tokens, int32_t* out_n_accepted, void* stream);
 
 /*
- * spec_verify_ex — spec_verify plus optional outputs and options.
- *   out_p, out_q  [B][k] fp32 or NULL: p_i(d_i) and q_i(d_i) at EVERY
- *                 position (also past the first rejection); stochastic mode
- *   out_status    1 int32 or NULL: SV_OK, or SV_ERR_DEVICE_TIMEOUT if a
- *                 device wait ran out (written by the call's kernels)
- *   opts          NULL or options (see sv_options_t)
+ * spec_verify_workspace_size — device workspace bytes spec_verify_ex needs
+ * for these arguments on the current device (0 on invalid arguments).
+ */
+SV_API size_t spec_verify_workspace_size(int B, int k, int V, int top_k, int mode,
+                                         const sv_options_t* opts);
+
+/*
+ * spec_verify_ex — spec_verify plus optional outputs, workspace and options.
+ *   out_p, out_q     [B][k] fp32 or NULL: p_i(d_i) and q_i(d_i) at EVERY
+ *                    position (also past the first rejection); stochastic mode
+ *   out_status       1 int32 or NULL: SV_OK, or SV_ERR_DEVICE_TIMEOUT if a
+ *                    device wait ran out (written by the call's kernels)
+ *   workspace        NULL (library pool) or >= spec_verify_workspace_size
+ *                    bytes, 16-byte aligned; calls that share a workspace must
+ *                    be ordered on one stream
+ *   workspace_bytes  its size
+ *   opts             NULL or options (see sv_options_t)
  */
 SV_API sv_status_t spec_verify_ex(const void* target_logits, const void* draft_logits,
-                           const int32_t* draft_tokens, const float* uniforms, int B, int k,
-                           int V, const float* temperature, int top_k, int mode,
-                           int32_t* out_tokens, int32_t* out_n_accepted, float* out_p,
-                           float* out_q, int32_t* out_status, const sv_options_t* opts,
-                           void* stream);
+                                  const int32_t* draft_tokens, const float* uniforms, int B, int k,
+                                  int V, const float* temperature, int top_k, int mode,
+                                  int32_t* out_tokens, int32_t* out_n_accepted, float* out_p,
+                                  float* out_q, int32_t* out_status, void* workspace,
+                                  size_t workspace_bytes, const sv_options_t* opts, void* stream);
 
 /*
  * spec_sample — the proposer's sampling step (section "提议与核验的基本步骤",
@@ -147,10 +166,15 @@ SV_API sv_status_t spec_sample(const void* logits, const float* uniforms, int ro
                         const float* temperature, int top_k, int mode, int32_t* out_tokens,
                         void* stream);
 
-/* spec_sample with options (opts may be NULL). */
+/* Workspace bytes of spec_sample_ex on the current device (0 on invalid arguments). */
+SV_API size_t spec_sample_workspace_size(int rows, int V, int top_k, int mode,
+                                         const sv_options_t* opts);
+
+/* spec_sample with a workspace (NULL: library pool) and options (may be NULL). */
 SV_API sv_status_t spec_sample_ex(const void* logits, const float* uniforms, int rows, int V,
-                           const float* temperature, int top_k, int mode, int32_t* out_tokens,
-                           const sv_options_t* opts, void* stream);
+                                  const float* temperature, int top_k, int mode,
+                                  int32_t* out_tokens, void* workspace, size_t workspace_bytes,
+                                  const sv_options_t* opts, void* stream);
 
 /* Static description of a status code. */
 SV_API const char* spec_verify_status_string(sv_status_t status);

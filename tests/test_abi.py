@@ -28,8 +28,8 @@ def declared_functions():
 
 def test_header_declares_entry_points():
     assert declared_functions() == sorted([
-        "spec_sample", "spec_sample_ex", "spec_verify", "spec_verify_ex",
-        "spec_verify_status_string", "spec_verify_version"])
+        "spec_sample", "spec_sample_ex", "spec_sample_workspace_size", "spec_verify", "spec_verify_ex",
+        "spec_verify_status_string", "spec_verify_version", "spec_verify_workspace_size"])
 
 
 def test_library_exports_every_declared_symbol(L):
@@ -44,7 +44,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_version_and_status_strings(L):
-    assert sv.spec_verify_version() == 10000
+    assert sv.spec_verify_version() == 20000
     assert sv.spec_verify_status_string(sv.SV_OK) == "ok"
     assert sv.spec_verify_status_string(sv.SV_ERR_DEVICE_TIMEOUT) == "device-side wait timed out"
     assert sv.spec_verify_status_string(123) == "unknown status"
@@ -58,7 +58,7 @@ def test_options_struct_layout_matches_c(tmp_path):
 #include "spec_verify.h"
 int main(void) {
   printf("%zu %zu %zu %zu %zu %zu %zu %zu\n", sizeof(sv_options_t),
-         offsetof(sv_options_t, cluster_size), offsetof(sv_options_t, threads),
+         offsetof(sv_options_t, chunks_per_row), offsetof(sv_options_t, threads),
          offsetof(sv_options_t, topk_path), offsetof(sv_options_t, event_start),
          offsetof(sv_options_t, event_stop), offsetof(sv_options_t, wait_timeout_ns),
          offsetof(sv_options_t, test_extra_tx));
@@ -112,12 +112,20 @@ def test_greedy_allows_null_draft_and_uniforms(L):
     assert st != sv.SV_ERR_INVALID_ARG
 
 
-@pytest.mark.parametrize("field,val", [("cluster_size", 3), ("cluster_size", 32), ("threads", 64),
+@pytest.mark.parametrize("field,val", [("chunks_per_row", -1), ("threads", 64),
                                        ("threads", 1024), ("topk_path", 3), ("topk_path", -1)])
 def test_invalid_options_rejected(L, field, val):
     o = sv.make_options(**{field: val})
-    st = sv.spec_verify_ex(P, P, P, P, 2, 3, 100, None, 0, 0, P, P, None, None, None, o, 0)
+    st = sv.spec_verify_ex(P, P, P, P, 2, 3, 100, None, 0, 0, P, P, None, None, None, None, 0, o, 0)
     assert st == sv.SV_ERR_INVALID_ARG
+    assert sv.spec_verify_workspace_size(2, 3, 100, 0, 0, o) == 0
+
+
+@pytest.mark.parametrize("kw", [dict(B=0), dict(k=0), dict(V=0), dict(top_k=-1), dict(mode=7)])
+def test_workspace_size_invalid_arguments(L, kw):
+    a = dict(B=2, k=3, V=100, top_k=0, mode=0)
+    a.update(kw)
+    assert sv.spec_verify_workspace_size(**a) == 0
 
 
 @pytest.mark.parametrize("kw", [dict(rows=0), dict(V=0), dict(top_k=-1), dict(mode=5),

@@ -182,18 +182,19 @@ def test_draft_token_outside_draft_top_k():
     compare(ref, gpu, case.uniforms)
 
 
-@pytest.mark.parametrize("cluster", [1, 2, 4, 8, 16])
+@pytest.mark.parametrize("chunks", [1, 2, 3, 5, 16])
 @pytest.mark.parametrize("threads", [128, 256, 512])
-def test_launch_shapes(cluster, threads):
-    case = workloads.make_case("tiny", seed=cluster * threads, B=6, k=3, V=20000, dtype="bf16",
-                               top_k=40 if threads == 256 else 0)
-    check_case(case, opts=sv.make_options(cluster_size=cluster, threads=threads))
+@pytest.mark.parametrize("K", [0, 40])
+def test_launch_shapes(chunks, threads, K):
+    case = workloads.make_case("tiny", seed=chunks * threads + K, B=6, k=3, V=20000, dtype="bf16", top_k=K)
+    check_case(case, opts=sv.make_options(chunks_per_row=chunks, threads=threads))
 
 
-@pytest.mark.parametrize("cluster", [4, 8, 16])
-def test_full_vocab_cluster_sizes(cluster):
-    case = workloads.make_case("batched", seed=cluster, B=4, k=2)
-    check_case(case, opts=sv.make_options(cluster_size=cluster))
+@pytest.mark.parametrize("chunks", [1, 4, 19])
+@pytest.mark.parametrize("K", [0, 50])
+def test_full_vocab_chunking(chunks, K):
+    case = workloads.make_case("batched", seed=chunks, B=4, k=2, top_k=K)
+    check_case(case, opts=sv.make_options(chunks_per_row=chunks))
 
 
 # --------------------------------------------------------------------------
