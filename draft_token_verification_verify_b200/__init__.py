@@ -27,6 +27,7 @@ SV_MODE_STOCHASTIC = 0
 SV_MODE_GREEDY = 1
 SV_DTYPE_BF16 = 0 << 8
 SV_DTYPE_F32 = 1 << 8
+SV_STATIC_WORKSPACE_BYTES = 4 << 20  # scratch bytes available to spec_verify_static
 
 LIB_PATH = _build.LIB
 
@@ -34,6 +35,7 @@ __all__ = [
     "SV_OK", "SV_ERR_INVALID_ARG", "SV_ERR_UNSUPPORTED", "SV_ERR_CUDA", "SV_ERR_DEVICE_TIMEOUT",
     "SV_MODE_STOCHASTIC", "SV_MODE_GREEDY", "SV_DTYPE_BF16", "SV_DTYPE_F32", "SvOptions",
     "SpecVerifyError", "lib", "spec_verify", "spec_verify_ex", "spec_verify_workspace_size",
+    "spec_verify_static", "SV_STATIC_WORKSPACE_BYTES",
     "spec_sample", "spec_sample_ex", "spec_sample_workspace_size", "make_options",
     "spec_verify_status_string", "spec_verify_version", "verify", "sample",
 ]
@@ -75,6 +77,8 @@ def lib() -> ctypes.CDLL:
         OP = ctypes.POINTER(SvOptions)
         L.spec_verify_ex.argtypes = [P, P, P, P, I, I, I, P, I, I, P, P, P, P, P, P, Z, OP, P]
         L.spec_verify_ex.restype = I
+        L.spec_verify_static.argtypes = [P, P, P, P, I, I, I, P, I, I, P, P, P, P, P, OP, P]
+        L.spec_verify_static.restype = I
         L.spec_verify_workspace_size.argtypes = [I, I, I, I, I, OP]
         L.spec_verify_workspace_size.restype = Z
         L.spec_sample.argtypes = [P, P, I, I, P, I, I, P, P]
@@ -145,6 +149,20 @@ def spec_verify_ex(target_logits, draft_logits, draft_tokens, uniforms, B, k, V,
                                 _p(out_tokens), _p(out_n_accepted), _p(out_p), _p(out_q),
                                 _p(out_status), _p(workspace), int(workspace_bytes), _opts(opts),
                                 _stream(stream))
+
+
+def spec_verify_static(target_logits, draft_logits, draft_tokens, uniforms, B, k, V, temperature, top_k,
+                       mode, out_tokens, out_n_accepted, out_p=None, out_q=None, out_status=None,
+                       opts: Optional[SvOptions] = None, stream=None) -> int:
+    """``spec_verify_ex`` without a workspace argument and without any device
+    allocation: scratch comes from the library's fixed per-device buffer of
+    ``SV_STATIC_WORKSPACE_BYTES``.  For callers that cannot allocate during
+    the call.  Overlapping calls on different streams share that buffer and
+    must not run at the same time."""
+    return lib().spec_verify_static(_p(target_logits), _p(draft_logits), _p(draft_tokens), _p(uniforms),
+                                    int(B), int(k), int(V), _p(temperature), int(top_k), int(mode),
+                                    _p(out_tokens), _p(out_n_accepted), _p(out_p), _p(out_q),
+                                    _p(out_status), _opts(opts), _stream(stream))
 
 
 def spec_verify_workspace_size(B, k, V, top_k, mode, opts: Optional[SvOptions] = None) -> int:

@@ -476,6 +476,33 @@ size_t workspace_for(const Call& cl, const sv_options_t* opts) {
     return p.ws_bytes;
 }
 
+// ---- static scratch for spec_verify_static ----------------------------------------
+
+// One fixed buffer per device, part of the library's device image: calls that
+// must not allocate take their scratch from here.
+std::once_flag g_static_once[kMaxDevices];
+void* g_static_ptr[kMaxDevices];
+
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_sv_static_scratch[SV_STATIC_WORKSPACE_BYTES];
+
+namespace {
+
+// Device address of the static buffer on `dev`, which must be the current
+// device; looked up once per device.  NULL if the lookup failed.
+void* static_scratch(int dev) {
+    std::call_once(g_static_once[dev], [dev] {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_sv_static_scratch) != cudaSuccess) {
+            cudaGetLastError();
+            ptr = nullptr;
+        }
+        g_static_ptr[dev] = ptr;
+    });
+    return g_static_ptr[dev];
+}
+
 }  // namespace
 
 extern "C" {
@@ -491,6 +518,25 @@ sv_status_t spec_verify_ex(const void* target_logits, const void* draft_logits, 
                                       true, &cl);
     if (s != SV_OK) return s;
     return run(cl, workspace, workspace_bytes, opts, static_cast<cudaStream_t>(stream));
+}
+
+sv_status_t spec_verify_static(const void* target_logits, const void* draft_logits, const int32_t* draft_tokens,
+                               const float* uniforms, int B, int k, int V, const float* temperature, int top_k,
+                               int mode, int32_t* out_tokens, int32_t* out_n_accepted, float* out_p, float* out_q,
+                               int32_t* out_status, const sv_options_t* opts, void* stream) {
+    Call cl;
+    sv_status_t s = verify_args(target_logits, draft_logits, draft_tokens, uniforms, B, k, V, temperature, top_k,
+                                mode, out_tokens, out_n_accepted, out_p, out_q, out_status, opts, true, &cl);
+    if (s != SV_OK) return s;
+    int dev = 0;
+    const DeviceInfo* info = device_info(&dev);
+    if (!info) return SV_ERR_UNSUPPORTED;
+    Plan p;
+    if ((s = make_plan(*info, cl.seqs, cl.k, cl.V, cl.dt, cl.greedy, cl.top_k, opts, &p)) != SV_OK) return s;
+    if (p.ws_bytes > SV_STATIC_WORKSPACE_BYTES) return SV_ERR_UNSUPPORTED;  // beyond the static buffer
+    void* ws = static_scratch(dev);
+    if (!ws) return SV_ERR_CUDA;
+    return run(cl, ws, SV_STATIC_WORKSPACE_BYTES, opts, static_cast<cudaStream_t>(stream));
 }
 
 sv_status_t spec_verify(const void* target_logits, const void* draft_logits, const int32_t* draft_tokens,

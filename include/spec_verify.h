@@ -150,6 +150,48 @@ SV_API sv_status_t spec_verify_ex(const void* target_logits, const void* draft_l
                                   float* out_q, int32_t* out_status, void* workspace,
                                   size_t workspace_bytes, const sv_options_t* opts, void* stream);
 
+/* Bytes of the library's static scratch buffer used by spec_verify_static. */
+#define SV_STATIC_WORKSPACE_BYTES (4u << 20)
+
+/*
+ * spec_verify_static — spec_verify_ex that allocates nothing.
+ *
+ * The method's description has no counterpart to this call: it is a
+ * library convenience for callers that must not allocate device memory
+ * while they run.  Examples are a serving loop that has given every free byte
+ * to its own cache allocator, and code that holds a lock that a
+ * stream-ordered pool may re-enter.  spec_verify_ex with a NULL workspace
+ * draws scratch from a library pool, and with a caller workspace it needs
+ * that buffer sized and kept alive.  This call instead uses a fixed
+ * SV_STATIC_WORKSPACE_BYTES buffer compiled into the library for each device
+ * (a __device__ array), so it performs no cudaMalloc, cudaFree or pool
+ * allocation of any kind.
+ *
+ * Arguments and outputs are those of spec_verify_ex without the workspace.
+ *
+ * Set-up: the first call on a device, with that device current, looks up the
+ * buffer's device address once and caches it.  Make that first call before
+ * any stream capture on that device.
+ *
+ * Limit: a problem whose scratch need (spec_verify_workspace_size with the
+ * same arguments and options) exceeds SV_STATIC_WORKSPACE_BYTES is rejected
+ * with SV_ERR_UNSUPPORTED before anything is launched.
+ *
+ * Contents: nothing in the buffer has to start at zero; each call writes
+ * every scratch record it reads, and writes *out_status itself.
+ *
+ * Concurrency: there is ONE buffer per device.  Calls on one stream run one
+ * after the other and are safe.  Calls whose execution can overlap, on
+ * different streams or from different host threads without ordering
+ * between them, use the same bytes at the same time and give wrong results.
+ */
+SV_API sv_status_t spec_verify_static(const void* target_logits, const void* draft_logits,
+                                      const int32_t* draft_tokens, const float* uniforms, int B,
+                                      int k, int V, const float* temperature, int top_k, int mode,
+                                      int32_t* out_tokens, int32_t* out_n_accepted, float* out_p,
+                                      float* out_q, int32_t* out_status, const sv_options_t* opts,
+                                      void* stream);
+
 /*
  * spec_sample — the proposer's sampling step (section "提议与核验的基本步骤",
  * paragraph 1: the proposer draws each candidate from its own

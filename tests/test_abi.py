@@ -29,7 +29,7 @@ def declared_functions():
 def test_header_declares_entry_points():
     assert declared_functions() == sorted([
         "spec_sample", "spec_sample_ex", "spec_sample_workspace_size", "spec_verify", "spec_verify_ex",
-        "spec_verify_status_string", "spec_verify_version", "spec_verify_workspace_size"])
+        "spec_verify_static", "spec_verify_status_string", "spec_verify_version", "spec_verify_workspace_size"])
 
 
 def test_library_exports_every_declared_symbol(L):
