@@ -25,6 +25,7 @@ constexpr int kListCap = 1024;        // shared candidate list of a streaming CT
 
 struct DeviceInfo {
     int ok = 0;
+    int id = 0;
     int sms = 0;
     int smem_optin = 0;
     int smem_per_sm = 0;
@@ -35,6 +36,8 @@ DeviceInfo g_dev[kMaxDevices];
 std::once_flag g_dev_once[kMaxDevices];
 std::once_flag g_pool_once[kMaxDevices];
 std::once_flag g_attr_once[kMaxDevices][26];
+std::once_flag g_occ_once[kMaxDevices][24];
+int g_occ[kMaxDevices][24];
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -57,6 +60,7 @@ const DeviceInfo* device_info(int* dev_out) {
             return;
         }
         d.ok = major >= 9 ? 1 : 0;
+        d.id = dev;
     });
     *dev_out = dev;
     return g_dev[dev].ok ? &g_dev[dev] : nullptr;
@@ -88,12 +92,14 @@ long long ceil_div(long long a, long long b) { return (a + b - 1) / b; }
 long long round_up(long long a, long long b) { return ceil_div(a, b) * b; }
 
 struct Plan {
-    int mode = 0, elt = 2, seg = 0, nseg = 0, nch = 1, spc = 1, nt1 = 256, stages = kStages;
-    int stage_bytes = 0, lcap = 0, kcap = 0, mg = 0;
+    int mode = 0, elt = 2, seg = 0, nseg = 0, nch = 1, spc = 1, nt1 = 128, stages = kStages;
+    int lcap = 0, kcap = 0, mg = 0;
     long long R = 0, tasks = 0;
     size_t smem1 = 0, smem2 = 0;
     size_t off_chunks = 0, off_cands = 0, ws_bytes = 0;
 };
+
+int rows_occupancy(int dev, int dt, int nt, int mode, size_t smem);
 
 // Plan the launches for `seqs` sequences of draft length k (rows = k+1 target
 // rows per sequence, plus k draft rows when stochastic).
@@ -116,7 +122,6 @@ sv_status_t make_plan(const DeviceInfo& dev, long long seqs, int k, int V, int d
     else
         p.mode = sv::MODE_MAXONLY;
     if (opts && opts->topk_path == 1 && top_k > 0 && p.mode != sv::MODE_TOPK) return SV_ERR_UNSUPPORTED;
-    p.stage_bytes = static_cast<int>(round_up(kSegBytes + 32, 128));
     if (p.mode == sv::MODE_TOPK) {
         // the running bound needs K <= threads (each warp contributes <= 32 ranks)
         if (top_k > p.nt1) {
@@ -129,14 +134,11 @@ sv_status_t make_plan(const DeviceInfo& dev, long long seqs, int k, int V, int d
         }
         if (p.mode == sv::MODE_TOPK) p.lcap = kListCap;
     }
-    p.smem1 = static_cast<size_t>(sv::ROWS_CTL_BYTES) + static_cast<size_t>(p.stages) * p.stage_bytes +
-              static_cast<size_t>(3) * sv::MAX_TILES_K1 * (p.nt1 / 32) * 4;
-    if (p.mode == sv::MODE_TOPK) p.smem1 += static_cast<size_t>(p.lcap) * 8;
+    p.smem1 = static_cast<size_t>(sv::rows_smem_bytes(p.mode, p.nt1, p.stages, p.lcap));
+    if (p.smem1 > static_cast<size_t>(dev.smem_optin)) return SV_ERR_UNSUPPORTED;
     // chunks per row: one when there are enough rows to fill the device
-    const long long per_sm_smem = dev.smem_per_sm > 0 ? dev.smem_per_sm : 233472;
-    long long occ = per_sm_smem / static_cast<long long>(p.smem1 + 1024);
-    if (occ > 2048 / p.nt1) occ = 2048 / p.nt1;
-    if (occ < 1) occ = 1;
+    long long occ = rows_occupancy(dev.id, dt, p.nt1, p.mode, p.smem1);
+    if (occ < 1) return SV_ERR_CUDA;
     const long long slots = occ * dev.sms;
     int nch;
     if (opts && opts->chunks_per_row) {
@@ -231,6 +233,23 @@ sv_status_t set_attrs(int dev, int dt, int nt, int mode) {
     return SV_OK;
 }
 
+// Resident streaming CTAs per SM for one instantiation (its shared memory
+// depends only on the slot), from the occupancy calculator; 0 on failure.
+int rows_occupancy(int dev, int dt, int nt, int mode, size_t smem) {
+    if (set_attrs(dev, dt, nt, mode) != SV_OK) return 0;
+    int slot = 0;
+    RowsFn f1 = pick_rows(dt, nt, mode, &slot);
+    std::call_once(g_occ_once[dev][slot], [&] {
+        int n = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, f1, nt + 32, smem) != cudaSuccess) {
+            cudaGetLastError();
+            n = 0;
+        }
+        g_occ[dev][slot] = n;
+    });
+    return g_occ[dev][slot];
+}
+
 struct Call {
     const void* target = nullptr;
     const void* draft = nullptr;
@@ -278,15 +297,12 @@ sv_status_t run(const Call& cl, void* workspace, size_t workspace_bytes, const s
     r.B = cl.seqs;
     r.k = cl.k;
     r.V = cl.V;
-    r.mode = p.mode;
     r.top_k = cl.top_k;
     r.temperature = cl.temperature;
-    r.seg = p.seg;
     r.nseg = p.nseg;
     r.spc = p.spc;
     r.nch = p.nch;
     r.stages = p.stages;
-    r.stage_bytes = p.stage_bytes;
     r.lcap = p.lcap;
     r.kcap = p.kcap;
     r.segs = reinterpret_cast<sv::SegRec*>(base);
@@ -336,7 +352,7 @@ sv_status_t run(const Call& cl, void* workspace, size_t workspace_bytes, const s
         cudaLaunchConfig_t c1;
         std::memset(&c1, 0, sizeof c1);
         c1.gridDim = dim3(static_cast<unsigned>(p.tasks), 1, 1);
-        c1.blockDim = dim3(p.nt1, 1, 1);
+        c1.blockDim = dim3(p.nt1 + 32, 1, 1);  // consumer warps + the producer warp
         c1.dynamicSmemBytes = p.smem1;
         c1.stream = st;
         if (cudaLaunchKernelEx(&c1, f1, r) != cudaSuccess) {

@@ -1,23 +1,31 @@
 // K1 — the streaming pass over every logit row of a verification batch.
 //
-// One CTA per task = one chunk (a run of consecutive segments) of one row.
-// The chunk streams through a ring of shared-memory stages filled by bulk
-// copies (cp.async.bulk, no multicast) that complete on mbarriers; every
-// wait is bounded in time.  The refill of a stage is issued as soon as every
-// thread has finished reading it; nothing else sits between a stage's
-// consumption and its refill.  Each segment (one stage) leaves a 16-byte
-// partial in the workspace, written at the end of the chunk:
-//   greedy   raw maximum and its lowest index,
-//   softmax  online (max, sum of 2^(z*c - max)) with c = log2(e)/T,
-//   top-k    raw maximum.
-// With top-k the chunk also keeps, in the same single pass, every element
-// that can belong to the top-k set: a running lower bound theta on the
-// chunk's K-th largest logit (the K-th largest of the groups' running maxima:
-// K distinct elements are >= it) filters the stream into a shared candidate
-// list.  At the end the exact K-th largest tau_c of the chunk and every
-// element >= tau_c are stored sorted by index, with the chunk maximum, the
-// sum of 2^(z*c - max*c) over the stored entries and the logit at the row's
-// draft token when it is among them.
+// One CTA per task = one chunk (a run of consecutive 16 KB segments) of one
+// row, warp-specialised.  Warp NW (the producer) streams the chunk into a
+// ring of shared-memory stages with bulk copies (cp.async.bulk, no
+// multicast); every stage has a "full" mbarrier (one arrival plus the copy's
+// bytes) and an "empty" mbarrier (one arrival per consumer warp).  Warps
+// 0..NW-1 (the consumers) work through the tiles independently of each other
+// and hand each stage back as soon as they are done with it: no block-wide
+// barrier runs per tile.  Every wait is bounded in time.
+//
+// Partials written to the workspace:
+//   greedy   per chunk: raw maximum and its lowest index,
+//   softmax  per segment: (max of z*c, sum of 2^(z*c - max)), c = log2(e)/T,
+//   max-only per chunk: raw maximum,
+//   top-k    per chunk: every element that can belong to the chunk's top-k
+//            set, found in the same single pass.  Warp w publishes a value
+//            b_w such that it has seen at least rsel = ceil(K / NW) distinct
+//            elements >= b_w (the rsel-th largest of its lanes' running
+//            maxima, or the rsel-th largest entry of its own candidate
+//            list).  Then at least NW * rsel >= K elements are >= min_w b_w,
+//            so that minimum never exceeds the chunk's K-th largest logit —
+//            whatever mix of older and newer published values a warp reads.
+//            Elements at or above it go to the warp's private list segment.
+//            At the end the exact K-th largest tau_c of the chunk and every
+//            element >= tau_c are stored, sorted by index, with the chunk
+//            maximum, the sum of 2^(z*c - max*c) over them and the logit at
+//            the row's draft token.
 // Rows are read from HBM exactly once; no CTA waits for another.
 #pragma once
 
@@ -28,9 +36,11 @@
 namespace sv {
 
 constexpr int MAX_STAGES = 8;
-constexpr int MAX_TILES_K1 = 64; // segments per chunk
-constexpr int RANK_MAX = 256;    // lists up to this size are ranked, larger ones sorted
-constexpr int TILE_BYTES = 16384; // bytes per segment (one ring stage)
+constexpr int MAX_TILES_K1 = 64;   // segments per chunk
+constexpr int RANK_MAX = 256;      // final lists up to this size are ranked, larger ones sorted
+constexpr int TILE_BYTES = 16384;  // bytes per segment (one ring stage)
+constexpr int REC_DIAG = 4;        // a device-side consistency check failed
+constexpr int MAX_CONSUMER_WARPS = 16;
 
 struct RowsParams {
     const void* target;          // [B][k+1][V] (sampler: [rows][V])
@@ -39,16 +49,13 @@ struct RowsParams {
     long long B;                 // sequences (sampler: rows)
     int k;                       // draft length (sampler: 0)
     int V;
-    int mode;                    // MODE_*
     int top_k;                   // effective K (MODE_TOPK)
     const float* temperature;    // [B] or null
-    int seg;                     // elements per segment (TILE_BYTES / element size)
     int nseg;                    // segments per row
     int spc;                     // segments per chunk (<= MAX_TILES_K1)
     int nch;                     // chunks per row
-    int stages;                  // ring stages (<= MAX_STAGES)
-    int stage_bytes;             // shared bytes per stage
-    int lcap;                    // shared candidate list capacity (power of two)
+    int stages;                  // ring stages (2..MAX_STAGES)
+    int lcap;                    // top-k candidate entries per CTA (NW segments)
     int kcap;                    // stored kept entries per chunk
     SegRec* segs;                // [R][nseg]
     ChunkRec* chunks;            // [R][nch]
@@ -59,20 +66,34 @@ struct RowsParams {
 };
 
 struct __align__(16) RowsCtl {
-    uint64_t mbar[MAX_STAGES];
-    float theta;
-    float theta_new;
-    int cnt;
+    uint64_t full[MAX_STAGES];
+    uint64_t empty[MAX_STAGES];
+    int issued;   // tiles the producer issued
+    int tmo;      // a wait ran out
+    int diag;     // a copy failed its self-check (skipped)
     int cnt2;
-    int overflow;
     int nkept;
     float tau;
-    float wsum[16];
-    float wzd[16];
-    float wsel[3][16];  // per-warp bound candidates: two tile slots and the final
+    int pad[2];
+    float wbound[MAX_CONSUMER_WARPS];  // published per-warp bounds (top-k)
+    float wmax[MAX_CONSUMER_WARPS];
+    float wbest[MAX_CONSUMER_WARPS];
+    int widx[MAX_CONSUMER_WARPS];
+    int wcnt[MAX_CONSUMER_WARPS];
+    int wovf[MAX_CONSUMER_WARPS];
+    float wsum[MAX_CONSUMER_WARPS + 1];
+    float wzd[MAX_CONSUMER_WARPS + 1];
 };
 
 constexpr int ROWS_CTL_BYTES = (int)((sizeof(RowsCtl) + 127) / 128 * 128);
+constexpr int STAGE_BYTES = (TILE_BYTES + 32 + 127) / 128 * 128;  // one segment plus one spare vector
+
+// Dynamic shared memory of one streaming CTA.
+__host__ __device__ constexpr int rows_smem_bytes(int mode, int nt, int stages, int lcap) {
+    return ROWS_CTL_BYTES + stages * STAGE_BYTES +
+           (mode == MODE_SOFTMAX ? 2 * MAX_TILES_K1 * (nt / 32) * 4 : 0) +
+           (mode == MODE_TOPK ? lcap * 8 : 0);
+}
 
 // Geometry of one segment in the ring: the stage mirrors the 16-byte aligned
 // global span [A0, A0 + 16*nvec) covering elements [lo, hi).
@@ -97,22 +118,61 @@ __device__ __forceinline__ TileGeom tile_geom(const char* row, int lo, int hi) {
     return g;
 }
 
+// Named barrier 1 over the NT consumer threads only.
+template <int NT>
+__device__ __forceinline__ void consumer_sync() {
+    asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory");
+}
+
+// Sort n (<= 32 * 16) (key, index) pairs of one warp's shared segment by key,
+// descending; entries past n are padded by the caller up to the power of two
+// `np2`.  Warp-synchronous.
+__device__ __forceinline__ void warp_sort_desc(float* key, int* idx, int np2, int lane) {
+    for (int size = 2; size <= np2; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            for (int t = lane; t < (np2 >> 1); t += 32) {
+                const int lo = 2 * stride * (t / stride) + (t % stride);
+                const int hi = lo + stride;
+                const bool up = (lo & size) == 0;
+                const float ka = key[lo], kb = key[hi];
+                if (up ? (kb > ka) : (ka > kb)) {
+                    const int ia = idx[lo];
+                    key[lo] = kb;
+                    key[hi] = ka;
+                    idx[lo] = idx[hi];
+                    idx[hi] = ia;
+                }
+            }
+            __syncwarp();
+        }
+    }
+}
+
+template <int NT>
+struct RowsOcc {  // CTAs per SM the register budget is sized for
+    static constexpr int value = NT <= 128 ? 6 : (NT <= 256 ? 4 : 2);
+};
+
 template <int DT, int NT, int MODE>
-__global__ void __launch_bounds__(NT, 1024 / NT) sv_rows_kernel(const RowsParams P) {
+__global__ void __launch_bounds__(NT + 32, RowsOcc<NT>::value) sv_rows_kernel(const RowsParams P) {
     constexpr int ELT = VT<DT>::ELT;
     constexpr int VEC = VT<DT>::VEC;
-    constexpr int NW = NT / 32;
-    constexpr int TV = TILE_BYTES / 16;  // vectors per tile
-    constexpr int VPT = TV / NT;         // vectors per thread per tile
-    static_assert(VPT * NT == TV, "tile must split evenly over the threads");
+    constexpr int NW = NT / 32;             // consumer warps; warp NW is the producer
+    constexpr int NTH = NT + 32;            // threads of the CTA
+    constexpr int TV = TILE_BYTES / 16;     // vectors per tile
+    constexpr int VPT = TV / NT;            // vectors per consumer thread per tile
+    constexpr int SEG = TILE_BYTES / ELT;   // elements per segment
+    static_assert(VPT * NT == TV, "tile must split evenly over the consumer threads");
+    static_assert(NW <= MAX_CONSUMER_WARPS, "too many consumer warps");
+    static_assert(VPT + 1 <= 32, "candidate mask");
     extern __shared__ __align__(128) unsigned char smem[];
     RowsCtl& S = *reinterpret_cast<RowsCtl*>(smem);
     unsigned char* const ring = smem + ROWS_CTL_BYTES;
-    float* const red_m = reinterpret_cast<float*>(ring + static_cast<size_t>(P.stages) * P.stage_bytes);
+    unsigned char* const tail = ring + static_cast<size_t>(P.stages) * STAGE_BYTES;
+    float* const red_m = reinterpret_cast<float*>(tail);      // softmax: [MAX_TILES_K1][NW]
     float* const red_s = red_m + MAX_TILES_K1 * NW;
-    int* const red_i = reinterpret_cast<int*>(red_s + MAX_TILES_K1 * NW);
-    float* const lkey = reinterpret_cast<float*>(red_i + MAX_TILES_K1 * NW);
-    int* const lidx = reinterpret_cast<int*>(lkey + P.lcap);
+    float* const lkey = reinterpret_cast<float*>(tail);       // top-k: [lcap]
+    int* const lidx = reinterpret_cast<int*>(lkey + P.lcap);  //        [lcap]
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const long long task = blockIdx.x;
@@ -139,299 +199,351 @@ __global__ void __launch_bounds__(NT, 1024 / NT) sv_rows_kernel(const RowsParams
         const float T = P.temperature ? P.temperature[b] : 1.f;
         if (T > 0.f && T != POS_INF) cscale = LOG2E / T;
     }
-    constexpr int SEG = TILE_BYTES / ELT;  // elements per segment
     const int s0 = c * P.spc;
     const int ntiles = min(P.spc, P.nseg - s0);
     const int K = P.top_k;
-
+    const int wcap = P.lcap / NW;  // top-k entries per warp segment
     auto geom = [&](int t) {
         const int lo = (s0 + t) * SEG;
         const int hi = min(P.V, lo + SEG);
         return tile_geom<ELT>(row, lo, hi);
     };
-    // producer: fill stage (t % stages) with tile t
-    auto issue = [&](int t) {
-        const int st = t % P.stages;
-        const TileGeom g = geom(t);
-        unsigned char* buf = ring + static_cast<size_t>(st) * P.stage_bytes;
-        uint32_t bytes = 0;
-        if (g.hi > g.lo) {
-            int nh, ntl;
-            if (g.ga16 >= g.gb16) {
-                nh = g.hi - g.lo;
-                ntl = 0;
-            } else {
-                nh = static_cast<int>((g.ga16 - g.ga) / ELT);
-                ntl = static_cast<int>((g.gb - g.gb16) / ELT);
-                bytes = static_cast<uint32_t>(g.gb16 - g.ga16);
-            }
-            // elements outside the aligned interior: plain loads before the arrive
-            for (int q = 0; q < nh + ntl; ++q) {
-                const int e = q < nh ? g.lo + q : g.hi - ntl + (q - nh);
-                if constexpr (DT == 0)
-                    reinterpret_cast<uint16_t*>(buf)[e - g.e0] = reinterpret_cast<const uint16_t*>(row)[e];
-                else
-                    reinterpret_cast<float*>(buf)[e - g.e0] = reinterpret_cast<const float*>(row)[e];
-            }
-        }
-        mbar_arrive_expect_tx(&S.mbar[st], bytes + P.test_extra_tx);
-        if (bytes) bulk_g2s(buf + (g.ga16 - g.A0), reinterpret_cast<const void*>(g.ga16), bytes, &S.mbar[st]);
-    };
 
     if (tid == 0) {
-        for (int st = 0; st < P.stages; ++st) mbar_init(&S.mbar[st], 1);
+        for (int st = 0; st < P.stages; ++st) {
+            mbar_init(&S.full[st], 1);
+            mbar_init(&S.empty[st], NW);
+        }
         fence_mbar_init();
-        S.theta = NEG_INF;
-        S.cnt = 0;
-        S.overflow = 0;
+        S.issued = 0;
+        S.tmo = 0;
+        S.diag = 0;
     }
+    if (tid < MAX_CONSUMER_WARPS) S.wbound[tid] = NEG_INF;
     __syncthreads();
-    if (tid == 0) {
-        for (int t = 0; t < min(P.stages, ntiles); ++t) issue(t);
-    }
 
-    float run = NEG_INF;     // running NaN-propagating maximum of this thread's elements
-    float wbest = NEG_INF;   // greedy: best value of this warp and its lowest index
-    int widx = -1;
-    // top-k bound.  Each warp sorts its lanes' running maxima (bitonic network
-    // in registers) and takes the rsel-th largest, rsel = ceil(K / warps): that
-    // warp holds rsel distinct elements at or above it, so the minimum over the
-    // warps has at least K elements at or above it and is <= the chunk's K-th
-    // largest logit.
-    const int rsel = (K + NW - 1) / NW;  // <= 32 (K <= threads on this path)
-    auto warp_bound = [&]() -> float {
-        float x = run == run ? run : NEG_INF;
-#pragma unroll
-        for (int k2 = 2; k2 <= 32; k2 <<= 1) {
-#pragma unroll
-            for (int j2 = k2 >> 1; j2 > 0; j2 >>= 1) {
-                const float y = __shfl_xor_sync(0xffffffffu, x, j2);
-                const bool desc = (lane & k2) == 0;
-                const bool lower = (lane & j2) == 0;
-                x = (lower == desc) ? fmaxf(x, y) : fminf(x, y);
-            }
-        }
-        return __shfl_sync(0xffffffffu, x, rsel - 1);
-    };
-    auto min_bound = [&](int slot) {
-        float mn = S.wsel[slot][0];
-        for (int w = 1; w < NW; ++w) mn = fminf(mn, S.wsel[slot][w]);
-        return mn;
-    };
-    float theta = NEG_INF;  // this thread's copy of the running bound
-
-    int tmo = 0;
-    int t = 0;
-    for (; t < ntiles; ++t) {
-        const int st = t % P.stages;
-        const uint32_t parity = static_cast<uint32_t>((t / P.stages) & 1);
-        const TileGeom g = geom(t);
-        const unsigned char* buf = ring + static_cast<size_t>(st) * P.stage_bytes;
-        const bool ok = mbar_wait_bounded(&S.mbar[st], parity, P.timeout_ns);
-        auto valid = [&](int e) { return e >= g.lo && e < g.hi; };
-        auto vec_at = [&](int j) { return *reinterpret_cast<const uint4*>(buf + 16 * j); };
-        // NaN-propagating maximum of the valid elements of vector j
-        auto vmax_masked = [&](int j) -> float {
-            const uint4 raw = vec_at(j);
-            const int e = g.e0 + j * VEC;
-            if (e >= g.lo && e + VEC <= g.hi) return vmax_nan<DT>(raw);
-            float v[VEC];
-            unpack<DT>(raw, v);
-            float vm = NEG_INF;
-#pragma unroll
-            for (int q = 0; q < VEC; ++q)
-                if (valid(e + q)) vm = fmax_nan(vm, v[q]);
-            return vm;
-        };
-        // valid elements of vector j (others -inf)
-        auto load_masked = [&](int j, float* v) {
-            unpack<DT>(vec_at(j), v);
-            const int e = g.e0 + j * VEC;
-            if (!(e >= g.lo && e + VEC <= g.hi)) {
-#pragma unroll
-                for (int q = 0; q < VEC; ++q)
-                    if (!valid(e + q)) v[q] = NEG_INF;
-            }
-        };
-
-        // pass A (no stores): every vector maximum of this thread's share of the
-        // tile.  Slot VPT is the one vector past TV that a segment starting off
-        // a 16-byte boundary spans (vector TV + tid, present for tid == 0 only).
-        auto jof = [&](int i) { return i < VPT ? tid + i * NT : TV + tid; };
-        float vm[VPT + 1];
-        const bool tile_full = ok && g.e0 == g.lo && g.nvec == TV && g.hi - g.lo == TV * VEC;
-        if (tile_full) {
-#pragma unroll
-            for (int i = 0; i < VPT; ++i) vm[i] = vmax_nan<DT>(vec_at(tid + i * NT));
-            vm[VPT] = NEG_INF;
-        } else {
-#pragma unroll
-            for (int i = 0; i <= VPT; ++i) {
-                const int j = jof(i);
-                vm[i] = (ok && j < g.nvec) ? vmax_masked(j) : NEG_INF;
-            }
-        }
-        float tm = vm[0];
-#pragma unroll
-        for (int i = 1; i <= VPT; ++i) tm = fmax_nan(tm, vm[i]);
-
-        if constexpr (MODE == MODE_GREEDY) {
-            run = fmax_nan(run, tm);
-            float wtm = tm != tm ? NEG_INF : tm;  // NaN is reported through run
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) wtm = fmaxf(wtm, __shfl_xor_sync(0xffffffffu, wtm, o));
-            if (wtm > wbest) {  // warp-uniform, rare after the first tiles
-                int my = INT_MAX;
-#pragma unroll
-                for (int i = 0; i <= VPT; ++i) {
-                    const int j = jof(i);
-                    if (my == INT_MAX && vm[i] == wtm) {
-                        float v[VEC];
-                        load_masked(j, v);
-                        const int e = g.e0 + j * VEC;
-#pragma unroll
-                        for (int q = VEC - 1; q >= 0; --q)
-                            if (v[q] == wtm) my = e + q;
+    if (warp == NW) {
+        // ================= producer: lane 0 fills the ring =================
+        if (lane == 0) {
+            int t = 0;
+            for (; t < ntiles; ++t) {
+                const int st = t % P.stages;
+                if (*reinterpret_cast<volatile int*>(&S.tmo)) break;
+                if (t >= P.stages &&
+                    !mbar_wait_bounded(&S.empty[st], static_cast<uint32_t>((t / P.stages - 1) & 1), P.timeout_ns)) {
+                    atomicOr(&S.tmo, 1);
+                    break;
+                }
+                const TileGeom g = geom(t);
+                unsigned char* buf = ring + static_cast<size_t>(st) * STAGE_BYTES;
+                uint32_t bytes = 0;
+                int nh = 0, ntl = 0;
+                if (g.hi > g.lo) {
+                    if (g.ga16 >= g.gb16) {
+                        nh = g.hi - g.lo;
+                    } else {
+                        nh = static_cast<int>((g.ga16 - g.ga) / ELT);
+                        ntl = static_cast<int>((g.gb - g.gb16) / ELT);
+                        bytes = static_cast<uint32_t>(g.gb16 - g.ga16);
                     }
                 }
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) my = min(my, __shfl_xor_sync(0xffffffffu, my, o));
-                wbest = wtm;
-                widx = my;
+                // self-check: a 16-byte aligned copy that stays inside its stage
+                const uintptr_t doff = g.ga16 - g.A0;
+                if (bytes != 0 &&
+                    ((((reinterpret_cast<uintptr_t>(buf) + doff) | g.ga16 | bytes) & 15u) != 0 ||
+                     doff + bytes > static_cast<uintptr_t>(STAGE_BYTES))) {
+                    atomicOr(&S.diag, 1);
+                    bytes = 0;
+                    nh = ntl = 0;
+                }
+                // elements outside the aligned interior: plain loads, published by the arrive
+                for (int q = 0; q < nh + ntl; ++q) {
+                    const int e = q < nh ? g.lo + q : g.hi - ntl + (q - nh);
+                    if constexpr (DT == 0)
+                        reinterpret_cast<uint16_t*>(buf)[e - g.e0] = reinterpret_cast<const uint16_t*>(row)[e];
+                    else
+                        reinterpret_cast<float*>(buf)[e - g.e0] = reinterpret_cast<const float*>(row)[e];
+                }
+                mbar_arrive_expect_tx(&S.full[st], bytes + P.test_extra_tx);
+                if (bytes) bulk_g2s(buf + doff, reinterpret_cast<const void*>(g.ga16), bytes, &S.full[st]);
             }
-        } else if constexpr (MODE == MODE_SOFTMAX) {
-            // one maximum per warp; pass B sums 2^(z*c - m) with two accumulators
-            float wtm = tm;
+            S.issued = t;
+        }
+        __syncwarp();
+    } else {
+        // ================= consumers =================
+        float run = NEG_INF;    // running NaN-propagating maximum of this thread's elements
+        float wbest = NEG_INF;  // greedy: best value of this warp and its lowest index
+        int widx = -1;
+        const int rsel = (K + NW - 1) / NW;  // <= 32 on the top-k path (K <= NT)
+        float* const wkey = lkey + warp * wcap;
+        int* const widxs = lidx + warp * wcap;
+        int wcnt = 0;       // entries in this warp's segment (warp-uniform)
+        bool wovf = false;  // the segment lost entries
+        float theta = NEG_INF;
+        float pub = NEG_INF;  // this warp's last published bound
+        // rsel-th largest of the lanes' running maxima
+        auto lane_bound = [&]() -> float {
+            float x = run == run ? run : NEG_INF;
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) wtm = fmax_nan(wtm, __shfl_xor_sync(0xffffffffu, wtm, o));
-            const float m = wtm * cscale;
-            float s0 = 0.f, s1 = 0.f;
-            if (ok && m > NEG_INF && m < POS_INF) {
+            for (int k2 = 2; k2 <= 32; k2 <<= 1) {
+#pragma unroll
+                for (int j2 = k2 >> 1; j2 > 0; j2 >>= 1) {
+                    const float y = __shfl_xor_sync(0xffffffffu, x, j2);
+                    const bool desc = (lane & k2) == 0;
+                    const bool lower = (lane & j2) == 0;
+                    x = (lower == desc) ? fmaxf(x, y) : fminf(x, y);
+                }
+            }
+            return __shfl_sync(0xffffffffu, x, rsel - 1);
+        };
+        auto publish = [&](float v) {
+            if (v > pub) {
+                pub = v;
+                if (lane == 0) *reinterpret_cast<volatile float*>(&S.wbound[warp]) = v;
+            }
+        };
+        auto read_bound = [&]() {
+            float mn = *reinterpret_cast<volatile float*>(&S.wbound[0]);
+#pragma unroll
+            for (int w = 1; w < NW; ++w) mn = fminf(mn, *reinterpret_cast<volatile float*>(&S.wbound[w]));
+            return mn;
+        };
+        // Segment full: sort it, publish its rsel-th largest entry, keep the
+        // entries >= the freshest bound.
+        auto compact = [&]() {
+            const int np2 = pow2_ceil(wcnt < 2 ? 2 : wcnt);
+            for (int q = wcnt + lane; q < np2; q += 32) {
+                wkey[q] = NEG_INF;
+                widxs[q] = INT_MAX;
+            }
+            __syncwarp();
+            warp_sort_desc(wkey, widxs, np2, lane);
+            if (wcnt >= rsel) publish(wkey[rsel - 1]);
+            theta = fmaxf(theta, read_bound());
+            int keep = 0;
+            for (int q0 = 0; q0 < wcnt; q0 += 32) {
+                const bool ge = q0 + lane < wcnt && wkey[q0 + lane] >= theta;
+                keep += __popc(__ballot_sync(0xffffffffu, ge));
+            }
+            wcnt = keep;  // sorted descending: the kept entries are the prefix
+        };
+
+        for (int t = 0; t < ntiles; ++t) {
+            const int st = t % P.stages;
+            const TileGeom g = geom(t);
+            const unsigned char* buf = ring + static_cast<size_t>(st) * STAGE_BYTES;
+            const bool ok = mbar_wait_bounded(&S.full[st], static_cast<uint32_t>((t / P.stages) & 1), P.timeout_ns);
+            if (!ok && lane == 0) atomicOr(&S.tmo, 1);
+            auto valid = [&](int e) { return e >= g.lo && e < g.hi; };
+            auto vec_at = [&](int j) { return *reinterpret_cast<const uint4*>(buf + 16 * j); };
+            auto vmax_masked = [&](int j) -> float {
+                const uint4 raw = vec_at(j);
+                const int e = g.e0 + j * VEC;
+                if (e >= g.lo && e + VEC <= g.hi) return vmax_nan<DT>(raw);
+                float v[VEC];
+                unpack<DT>(raw, v);
+                float vm = NEG_INF;
+#pragma unroll
+                for (int q = 0; q < VEC; ++q)
+                    if (valid(e + q)) vm = fmax_nan(vm, v[q]);
+                return vm;
+            };
+            auto load_masked = [&](int j, float* v) {
+                unpack<DT>(vec_at(j), v);
+                const int e = g.e0 + j * VEC;
+                if (!(e >= g.lo && e + VEC <= g.hi)) {
+#pragma unroll
+                    for (int q = 0; q < VEC; ++q)
+                        if (!valid(e + q)) v[q] = NEG_INF;
+                }
+            };
+            // this thread's vectors: slot i < VPT is vector tid + i*NT; slot VPT
+            // is the one vector past TV that a segment starting off a 16-byte
+            // boundary spans (vector TV + tid, tid == 0 only)
+            auto jof = [&](int i) { return i < VPT ? tid + i * NT : TV + tid; };
+            float vm[VPT + 1];
+            const bool tile_full = ok && g.e0 == g.lo && g.nvec == TV && g.hi - g.lo == TV * VEC;
+            if (tile_full) {
+#pragma unroll
+                for (int i = 0; i < VPT; ++i) vm[i] = vmax_nan<DT>(vec_at(tid + i * NT));
+                vm[VPT] = NEG_INF;
+            } else {
 #pragma unroll
                 for (int i = 0; i <= VPT; ++i) {
                     const int j = jof(i);
-                    if (j < g.nvec) {
-                        float v[VEC];
-                        load_masked(j, v);
+                    vm[i] = (ok && j < g.nvec) ? vmax_masked(j) : NEG_INF;
+                }
+            }
+            float tm = vm[0];
 #pragma unroll
-                        for (int q = 0; q < VEC; q += 2) {
-                            s0 += ex2(fmaf(v[q], cscale, -m));
-                            s1 += ex2(fmaf(v[q + 1], cscale, -m));
+            for (int i = 1; i <= VPT; ++i) tm = fmax_nan(tm, vm[i]);
+
+            if constexpr (MODE == MODE_GREEDY) {
+                run = fmax_nan(run, tm);
+                float wtm = tm != tm ? NEG_INF : tm;  // NaN is reported through run
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) wtm = fmaxf(wtm, __shfl_xor_sync(0xffffffffu, wtm, o));
+                if (wtm > wbest) {  // warp-uniform, rare after the first tiles
+                    int my = INT_MAX;
+#pragma unroll
+                    for (int i = 0; i <= VPT; ++i) {
+                        const int j = jof(i);
+                        if (my == INT_MAX && vm[i] == wtm) {
+                            float v[VEC];
+                            load_masked(j, v);
+                            const int e = g.e0 + j * VEC;
+#pragma unroll
+                            for (int q = VEC - 1; q >= 0; --q)
+                                if (v[q] == wtm) my = e + q;
+                        }
+                    }
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) my = min(my, __shfl_xor_sync(0xffffffffu, my, o));
+                    wbest = wtm;
+                    widx = my;
+                }
+            } else if constexpr (MODE == MODE_SOFTMAX) {
+                // one maximum per warp; pass B sums 2^(z*c - m) with two accumulators
+                float wtm = tm;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) wtm = fmax_nan(wtm, __shfl_xor_sync(0xffffffffu, wtm, o));
+                const float m = wtm * cscale;
+                float sa = 0.f, sb = 0.f;
+                if (ok && m > NEG_INF && m < POS_INF) {
+#pragma unroll
+                    for (int i = 0; i <= VPT; ++i) {
+                        const int j = jof(i);
+                        if (j < g.nvec) {
+                            float v[VEC];
+                            load_masked(j, v);
+#pragma unroll
+                            for (int q = 0; q < VEC; q += 2) {
+                                sa += ex2(fmaf(v[q], cscale, -m));
+                                sb += ex2(fmaf(v[q + 1], cscale, -m));
+                            }
                         }
                     }
                 }
-            }
-            const float ws = warp_sum(s0 + s1);
-            if (lane == 0) {
-                red_m[t * NW + warp] = m;
-                red_s[t * NW + warp] = ws;
-            }
-        } else if constexpr (MODE == MODE_TOPK) {
-            run = fmax_nan(run, tm);
-            if (t == 0) {
-                // first tile: a bound from the tile itself before any append
-                const float wb = warp_bound();
-                if (lane == 0) S.wsel[2][warp] = wb;
-                __syncthreads();
-                theta = fmaxf(theta, min_bound(2));
-            }
-            const float th = theta;
-            // pass B: the elements >= th, appended warp by warp (rare)
+                const float ws = warp_sum(sa + sb);
+                if (lane == 0) {
+                    red_m[t * NW + warp] = m;
+                    red_s[t * NW + warp] = ws;
+                }
+            } else if constexpr (MODE == MODE_TOPK) {
+                run = fmax_nan(run, tm);
+                if (t == 0) {
+                    // every warp publishes a bound from the first tile before any append
+                    publish(lane_bound());
+                    consumer_sync<NT>();
+                } else if (t & 1) {
+                    publish(lane_bound());
+                }
+                theta = fmaxf(theta, read_bound());
+                // pass B: this tile's elements >= theta go to the warp's segment
+                unsigned cm = 0u;
 #pragma unroll
-            for (int i = 0; i <= VPT; ++i) {
-                const bool cand = ok && vm[i] >= th;
-                if (__any_sync(0xffffffffu, cand)) {
-                    const int j = jof(i);
-                    const int e = g.e0 + j * VEC;
-                    float v[VEC];
-                    unsigned mask = 0u;
-                    if (cand) {
-                        load_masked(j, v);
+                for (int i = 0; i <= VPT; ++i)
+                    if (ok && vm[i] >= theta) cm |= 1u << i;
+                if (__any_sync(0xffffffffu, cm != 0u)) {
+                    auto count = [&](float th) {
+                        int n = 0;
 #pragma unroll
-                        for (int q = 0; q < VEC; ++q)
-                            if (v[q] >= th) mask |= 1u << q;
-                    }
-                    const int cnt = __popc(mask);
+                        for (int i = 0; i <= VPT; ++i) {
+                            if ((cm >> i) & 1u) {
+                                float v[VEC];
+                                load_masked(jof(i), v);
+#pragma unroll
+                                for (int q = 0; q < VEC; ++q) n += v[q] >= th;
+                            }
+                        }
+                        return n;
+                    };
+                    int cnt = count(theta);
                     int incl = cnt;
 #pragma unroll
                     for (int o = 1; o < 32; o <<= 1) {
                         const int y = __shfl_up_sync(0xffffffffu, incl, o);
                         if (lane >= o) incl += y;
                     }
-                    const int total = __shfl_sync(0xffffffffu, incl, 31);
-                    int base = 0;
-                    if (lane == 0) base = atomicAdd(&S.cnt, total);
-                    base = __shfl_sync(0xffffffffu, base, 0);
-                    int p = base + incl - cnt;
+                    int total = __shfl_sync(0xffffffffu, incl, 31);
+                    if (wcnt + total > wcap && !wovf) {
+                        compact();
+                        cnt = count(theta);
+                        incl = cnt;
 #pragma unroll
-                    for (int q = 0; q < VEC; ++q) {
-                        if ((mask >> q) & 1u) {
-                            if (p < P.lcap) {
-                                lkey[p] = v[q];
-                                lidx[p] = e + q;
-                            } else {
-                                S.overflow = 1;
+                        for (int o = 1; o < 32; o <<= 1) {
+                            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                            if (lane >= o) incl += y;
+                        }
+                        total = __shfl_sync(0xffffffffu, incl, 31);
+                    }
+                    int p = wcnt + incl - cnt;
+#pragma unroll
+                    for (int i = 0; i <= VPT; ++i) {
+                        if ((cm >> i) & 1u) {
+                            const int j = jof(i);
+                            const int e = g.e0 + j * VEC;
+                            float v[VEC];
+                            load_masked(j, v);
+#pragma unroll
+                            for (int q = 0; q < VEC; ++q) {
+                                if (v[q] >= theta) {
+                                    if (p < wcap) {
+                                        wkey[p] = v[q];
+                                        widxs[p] = e + q;
+                                    }
+                                    ++p;
+                                }
                             }
-                            ++p;
                         }
                     }
+                    if (wcnt + total > wcap) wovf = true;
+                    wcnt = min(wcnt + total, wcap);
                 }
+            } else {
+                run = fmax_nan(run, tm);  // MODE_MAXONLY
             }
-            // publish this tile's warp bounds; read after the tile barrier
-            const float wb = warp_bound();
-            if (lane == 0) S.wsel[t & 1][warp] = wb;
-        } else {
-            run = fmax_nan(run, tm);  // MODE_MAXONLY
+
+            // hand the stage back to the producer
+            __syncwarp();
+            if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&S.empty[st])) : "memory");
+            if (!ok) break;
         }
 
-        tmo = __syncthreads_or(!ok);  // every thread is done with the stage
-        if (tid == 0 && !tmo && t + P.stages < ntiles) issue(t + P.stages);
-        if (tmo) break;
-        if constexpr (MODE == MODE_TOPK) theta = fmaxf(theta, min_bound(t & 1));
-
+        // ---- per-warp results ------------------------------------------------------
+        if constexpr (MODE != MODE_SOFTMAX) {
+            const float wm = warp_max_nan(run);
+            if (lane == 0) {
+                S.wmax[warp] = wm;
+                S.wbest[warp] = wbest;
+                S.widx[warp] = widx;
+            }
+        }
         if constexpr (MODE == MODE_TOPK) {
-            // Compact the candidate list when it is half full (rare).  The
-            // decision is taken from a snapshot that every thread reads
-            // between two barriers: without the second one a fast warp could
-            // append the next tile's candidates before a slow warp reads the
-            // count, and the warps would disagree about entering the
-            // compaction (and its barriers).
-            const int cnt_now = S.cnt;
-            const int ovf_now = S.overflow;
-            __syncthreads();
-            if (cnt_now > (P.lcap >> 1) && !ovf_now) {
-                const int n = cnt_now;
-                const int N = pow2_ceil(n);
-                for (int q = n + tid; q < N; q += NT) {
-                    lkey[q] = NEG_INF;
-                    lidx[q] = INT_MAX;
-                }
-                __syncthreads();
-                block_sort<true>(lkey, lidx, N);
-                const float th2 = fmaxf(theta, lkey[K - 1]);
-                __syncthreads();
-                if (tid == 0) {
-                    int m = K;
-                    while (m < n && lkey[m] >= th2) ++m;
-                    S.cnt = m;
-                }
-                theta = th2;
-                __syncthreads();
+            publish(lane_bound());  // from every element of the chunk
+            if (lane == 0) {
+                S.wcnt[warp] = wcnt;
+                S.wovf[warp] = wovf ? 1 : 0;
             }
         }
     }
+    __syncthreads();  // every tile is consumed (or a wait ran out)
+
+    const int tmo = S.tmo;
+    const int diag = S.diag;
+    const int bad = tmo | diag;
+    const int flag = (tmo ? REC_TIMEOUT : 0) | (diag ? REC_DIAG : 0);
 
     // ---- partial records ------------------------------------------------------------
     if constexpr (MODE == MODE_SOFTMAX) {
-        // one per segment
-        for (int q = tid; q < ntiles; q += NT) {
+        for (int q = tid; q < ntiles; q += NTH) {
             SegRec rec;
             rec.arg = -1;
-            rec.flags = 0;
-            if (tmo && q >= t) {  // the tile whose wait ran out, and every later one
+            rec.flags = flag;
+            if (bad) {
                 rec.m = __int_as_float(0x7fc00000);
                 rec.s = 0.f;
-                rec.flags = REC_TIMEOUT;
             } else {
                 float m = red_m[q * NW], sm = red_s[q * NW];
                 for (int w = 1; w < NW; ++w) ms_combine(m, sm, red_m[q * NW + w], red_s[q * NW + w]);
@@ -441,180 +553,185 @@ __global__ void __launch_bounds__(NT, 1024 / NT) sv_rows_kernel(const RowsParams
             P.segs[r * P.nseg + s0 + q] = rec;
         }
     } else if constexpr (MODE == MODE_GREEDY || MODE == MODE_MAXONLY) {
-        // one per chunk, stored in slot c of the row
-        run = warp_max_nan(run);
-        if (lane == 0) {
-            red_m[warp] = run;
-            red_s[warp] = wbest;
-            red_i[warp] = widx;
-        }
-        __syncthreads();
         if (tid == 0) {
             SegRec rec;
-            rec.m = red_m[0];
+            rec.m = S.wmax[0];
             rec.s = 0.f;
-            float bv = red_s[0];
-            int bi = red_i[0];
+            float bv = S.wbest[0];
+            int bi = S.widx[0];
             for (int w = 1; w < NW; ++w) {
-                rec.m = fmax_nan(rec.m, red_m[w]);
-                if (arg_better(red_s[w], red_i[w], bv, bi)) {
-                    bv = red_s[w];
-                    bi = red_i[w];
+                rec.m = fmax_nan(rec.m, S.wmax[w]);
+                if (arg_better(S.wbest[w], S.widx[w], bv, bi)) {
+                    bv = S.wbest[w];
+                    bi = S.widx[w];
                 }
             }
             rec.arg = MODE == MODE_GREEDY ? bi : -1;
-            rec.flags = tmo ? REC_TIMEOUT : 0;
-            if (tmo) rec.m = __int_as_float(0x7fc00000);
+            rec.flags = flag;
+            if (bad) rec.m = __int_as_float(0x7fc00000);
             P.segs[r * P.nseg + c] = rec;
         }
     }
 
-    if (tmo) {
+    if (bad) {
         if (tid == 0) {
             if constexpr (MODE == MODE_TOPK) {
                 ChunkRec ch;
                 ch.tau = NEG_INF;
                 ch.last = NEG_INF;
                 ch.n = 0;
-                ch.flags = REC_TIMEOUT;
+                ch.flags = flag;
                 ch.m = __int_as_float(0x7fc00000);
                 ch.s = 0.f;
                 ch.zd = NEG_INF;
                 ch.pad = 0;
                 P.chunks[r * P.nch + c] = ch;
             }
-            // wait (bounded) for copies still in flight before the CTA exits
-            for (int q = t; q < min(ntiles, t + P.stages); ++q)
-                mbar_wait_bounded(&S.mbar[q % P.stages], static_cast<uint32_t>((q / P.stages) & 1), P.timeout_ns);
-        }
-        return;
-    }
-    if constexpr (MODE != MODE_TOPK) {
-        return;
-    } else {
-
-    // ---- top-k: exact K-th largest of the chunk and its kept entries ----------
-    const float mrow = warp_max_nan(run);  // chunk maximum (NaN-propagating)
-    const float wbf = warp_bound();        // final bound from every element
-    if (lane == 0) {
-        S.wzd[warp] = mrow;
-        S.wsel[2][warp] = wbf;
-    }
-    __syncthreads();
-    const float thf = fmaxf(theta, min_bound(2));
-    float cmax = S.wzd[0];
-    for (int w = 1; w < NW; ++w) cmax = fmax_nan(cmax, S.wzd[w]);
-    const int n0 = min(S.cnt, P.lcap);
-    const int ovf = S.overflow;
-    const int d = (pos < P.k && P.draft_tokens) ? P.draft_tokens[b * P.k + pos] : -1;
-    // filtered copy of the list (entries >= the final bound) in the free ring
-    Cand* fl = reinterpret_cast<Cand*>(ring);
-    const int fcap = (P.stages * P.stage_bytes) / static_cast<int>(sizeof(Cand));
-    if (tid == 0) S.cnt2 = 0;
-    __syncthreads();
-    for (int q = tid; q < n0; q += NT) {
-        if (lkey[q] >= thf) {
-            const int p = atomicAdd(&S.cnt2, 1);
-            if (p < fcap) fl[p] = Cand{lkey[q], lidx[q]};
-        }
-    }
-    if (tid == 0) {
-        S.nkept = 0;
-        S.tau = NEG_INF;
-    }
-    __syncthreads();
-    const int n2 = S.cnt2;
-    Cand* out = P.cands + (r * P.nch + c) * static_cast<long long>(P.kcap);
-    float lastv = NEG_INF;
-    int nk;
-    if (n2 <= RANK_MAX && n2 <= fcap) {
-        // rank by (value desc, index asc): tau is the value at rank K-1
-        for (int q = tid; q < n2; q += NT) {
-            const Cand e = fl[q];
-            int rk = 0;
-            for (int f = 0; f < n2; ++f) {
-                const Cand o = fl[f];
-                rk += (o.v > e.v) || (o.v == e.v && o.i < e.i);
+            // wait (bounded) for the last copy issued into each stage
+            const int issued = S.issued;
+            for (int q = 0; q < min(issued, P.stages); ++q) {
+                const int last = q + ((issued - 1 - q) / P.stages) * P.stages;
+                mbar_wait_bounded(&S.full[q], static_cast<uint32_t>((last / P.stages) & 1), P.timeout_ns);
             }
-            if (rk == K - 1) S.tau = e.v;
+        }
+        return;
+    }
+    if constexpr (MODE == MODE_TOPK) {
+        // ---- exact K-th largest of the chunk and its kept entries -----------------
+        float cmax = S.wmax[0];
+        float thf = S.wbound[0];
+        int ovf = S.wovf[0];
+        for (int w = 1; w < NW; ++w) {
+            cmax = fmax_nan(cmax, S.wmax[w]);
+            thf = fminf(thf, S.wbound[w]);
+            ovf |= S.wovf[w];
+        }
+        const int d = (pos < P.k && P.draft_tokens) ? P.draft_tokens[b * P.k + pos] : -1;
+        // entries >= the final bound, copied from the warp segments into the free ring
+        Cand* fl = reinterpret_cast<Cand*>(ring);
+        const int fcap = (P.stages * STAGE_BYTES) / static_cast<int>(sizeof(Cand));
+        if (tid == 0) {
+            S.cnt2 = 0;
+            S.nkept = 0;
+            S.tau = NEG_INF;
         }
         __syncthreads();
-        const float tau = n2 >= K ? S.tau : NEG_INF;
-        for (int q = tid; q < n2; q += NT) {
-            const Cand e = fl[q];
-            if (!(e.v >= tau)) continue;
-            int ri = 0;
-            for (int f = 0; f < n2; ++f) ri += (fl[f].v >= tau && fl[f].i < e.i);
-            atomicAdd(&S.nkept, 1);
-            if (ri < P.kcap) out[ri] = e;
+        if (warp < NW) {
+            const int n = S.wcnt[warp];
+            const float* wk = lkey + warp * wcap;
+            const int* wi = lidx + warp * wcap;
+            for (int q0 = 0; q0 < n; q0 += 32) {
+                const int q = q0 + lane;
+                const bool ge = q < n && wk[q] >= thf;
+                const unsigned m = __ballot_sync(0xffffffffu, ge);
+                int base = 0;
+                if (lane == 0 && m) base = atomicAdd(&S.cnt2, __popc(m));
+                base = __shfl_sync(0xffffffffu, base, 0);
+                const int p = base + __popc(m & ((1u << lane) - 1u));
+                if (ge && p < fcap) fl[p] = Cand{wk[q], wi[q]};
+            }
         }
         __syncthreads();
-        nk = S.nkept;
-        if (tid == 0) S.tau = tau;
-        lastv = tau;  // every kept entry is >= tau
-    } else {
-        // large lists: sort the unfiltered list by value
-        const int N = pow2_ceil(n0 < 2 ? 2 : n0);
-        for (int q = n0 + tid; q < N; q += NT) {
-            lkey[q] = NEG_INF;
-            lidx[q] = INT_MAX;
+        const int n2 = S.cnt2;
+        // kept entries, index-sorted, staged in shared memory: in the (now free)
+        // segment area after ranking, in the ring after sorting
+        Cand* ks = reinterpret_cast<Cand*>(lkey);
+        const int kscap = P.lcap;
+        Cand* out = P.cands + (r * P.nch + c) * static_cast<long long>(P.kcap);
+        float lastv = NEG_INF;
+        int nk;
+        if (n2 <= RANK_MAX) {
+            // rank by (value desc, index asc): tau is the value at rank K-1
+            for (int q = tid; q < n2; q += NTH) {
+                const Cand e = fl[q];
+                int rk = 0;
+                for (int f = 0; f < n2; ++f) {
+                    const Cand o = fl[f];
+                    rk += (o.v > e.v) || (o.v == e.v && o.i < e.i);
+                }
+                if (rk == K - 1) S.tau = e.v;
+            }
+            __syncthreads();
+            const float tau = n2 >= K ? S.tau : NEG_INF;
+            for (int q = tid; q < n2; q += NTH) {
+                const Cand e = fl[q];
+                if (!(e.v >= tau)) continue;
+                int ri = 0;
+                for (int f = 0; f < n2; ++f) ri += (fl[f].v >= tau && fl[f].i < e.i);
+                atomicAdd(&S.nkept, 1);
+                if (ri < kscap) ks[ri] = e;
+            }
+            __syncthreads();
+            nk = S.nkept;
+            lastv = tau;  // every kept entry is >= tau
+        } else {
+            // large lists: sort by value, cut at rank K (with ties), sort the cut by index
+            const int n0 = min(n2, min(fcap, P.lcap));
+            float* sk = lkey;
+            int* si = lidx;
+            const int N = pow2_ceil(n0 < 2 ? 2 : n0);
+            for (int q = tid; q < N; q += NTH) {
+                sk[q] = q < n0 ? fl[q].v : NEG_INF;
+                si[q] = q < n0 ? fl[q].i : INT_MAX;
+            }
+            __syncthreads();
+            block_sort<true>(sk, si, N);
+            const float tau = (n0 >= K) ? sk[K - 1] : NEG_INF;
+            for (int q = tid; q < n0; q += NTH)
+                if (sk[q] >= tau && (q + 1 == n0 || !(sk[q + 1] >= tau))) S.nkept = q + 1;
+            __syncthreads();
+            nk = S.nkept;
+            const int m = min(nk, P.kcap);
+            lastv = m > 0 ? sk[m - 1] : NEG_INF;
+            const int M2 = pow2_ceil(m < 2 ? 2 : m);
+            for (int q = m + tid; q < M2; q += NTH) {
+                sk[q] = NEG_INF;
+                si[q] = INT_MAX;
+            }
+            __syncthreads();
+            block_sort<false>(sk, si, M2);
+            ks = fl;  // the ring was copied out before the sorts (m <= kcap < fcap)
+            for (int q = tid; q < m; q += NTH) ks[q] = Cand{sk[q], si[q]};
+            if (tid == 0) S.tau = tau;
+            if (n2 > fcap || n2 > P.lcap) ovf = 1;
+            __syncthreads();
         }
-        __syncthreads();
-        block_sort<true>(lkey, lidx, N);
-        const float tau = (n0 >= K) ? lkey[K - 1] : NEG_INF;
-        for (int q = tid; q < n0; q += NT)
-            if (lkey[q] >= tau && (q + 1 == n0 || !(lkey[q + 1] >= tau))) S.nkept = q + 1;
-        __syncthreads();
-        nk = S.nkept;
+        // exp-sum and draft-token logit over the stored (index-sorted) entries
         const int m = min(nk, P.kcap);
-        lastv = m > 0 ? lkey[m - 1] : NEG_INF;
-        const int M2 = pow2_ceil(m < 2 ? 2 : m);
-        for (int q = m + tid; q < M2; q += NT) {
-            lkey[q] = NEG_INF;
-            lidx[q] = INT_MAX;
+        const float msc = cmax * cscale;
+        float acc = 0.f, zd = NEG_INF;
+        for (int q = tid; q < m; q += NTH) {
+            const Cand e = ks[q];
+            out[q] = e;
+            acc += ex2(fmaf(e.v, cscale, -msc));
+            if (e.i == d) zd = e.v;
         }
-        __syncthreads();
-        block_sort<false>(lkey, lidx, M2);
-        for (int q = tid; q < m; q += NT) out[q] = Cand{lkey[q], lidx[q]};
-        if (tid == 0) S.tau = tau;
-        __syncthreads();
-    }
-    // maximum, exp-sum and draft-token logit over the stored (index-sorted) entries
-    const int m = min(nk, P.kcap);
-    __syncthreads();
-    const float msc = cmax * cscale;
-    float acc = 0.f, zd = NEG_INF;
-    for (int q = tid; q < m; q += NT) {
-        const Cand e = out[q];
-        acc += ex2(fmaf(e.v, cscale, -msc));
-        if (e.i == d) zd = e.v;
-    }
-    acc = warp_sum(acc);
+        acc = warp_sum(acc);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) zd = fmaxf(zd, __shfl_xor_sync(0xffffffffu, zd, o));
-    if (lane == 0) {
-        S.wsum[warp] = acc;
-        S.wzd[warp] = zd;
-    }
-    __syncthreads();
-    if (tid == 0) {
-        float s = 0.f, z = NEG_INF;
-        for (int w = 0; w < NW; ++w) {
-            s += S.wsum[w];
-            z = fmaxf(z, S.wzd[w]);
+        for (int o = 16; o > 0; o >>= 1) zd = fmaxf(zd, __shfl_xor_sync(0xffffffffu, zd, o));
+        if (lane == 0) {
+            S.wsum[warp] = acc;
+            S.wzd[warp] = zd;
         }
-        ChunkRec ch;
-        ch.tau = S.tau;
-        ch.last = lastv;
-        ch.n = m;
-        ch.flags = (ovf || nk > P.kcap || n2 > fcap) ? REC_OVERFLOW : 0;
-        ch.m = cmax;
-        ch.s = s;
-        ch.zd = z;
-        ch.pad = 0;
-        P.chunks[r * P.nch + c] = ch;
+        __syncthreads();
+        if (tid == 0) {
+            float s = 0.f, z = NEG_INF;
+            for (int w = 0; w <= NW; ++w) {
+                s += S.wsum[w];
+                z = fmaxf(z, S.wzd[w]);
+            }
+            ChunkRec ch;
+            ch.tau = S.tau;
+            ch.last = lastv;
+            ch.n = m;
+            ch.flags = (ovf || nk > P.kcap) ? REC_OVERFLOW : 0;
+            ch.m = cmax;
+            ch.s = s;
+            ch.zd = z;
+            ch.pad = 0;
+            P.chunks[r * P.nch + c] = ch;
+        }
     }
-    }  // MODE_TOPK
 }
 
 }  // namespace sv
