@@ -118,6 +118,15 @@ __device__ __forceinline__ TileGeom tile_geom(const char* row, int lo, int hi) {
     return g;
 }
 
+// Element `el` of a ring stage (raw logit as fp32).
+template <int DT>
+__device__ __forceinline__ float smem_elem(const unsigned char* buf, int el) {
+    if constexpr (DT == 0)
+        return __uint_as_float(static_cast<uint32_t>(reinterpret_cast<const uint16_t*>(buf)[el]) << 16);
+    else
+        return reinterpret_cast<const float*>(buf)[el];
+}
+
 // Named barrier 1 over the NT consumer threads only.
 template <int NT>
 __device__ __forceinline__ void consumer_sync() {
@@ -164,7 +173,7 @@ __global__ void __launch_bounds__(NT + 32, RowsOcc<NT>::value) sv_rows_kernel(co
     constexpr int SEG = TILE_BYTES / ELT;   // elements per segment
     static_assert(VPT * NT == TV, "tile must split evenly over the consumer threads");
     static_assert(NW <= MAX_CONSUMER_WARPS, "too many consumer warps");
-    static_assert(VPT + 1 <= 32, "candidate mask");
+    static_assert(VPT * VEC <= 64, "candidate mask");
     extern __shared__ __align__(128) unsigned char smem[];
     RowsCtl& S = *reinterpret_cast<RowsCtl*>(smem);
     unsigned char* const ring = smem + ROWS_CTL_BYTES;
@@ -440,62 +449,78 @@ __global__ void __launch_bounds__(NT + 32, RowsOcc<NT>::value) sv_rows_kernel(co
                     publish(lane_bound());
                 }
                 theta = fmaxf(theta, read_bound());
-                // pass B: this tile's elements >= theta go to the warp's segment
-                unsigned cm = 0u;
-#pragma unroll
-                for (int i = 0; i <= VPT; ++i)
-                    if (ok && vm[i] >= theta) cm |= 1u << i;
-                if (__any_sync(0xffffffffu, cm != 0u)) {
-                    auto count = [&](float th) {
-                        int n = 0;
-#pragma unroll
-                        for (int i = 0; i <= VPT; ++i) {
-                            if ((cm >> i) & 1u) {
-                                float v[VEC];
-                                load_masked(jof(i), v);
-#pragma unroll
-                                for (int q = 0; q < VEC; ++q) n += v[q] >= th;
-                            }
-                        }
-                        return n;
-                    };
-                    int cnt = count(theta);
-                    int incl = cnt;
-#pragma unroll
-                    for (int o = 1; o < 32; o <<= 1) {
-                        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-                        if (lane >= o) incl += y;
-                    }
-                    int total = __shfl_sync(0xffffffffu, incl, 31);
-                    if (wcnt + total > wcap && !wovf) {
-                        compact();
-                        cnt = count(theta);
-                        incl = cnt;
-#pragma unroll
-                        for (int o = 1; o < 32; o <<= 1) {
-                            const int y = __shfl_up_sync(0xffffffffu, incl, o);
-                            if (lane >= o) incl += y;
-                        }
-                        total = __shfl_sync(0xffffffffu, incl, 31);
-                    }
-                    int p = wcnt + incl - cnt;
+                // Candidate bits of this tile: bit i*VEC + q of em is element q of
+                // vector slot i < VPT, bit q of emx element q of the extra slot.
+                // Only elements inside [lo, hi) qualify.
+                uint64_t em = 0u;
+                uint32_t emx = 0u;
+                if (ok && tm >= theta) {
 #pragma unroll
                     for (int i = 0; i <= VPT; ++i) {
-                        if ((cm >> i) & 1u) {
+                        if (vm[i] >= theta) {
                             const int j = jof(i);
-                            const int e = g.e0 + j * VEC;
                             float v[VEC];
-                            load_masked(j, v);
+                            unpack<DT>(vec_at(j), v);
+                            const int e = g.e0 + j * VEC;
+                            uint32_t m = 0u;
 #pragma unroll
-                            for (int q = 0; q < VEC; ++q) {
-                                if (v[q] >= theta) {
-                                    if (p < wcap) {
-                                        wkey[p] = v[q];
-                                        widxs[p] = e + q;
-                                    }
-                                    ++p;
-                                }
-                            }
+                            for (int q = 0; q < VEC; ++q) m |= (v[q] >= theta && valid(e + q)) ? (1u << q) : 0u;
+                            if (i < VPT)
+                                em |= static_cast<uint64_t>(m) << (i * VEC);
+                            else
+                                emx = m;
+                        }
+                    }
+                }
+                int cnt = __popcll(em) + __popc(emx);
+                if (__any_sync(0xffffffffu, cnt != 0)) {
+                    auto scan = [&](int x, int& tot) {
+                        int in = x;
+#pragma unroll
+                        for (int o = 1; o < 32; o <<= 1) {
+                            const int y = __shfl_up_sync(0xffffffffu, in, o);
+                            if (lane >= o) in += y;
+                        }
+                        tot = __shfl_sync(0xffffffffu, in, 31);
+                        return in - x;
+                    };
+                    int total;
+                    int excl = scan(cnt, total);
+                    if (wcnt + total > wcap && !wovf) {
+                        compact();
+                        // drop this tile's candidates below the raised bound
+                        for (uint64_t mm = em; mm;) {
+                            const int bit = __ffsll(static_cast<long long>(mm)) - 1;
+                            mm &= mm - 1;
+                            if (!(smem_elem<DT>(buf, (tid + (bit / VEC) * NT) * VEC + bit % VEC) >= theta))
+                                em &= ~(static_cast<uint64_t>(1) << bit);
+                        }
+                        for (uint32_t mm = emx; mm;) {
+                            const int q = __ffs(mm) - 1;
+                            mm &= mm - 1;
+                            if (!(smem_elem<DT>(buf, (TV + tid) * VEC + q) >= theta)) emx &= ~(1u << q);
+                        }
+                        cnt = __popcll(em) + __popc(emx);
+                        excl = scan(cnt, total);
+                    }
+                    // write this lane's candidates: value from the stage, index in the row
+                    int p = wcnt + excl;
+                    for (uint64_t mm = em; mm; ++p) {
+                        const int bit = __ffsll(static_cast<long long>(mm)) - 1;
+                        mm &= mm - 1;
+                        const int el = (tid + (bit / VEC) * NT) * VEC + bit % VEC;
+                        if (p < wcap) {
+                            wkey[p] = smem_elem<DT>(buf, el);
+                            widxs[p] = g.e0 + el;
+                        }
+                    }
+                    for (uint32_t mm = emx; mm; ++p) {
+                        const int q = __ffs(mm) - 1;
+                        mm &= mm - 1;
+                        const int el = (TV + tid) * VEC + q;
+                        if (p < wcap) {
+                            wkey[p] = smem_elem<DT>(buf, el);
+                            widxs[p] = g.e0 + el;
                         }
                     }
                     if (wcnt + total > wcap) wovf = true;
@@ -645,6 +670,7 @@ __global__ void __launch_bounds__(NT + 32, RowsOcc<NT>::value) sv_rows_kernel(co
             for (int q = tid; q < n2; q += NTH) {
                 const Cand e = fl[q];
                 int rk = 0;
+#pragma unroll 8
                 for (int f = 0; f < n2; ++f) {
                     const Cand o = fl[f];
                     rk += (o.v > e.v) || (o.v == e.v && o.i < e.i);
@@ -657,6 +683,7 @@ __global__ void __launch_bounds__(NT + 32, RowsOcc<NT>::value) sv_rows_kernel(co
                 const Cand e = fl[q];
                 if (!(e.v >= tau)) continue;
                 int ri = 0;
+#pragma unroll 8
                 for (int f = 0; f < n2; ++f) ri += (fl[f].v >= tau && fl[f].i < e.i);
                 atomicAdd(&S.nkept, 1);
                 if (ri < kscap) ks[ri] = e;
