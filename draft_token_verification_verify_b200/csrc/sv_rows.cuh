@@ -13,19 +13,24 @@
 //   greedy   per chunk: raw maximum and its lowest index,
 //   softmax  per segment: (max of z*c, sum of 2^(z*c - max)), c = log2(e)/T,
 //   max-only per chunk: raw maximum,
-//   top-k    per chunk: every element that can belong to the chunk's top-k
-//            set, found in the same single pass.  Warp w publishes a value
-//            b_w such that it has seen at least rsel = ceil(K / NW) distinct
-//            elements >= b_w (the rsel-th largest of its lanes' running
-//            maxima, or the rsel-th largest entry of its own candidate
-//            list).  Then at least NW * rsel >= K elements are >= min_w b_w,
-//            so that minimum never exceeds the chunk's K-th largest logit —
-//            whatever mix of older and newer published values a warp reads.
-//            Elements at or above it go to the warp's private list segment.
-//            At the end the exact K-th largest tau_c of the chunk and every
-//            element >= tau_c are stored, sorted by index, with the chunk
-//            maximum, the sum of 2^(z*c - max*c) over them and the logit at
-//            the row's draft token.
+//   top-k    per chunk: the exact K-th largest logit tau_c and every element
+//            >= tau_c, sorted by index, with the chunk maximum, the sum of
+//            2^(z*c - max*c) over them and the logit at the row's draft token.
+//            The pass works on 16-byte vectors and their maxima (each maximum
+//            is one element, so distinct vectors give distinct elements).
+//            Warp w publishes a value b_w such that at least rsel =
+//            ceil(K / NW) distinct vectors it has seen have a maximum >= b_w
+//            (the rsel-th largest of its lanes' running maxima, or the
+//            rsel-th largest entry of its own candidate list).  Then at least
+//            NW * rsel >= K vector maxima are >= min_w b_w, so that minimum
+//            never exceeds the K-th largest vector maximum tau_v — whatever mix
+//            of older and newer published values a warp reads — and vectors
+//            whose maximum reaches it go to the warp's private list (one
+//            ballot per vector slot, no per-element work).  At the end tau_v is
+//            taken exactly from the list; the chunk's K-th largest logit is
+//            >= tau_v and every element >= it lies in a vector whose maximum
+//            is >= tau_v, so only those ~K vectors are read again (from L2 or
+//            HBM) and expanded to elements.
 // Rows are read from HBM exactly once; no CTA waits for another.
 #pragma once
 
@@ -37,7 +42,7 @@ namespace sv {
 
 constexpr int MAX_STAGES = 8;
 constexpr int MAX_TILES_K1 = 64;   // segments per chunk
-constexpr int RANK_MAX = 256;      // final lists up to this size are ranked, larger ones sorted
+constexpr int RANK_MAX = 256;      // expanded top-k elements ranked per chunk (more: exact fallback)
 constexpr int TILE_BYTES = 16384;  // bytes per segment (one ring stage)
 constexpr int REC_DIAG = 4;        // a device-side consistency check failed
 constexpr int MAX_CONSUMER_WARPS = 16;
@@ -74,7 +79,8 @@ struct __align__(16) RowsCtl {
     int cnt2;
     int nkept;
     float tau;
-    int pad[2];
+    int ne;     // expanded elements (top-k)
+    float tauv; // K-th largest candidate-vector maximum (top-k)
     float wbound[MAX_CONSUMER_WARPS];  // published per-warp bounds (top-k)
     float wmax[MAX_CONSUMER_WARPS];
     float wbest[MAX_CONSUMER_WARPS];
@@ -449,82 +455,30 @@ __global__ void __launch_bounds__(NT + 32, RowsOcc<NT>::value) sv_rows_kernel(co
                     publish(lane_bound());
                 }
                 theta = fmaxf(theta, read_bound());
-                // Candidate bits of this tile: bit i*VEC + q of em is element q of
-                // vector slot i < VPT, bit q of emx element q of the extra slot.
-                // Only elements inside [lo, hi) qualify.
-                uint64_t em = 0u;
-                uint32_t emx = 0u;
-                if (ok && tm >= theta) {
+                // Candidate vectors: finite maximum at or above the bound.  A
+                // vector's maximum is one of its elements, so distinct vectors
+                // give distinct elements for the bounds.
+                int mine = 0;
+#pragma unroll
+                for (int i = 0; i <= VPT; ++i) mine += (ok && vm[i] > NEG_INF && vm[i] >= theta) ? 1 : 0;
+                const int total = __reduce_add_sync(0xffffffffu, mine);
+                if (total) {
+                    if (wcnt + total > wcap && !wovf) compact();  // raises theta
 #pragma unroll
                     for (int i = 0; i <= VPT; ++i) {
-                        if (vm[i] >= theta) {
-                            const int j = jof(i);
-                            float v[VEC];
-                            unpack<DT>(vec_at(j), v);
-                            const int e = g.e0 + j * VEC;
-                            uint32_t m = 0u;
-#pragma unroll
-                            for (int q = 0; q < VEC; ++q) m |= (v[q] >= theta && valid(e + q)) ? (1u << q) : 0u;
-                            if (i < VPT)
-                                em |= static_cast<uint64_t>(m) << (i * VEC);
-                            else
-                                emx = m;
+                        const bool cnd = ok && vm[i] > NEG_INF && vm[i] >= theta;
+                        const unsigned m = __ballot_sync(0xffffffffu, cnd);
+                        if (m) {
+                            const int p = wcnt + __popc(m & ((1u << lane) - 1u));
+                            if (cnd && p < wcap) {
+                                wkey[p] = vm[i];
+                                widxs[p] = t * (TV + 1) + jof(i);
+                            }
+                            const int n = __popc(m);
+                            if (wcnt + n > wcap) wovf = true;
+                            wcnt = min(wcnt + n, wcap);
                         }
                     }
-                }
-                int cnt = __popcll(em) + __popc(emx);
-                if (__any_sync(0xffffffffu, cnt != 0)) {
-                    auto scan = [&](int x, int& tot) {
-                        int in = x;
-#pragma unroll
-                        for (int o = 1; o < 32; o <<= 1) {
-                            const int y = __shfl_up_sync(0xffffffffu, in, o);
-                            if (lane >= o) in += y;
-                        }
-                        tot = __shfl_sync(0xffffffffu, in, 31);
-                        return in - x;
-                    };
-                    int total;
-                    int excl = scan(cnt, total);
-                    if (wcnt + total > wcap && !wovf) {
-                        compact();
-                        // drop this tile's candidates below the raised bound
-                        for (uint64_t mm = em; mm;) {
-                            const int bit = __ffsll(static_cast<long long>(mm)) - 1;
-                            mm &= mm - 1;
-                            if (!(smem_elem<DT>(buf, (tid + (bit / VEC) * NT) * VEC + bit % VEC) >= theta))
-                                em &= ~(static_cast<uint64_t>(1) << bit);
-                        }
-                        for (uint32_t mm = emx; mm;) {
-                            const int q = __ffs(mm) - 1;
-                            mm &= mm - 1;
-                            if (!(smem_elem<DT>(buf, (TV + tid) * VEC + q) >= theta)) emx &= ~(1u << q);
-                        }
-                        cnt = __popcll(em) + __popc(emx);
-                        excl = scan(cnt, total);
-                    }
-                    // write this lane's candidates: value from the stage, index in the row
-                    int p = wcnt + excl;
-                    for (uint64_t mm = em; mm; ++p) {
-                        const int bit = __ffsll(static_cast<long long>(mm)) - 1;
-                        mm &= mm - 1;
-                        const int el = (tid + (bit / VEC) * NT) * VEC + bit % VEC;
-                        if (p < wcap) {
-                            wkey[p] = smem_elem<DT>(buf, el);
-                            widxs[p] = g.e0 + el;
-                        }
-                    }
-                    for (uint32_t mm = emx; mm; ++p) {
-                        const int q = __ffs(mm) - 1;
-                        mm &= mm - 1;
-                        const int el = (TV + tid) * VEC + q;
-                        if (p < wcap) {
-                            wkey[p] = smem_elem<DT>(buf, el);
-                            widxs[p] = g.e0 + el;
-                        }
-                    }
-                    if (wcnt + total > wcap) wovf = true;
-                    wcnt = min(wcnt + total, wcap);
                 }
             } else {
                 run = fmax_nan(run, tm);  // MODE_MAXONLY
@@ -632,15 +586,19 @@ __global__ void __launch_bounds__(NT + 32, RowsOcc<NT>::value) sv_rows_kernel(co
             ovf |= S.wovf[w];
         }
         const int d = (pos < P.k && P.draft_tokens) ? P.draft_tokens[b * P.k + pos] : -1;
-        // entries >= the final bound, copied from the warp segments into the free ring
-        Cand* fl = reinterpret_cast<Cand*>(ring);
+        Cand* fl = reinterpret_cast<Cand*>(ring);  // candidate vectors (the ring is free now)
         const int fcap = (P.stages * STAGE_BYTES) / static_cast<int>(sizeof(Cand));
+        Cand* E = reinterpret_cast<Cand*>(lkey);  // expanded elements (after step 1)
+        const int ecap = P.lcap;
         if (tid == 0) {
             S.cnt2 = 0;
+            S.ne = 0;
             S.nkept = 0;
             S.tau = NEG_INF;
+            S.tauv = NEG_INF;
         }
         __syncthreads();
+        // 1. candidate vectors whose maximum reaches the final bound
         if (warp < NW) {
             const int n = S.wcnt[warp];
             const float* wk = lkey + warp * wcap;
@@ -657,72 +615,83 @@ __global__ void __launch_bounds__(NT + 32, RowsOcc<NT>::value) sv_rows_kernel(co
             }
         }
         __syncthreads();
-        const int n2 = S.cnt2;
-        // kept entries, index-sorted, staged in shared memory: in the (now free)
-        // segment area after ranking, in the ring after sorting
-        Cand* ks = reinterpret_cast<Cand*>(lkey);
-        const int kscap = P.lcap;
-        Cand* out = P.cands + (r * P.nch + c) * static_cast<long long>(P.kcap);
-        float lastv = NEG_INF;
-        int nk;
-        if (n2 <= RANK_MAX) {
-            // rank by (value desc, index asc): tau is the value at rank K-1
-            for (int q = tid; q < n2; q += NTH) {
-                const Cand e = fl[q];
-                int rk = 0;
+        const int nv = min(S.cnt2, fcap);
+        // 2. tau_v = K-th largest vector maximum (with multiplicity); at least
+        //    K distinct elements are >= tau_v, so the chunk's K-th largest
+        //    logit is >= tau_v and lies in a vector whose maximum is >= tau_v.
+        for (int q = tid; q < nv; q += NTH) {
+            const float x = fl[q].v;
+            int gt = 0, ge = 0;
 #pragma unroll 8
-                for (int f = 0; f < n2; ++f) {
-                    const Cand o = fl[f];
-                    rk += (o.v > e.v) || (o.v == e.v && o.i < e.i);
-                }
-                if (rk == K - 1) S.tau = e.v;
+            for (int f = 0; f < nv; ++f) {
+                const float y = fl[f].v;
+                gt += y > x;
+                ge += y >= x;
             }
-            __syncthreads();
-            const float tau = n2 >= K ? S.tau : NEG_INF;
-            for (int q = tid; q < n2; q += NTH) {
-                const Cand e = fl[q];
-                if (!(e.v >= tau)) continue;
+            if (gt < K && K <= ge) S.tauv = x;
+        }
+        __syncthreads();
+        const float tauv = S.tauv;  // -inf: fewer than K candidate vectors (all are expanded)
+        // 3. the elements >= tau_v of those vectors, read again from the row
+        for (int q = tid; q < nv; q += NTH) {
+            const Cand cv = fl[q];
+            if (!(cv.v >= tauv)) continue;
+            const int tt = cv.i / (TV + 1), j = cv.i - tt * (TV + 1);
+            const TileGeom g = geom(tt);
+            const int e = g.e0 + j * VEC;
+            float v[VEC];
+            if (e >= g.lo && e + VEC <= g.hi) {
+                unpack<DT>(__ldg(reinterpret_cast<const uint4*>(g.A0 + 16u * static_cast<uintptr_t>(j))), v);
+            } else {
+#pragma unroll
+                for (int u = 0; u < VEC; ++u) v[u] = (e + u >= g.lo && e + u < g.hi) ? load_elem<DT>(row, e + u) : NEG_INF;
+            }
+#pragma unroll
+            for (int u = 0; u < VEC; ++u) {
+                if (v[u] >= tauv && e + u >= g.lo && e + u < g.hi) {
+                    const int p = atomicAdd(&S.ne, 1);
+                    if (p < ecap) E[p] = Cand{v[u], e + u};
+                }
+            }
+        }
+        __syncthreads();
+        const int ne_all = S.ne;
+        const int ne = min(ne_all, ecap);
+        if (ne_all > ecap || ne > RANK_MAX) ovf = 1;  // massive ties: exact fallback downstream
+        // 4. tau = K-th largest element (with multiplicity)
+        if (!ovf) {
+            for (int q = tid; q < ne; q += NTH) {
+                const float x = E[q].v;
+                int gt = 0, ge = 0;
+#pragma unroll 8
+                for (int f = 0; f < ne; ++f) {
+                    const float y = E[f].v;
+                    gt += y > x;
+                    ge += y >= x;
+                }
+                if (gt < K && K <= ge) S.tau = x;
+            }
+        }
+        __syncthreads();
+        const float tau = S.tau;  // -inf: fewer than K elements, every one is kept
+        // 5. kept entries (>= tau) in index order, staged in the ring
+        Cand* ks = fl;  // fl is no longer read after step 3
+        const int kscap = fcap;
+        Cand* out = P.cands + (r * P.nch + c) * static_cast<long long>(P.kcap);
+        if (!ovf) {
+            for (int q = tid; q < ne; q += NTH) {
+                const Cand x = E[q];
+                if (!(x.v >= tau)) continue;
                 int ri = 0;
 #pragma unroll 8
-                for (int f = 0; f < n2; ++f) ri += (fl[f].v >= tau && fl[f].i < e.i);
+                for (int f = 0; f < ne; ++f) ri += (E[f].v >= tau && E[f].i < x.i);
                 atomicAdd(&S.nkept, 1);
-                if (ri < kscap) ks[ri] = e;
+                if (ri < kscap) ks[ri] = x;
             }
-            __syncthreads();
-            nk = S.nkept;
-            lastv = tau;  // every kept entry is >= tau
-        } else {
-            // large lists: sort by value, cut at rank K (with ties), sort the cut by index
-            const int n0 = min(n2, min(fcap, P.lcap));
-            float* sk = lkey;
-            int* si = lidx;
-            const int N = pow2_ceil(n0 < 2 ? 2 : n0);
-            for (int q = tid; q < N; q += NTH) {
-                sk[q] = q < n0 ? fl[q].v : NEG_INF;
-                si[q] = q < n0 ? fl[q].i : INT_MAX;
-            }
-            __syncthreads();
-            block_sort<true>(sk, si, N);
-            const float tau = (n0 >= K) ? sk[K - 1] : NEG_INF;
-            for (int q = tid; q < n0; q += NTH)
-                if (sk[q] >= tau && (q + 1 == n0 || !(sk[q + 1] >= tau))) S.nkept = q + 1;
-            __syncthreads();
-            nk = S.nkept;
-            const int m = min(nk, P.kcap);
-            lastv = m > 0 ? sk[m - 1] : NEG_INF;
-            const int M2 = pow2_ceil(m < 2 ? 2 : m);
-            for (int q = m + tid; q < M2; q += NTH) {
-                sk[q] = NEG_INF;
-                si[q] = INT_MAX;
-            }
-            __syncthreads();
-            block_sort<false>(sk, si, M2);
-            ks = fl;  // the ring was copied out before the sorts (m <= kcap < fcap)
-            for (int q = tid; q < m; q += NTH) ks[q] = Cand{sk[q], si[q]};
-            if (tid == 0) S.tau = tau;
-            if (n2 > fcap || n2 > P.lcap) ovf = 1;
-            __syncthreads();
         }
+        __syncthreads();
+        const int nk = S.nkept;
+        const float lastv = tau;  // every kept entry is >= tau
         // exp-sum and draft-token logit over the stored (index-sorted) entries
         const int m = min(nk, P.kcap);
         const float msc = cmax * cscale;
@@ -752,6 +721,7 @@ __global__ void __launch_bounds__(NT + 32, RowsOcc<NT>::value) sv_rows_kernel(co
             ch.last = lastv;
             ch.n = m;
             ch.flags = (ovf || nk > P.kcap) ? REC_OVERFLOW : 0;
+            if (ovf) ch.n = 0;
             ch.m = cmax;
             ch.s = s;
             ch.zd = z;
