@@ -100,7 +100,7 @@ __device__ __forceinline__ void load_vec(const void* row, bool aligned, int q, i
 }
 
 template <int DT>
-__global__ void __launch_bounds__(SEQ_NT, 2) sv_seq_kernel(const SeqParams P) {
+__global__ void __launch_bounds__(SEQ_NT, 3) sv_seq_kernel(const SeqParams P) {
     constexpr int VEC = VT<DT>::VEC;
     constexpr int ELT = VT<DT>::ELT;
     constexpr int NT = SEQ_NT, NW = SEQ_NW;
