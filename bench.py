@@ -37,7 +37,7 @@ PROFILE_DIR = os.path.join(ROOT, "profiles")
 KSAMPLE = 8  # timed steps per streaming-kernel event sample
 
 KERNEL_SOURCES = [os.path.join(ROOT, "draft_token_verification_verify_b200", "csrc", f)
-                  for f in ("sv_common.cuh", "sv_rows.cuh", "sv_seq.cuh", "sv_ptx.cuh", "spec_verify.cu")]
+                  for f in ("sv_common.cuh", "sv_rows.cuh", "sv_seq.cuh", "sv_resid.cuh", "sv_ptx.cuh", "spec_verify.cu")]
 
 DESCR = {
     "tiny": "tiny stochastic verify B=1 k=4 V=32 fp32 T=1",
@@ -137,6 +137,14 @@ class ClockSampler:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
                 "reasons": sorted(reasons)}
+
+
+def launches_per_step(case) -> int:
+    """Kernels one spec_verify call launches: the streaming pass and the
+    per-sequence kernel, plus the residual segment kernel for stochastic
+    verification without top-k."""
+    stochastic_softmax = case.mode != "greedy" and not (0 < case.top_k < case.V)
+    return 3 if stochastic_softmax else 2
 
 
 def to_dev(a, device):
@@ -412,7 +420,7 @@ def run_ours(args):
                      "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
                      "kernel": "sv_rows_kernel", "kernel_ms_mean": kmean,
                      "kernel_ms_median": statistics.median(kern_ms)},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": launches_per_step(case) * args.steps,
         "clocks": clocks,
         "e2e": e2e,
         "cpu_baseline": cpu,

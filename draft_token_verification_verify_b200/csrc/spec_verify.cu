@@ -1,6 +1,8 @@
 // Host side of the spec_verify C ABI: argument checks, launch planning,
-// workspace handling and the two launches (the streaming pass, then the
-// per-sequence kernel as a programmatic dependent launch).  Nothing here
+// workspace handling and the launches: the streaming pass, then the
+// per-sequence kernel as a programmatic dependent launch, then (softmax
+// verification only) the segment kernel of the residual draws, also as a
+// programmatic dependent launch.  Nothing here
 // synchronises the caller's stream.
 #include <cuda_runtime.h>
 
@@ -11,6 +13,7 @@
 
 #include "../../include/spec_verify.h"
 #include "sv_rows.cuh"
+#include "sv_resid.cuh"
 #include "sv_seq.cuh"
 
 namespace {
@@ -97,6 +100,8 @@ struct Plan {
     long long R = 0, tasks = 0;
     size_t smem1 = 0, smem2 = 0;
     size_t off_chunks = 0, off_cands = 0, ws_bytes = 0;
+    bool defer = false;  // residual draws by the segment kernel
+    size_t off_req = 0, off_mass = 0, off_counter = 0;
 };
 
 int rows_occupancy(int dev, int dt, int nt, int mode, size_t smem);
@@ -174,6 +179,15 @@ sv_status_t make_plan(const DeviceInfo& dev, long long seqs, int k, int V, int d
     }
     p.off_cands = round_up(p.off_chunks + chunks, 256);
     p.ws_bytes = round_up(p.off_cands + cands, 256);
+    // softmax verification: residual draws by the segment kernel
+    p.defer = p.mode == sv::MODE_SOFTMAX && k > 0;
+    if (p.defer) {
+        if (seqs * static_cast<long long>(p.nseg) > INT_MAX) return SV_ERR_INVALID_ARG;
+        p.off_req = p.ws_bytes;
+        p.off_mass = round_up(p.off_req + static_cast<size_t>(seqs) * sizeof(sv::DrawReq), 256);
+        p.off_counter = round_up(p.off_mass + static_cast<size_t>(seqs) * p.nseg * sizeof(float2), 256);
+        p.ws_bytes = round_up(p.off_counter + static_cast<size_t>(seqs) * sizeof(int), 256);
+    }
     // per-sequence kernel: control, row stats, gather buffers, segment masses
     const int nrows = greedy ? k + 1 : 2 * k + 1;
     size_t head = static_cast<size_t>(nrows) * sizeof(sv::RowStat) + static_cast<size_t>(k + 1) * 8 + 8;
@@ -189,6 +203,7 @@ sv_status_t make_plan(const DeviceInfo& dev, long long seqs, int k, int V, int d
 
 using RowsFn = void (*)(sv::RowsParams);
 using SeqFn = void (*)(sv::SeqParams);
+using ResFn = void (*)(sv::ResidParams);
 
 template <int DT, int NT>
 RowsFn rows_for_mode(int mode) {
@@ -339,6 +354,23 @@ sv_status_t run(const Call& cl, void* workspace, size_t workspace_bytes, const s
     q.out_p = cl.out_p;
     q.out_q = cl.out_q;
     q.out_status = cl.sample ? nullptr : cl.out_status;
+    q.defer = p.defer ? 1 : 0;
+    q.req = p.defer ? reinterpret_cast<sv::DrawReq*>(base + p.off_req) : nullptr;
+    q.counter = p.defer ? reinterpret_cast<int*>(base + p.off_counter) : nullptr;
+
+    sv::ResidParams rp;
+    std::memset(&rp, 0, sizeof rp);
+    rp.target = cl.target;
+    rp.draft = cl.draft;
+    rp.V = cl.V;
+    rp.k = cl.k;
+    rp.seg = p.seg;
+    rp.nseg = p.nseg;
+    rp.req = q.req;
+    rp.mass = p.defer ? reinterpret_cast<float2*>(base + p.off_mass) : nullptr;
+    rp.counter = q.counter;
+    rp.out_tokens = cl.out_tokens;
+    rp.out_n = cl.out_n;
 
     sv_status_t result = SV_OK;
     do {
@@ -379,6 +411,21 @@ sv_status_t run(const Call& cl, void* workspace, size_t workspace_bytes, const s
         if (cudaLaunchKernelEx(&c2, f2, q) != cudaSuccess) {
             result = SV_ERR_CUDA;
             break;
+        }
+        if (p.defer) {
+            cudaLaunchConfig_t c3;
+            std::memset(&c3, 0, sizeof c3);
+            c3.gridDim = dim3(static_cast<unsigned>(cl.seqs * p.nseg), 1, 1);
+            c3.blockDim = dim3(sv::RES_NT, 1, 1);
+            c3.dynamicSmemBytes = 0;
+            c3.stream = st;
+            c3.attrs = a2;  // programmatic dependent launch, like the per-sequence kernel
+            c3.numAttrs = 1;
+            ResFn f3 = cl.dt ? sv::sv_resid_kernel<1> : sv::sv_resid_kernel<0>;
+            if (cudaLaunchKernelEx(&c3, f3, rp) != cudaSuccess) {
+                result = SV_ERR_CUDA;
+                break;
+            }
         }
     } while (false);
     if (result != SV_OK) cudaGetLastError();

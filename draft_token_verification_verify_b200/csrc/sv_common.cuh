@@ -50,6 +50,23 @@ struct Cand {
     int i;
 };
 
+// A final draw handed from the per-sequence kernel to the segment kernel
+// (64 bytes): weights w(v) = max(0, p(v) - q(v)) over the row pair of position
+// j, or p(v) alone, with p(v) = [z_t(v) >= t_tau] 2^(z_t(v)*c - t_msc) * t_invS
+// and q(v) likewise from the draft row.
+struct DrawReq {
+    int need;        // 1: this sequence's draw is done by the segment kernel
+    int j;           // position of the draw (= accepted draft tokens)
+    int use_q;       // 1: residual weights, 0: p alone
+    int pad0;
+    long long rowt;  // row index of the target row in the target tensor
+    long long rowd;  // row index of the draft row in the draft tensor
+    float t_msc, t_invS, t_tau;
+    float d_msc, d_invS, d_tau;
+    float u;         // the sequence's final uniform u_k
+    float c;         // log2(e) / T
+};
+
 template <int DT>
 struct VT;
 template <>

@@ -12,8 +12,10 @@
 // Draws: with top-k, from the kept lists gathered by the streaming pass (no
 // logit is read again); without top-k, the bonus draw locates its segment
 // from the streaming partials and rescans that segment only, while a
-// residual draw streams the rejected (target, draft) pair once to get
-// per-segment masses and rescans the segment that holds u * W.  Rows whose
+// residual draw is handed to the segment kernel (one CTA per segment of the
+// rejected (target, draft) pair).  The rare cases left here (zero-mass
+// retries of top-k rows resolved by radix select) stream the pair in this
+// CTA.  Rows whose
 // kept list did not fit (massive ties) or top-k above the list capacity fall
 // back to an exact radix select over the row in global memory.
 #pragma once
@@ -49,6 +51,9 @@ struct SeqParams {
     float* out_p;                // [B][k] or null
     float* out_q;                // [B][k] or null
     int32_t* out_status;         // or null
+    int defer;                   // residual draws go to the segment kernel (softmax, verify)
+    DrawReq* req;                // [B] when defer
+    int* counter;                // [B] when defer: zeroed here for the segment kernel
 };
 
 struct RowStat {
@@ -146,7 +151,8 @@ __global__ void __launch_bounds__(SEQ_NT, 3) sv_seq_kernel(const SeqParams P) {
         }
         S.err = bad;
     }
-    pdl_wait_primary();  // the streaming pass is complete from here on
+    pdl_launch_dependents();  // the segment kernel may be placed early; it waits for this grid
+    pdl_wait_primary();       // the streaming pass is complete from here on
 
     auto row_ptr = [&](int rr) -> const void* {
         if (rr <= k)
@@ -496,6 +502,29 @@ __global__ void __launch_bounds__(SEQ_NT, 3) sv_seq_kernel(const SeqParams P) {
                 if (lane == 0) S.token = token;
             }
             __syncthreads();
+        } else if (P.defer && use_q0) {
+            // residual draw: handed to the segment kernel (one CTA per segment)
+            if (tid == 0) {
+                DrawReq q;
+                q.need = 1;
+                q.j = j;
+                q.use_q = 1;
+                q.pad0 = 0;
+                q.rowt = b * (k + 1) + j;
+                q.rowd = b * k + j;
+                q.t_msc = tst.msc;
+                q.t_invS = tst.invS;
+                q.t_tau = tst.tau;
+                q.d_msc = dst.msc;
+                q.d_invS = dst.invS;
+                q.d_tau = dst.tau;
+                q.u = u;
+                q.c = c;
+                P.req[b] = q;
+                P.counter[b] = 0;
+                S.token = INT_MAX;  // written by the segment kernel
+            }
+            __syncthreads();
         } else {
             // streaming draw over the row(s): per-segment masses, then one segment
             const void* rowt = row_ptr(j);
@@ -654,6 +683,14 @@ __global__ void __launch_bounds__(SEQ_NT, 3) sv_seq_kernel(const SeqParams P) {
     if (tid == 0) {
         int err = S.err;
         const int j = S.j;
+        const bool deferred = !err && !greedy && S.token == INT_MAX;
+        if (P.defer && !deferred) P.req[b].need = 0;
+        if (deferred) {
+            int32_t* out = P.out_tokens + b * (k + 1);
+            for (int i = 0; i <= k; ++i) out[i] = i < j ? dtok[i] : -1;
+            P.out_n[b] = j;
+            return;
+        }
         const int y = err ? -1 : S.token;
         if (y < 0) err = 1;
         if (P.sample_only) {
