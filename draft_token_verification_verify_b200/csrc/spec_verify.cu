@@ -101,6 +101,8 @@ struct Plan {
     size_t smem1 = 0, smem2 = 0;
     size_t off_chunks = 0, off_cands = 0, ws_bytes = 0;
     bool defer = false;  // residual draws by the segment kernel
+    bool pre = false;    // per-sequence kernel loads every row's kept list at once
+    size_t pre_off = 0;
     size_t off_req = 0, off_mass = 0, off_counter = 0;
 };
 
@@ -194,6 +196,13 @@ sv_status_t make_plan(const DeviceInfo& dev, long long seqs, int k, int V, int d
     head = round_up(head, 128);
     p.smem2 = sv::SEQ_CTL_BYTES + head + static_cast<size_t>(sv::SEQ_NW) * p.mg * sizeof(sv::Cand) +
               static_cast<size_t>(p.nseg) * (sv::SEQ_NW + 1) * sizeof(float);
+    // top-k with one chunk per row: every row's record and kept list in shared memory
+    const size_t pre_bytes = static_cast<size_t>(nrows) * (static_cast<size_t>(p.kcap) * sizeof(sv::Cand) + sizeof(sv::ChunkRec));
+    if (p.mode == sv::MODE_TOPK && p.nch == 1 && pre_bytes <= 64 * 1024) {
+        p.pre = true;
+        p.pre_off = round_up(p.smem2, 16);
+        p.smem2 = p.pre_off + pre_bytes;
+    }
     if (p.smem1 > static_cast<size_t>(dev.smem_optin) || p.smem2 > static_cast<size_t>(dev.smem_optin))
         return SV_ERR_UNSUPPORTED;
     (void)vec;
@@ -355,6 +364,8 @@ sv_status_t run(const Call& cl, void* workspace, size_t workspace_bytes, const s
     q.out_q = cl.out_q;
     q.out_status = cl.sample ? nullptr : cl.out_status;
     q.defer = p.defer ? 1 : 0;
+    q.pre = p.pre ? 1 : 0;
+    q.pre_off = static_cast<int>(p.pre_off);
     q.req = p.defer ? reinterpret_cast<sv::DrawReq*>(base + p.off_req) : nullptr;
     q.counter = p.defer ? reinterpret_cast<int*>(base + p.off_counter) : nullptr;
 

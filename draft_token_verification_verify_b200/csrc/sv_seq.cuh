@@ -51,6 +51,9 @@ struct SeqParams {
     float* out_p;                // [B][k] or null
     float* out_q;                // [B][k] or null
     int32_t* out_status;         // or null
+    int pre;                     // top-k with one chunk per row: every row's record and kept
+                                 // list is loaded into shared memory at offset pre_off
+    int pre_off;
     int defer;                   // residual draws go to the segment kernel (softmax, verify)
     DrawReq* req;                // [B] when defer
     int* counter;                // [B] when defer: zeroed here for the segment kernel
@@ -154,6 +157,36 @@ __global__ void __launch_bounds__(SEQ_NT, 3) sv_seq_kernel(const SeqParams P) {
     pdl_launch_dependents();  // the segment kernel may be placed early; it waits for this grid
     pdl_wait_primary();       // the streaming pass is complete from here on
 
+    // top-k, one chunk per row: all of the sequence's chunk records and kept
+    // lists in one cooperative round of independent loads
+    Cand* const plist = P.pre ? reinterpret_cast<Cand*>(smem + P.pre_off) : nullptr;  // [nrows][kcap]
+    ChunkRec* const prec = P.pre ? reinterpret_cast<ChunkRec*>(plist + static_cast<size_t>(nrows) * P.kcap) : nullptr;
+    if (P.pre) {
+        const int per = 2 + P.kcap / 2;  // 16-byte vectors per row: record, then list
+        constexpr int PF = 4;            // loads in flight per thread before their stores
+        auto src = [&](int x) {
+            const int rr = x / per, o = x - (x / per) * per;
+            const long long r = rr <= k ? b * (k + 1) + rr : Rt + b * k + (rr - k - 1);
+            return o < 2 ? reinterpret_cast<const uint4*>(P.chunks + r) + o
+                         : reinterpret_cast<const uint4*>(P.cands + r * P.kcap) + (o - 2);
+        };
+        auto dst = [&](int x) {
+            const int rr = x / per, o = x - (x / per) * per;
+            return o < 2 ? reinterpret_cast<uint4*>(prec + rr) + o
+                         : reinterpret_cast<uint4*>(plist + static_cast<size_t>(rr) * P.kcap) + (o - 2);
+        };
+        for (int x0 = tid; x0 < nrows * per; x0 += NT * PF) {
+            uint4 tmp[PF];
+#pragma unroll
+            for (int u = 0; u < PF; ++u)
+                if (x0 + u * NT < nrows * per) tmp[u] = *src(x0 + u * NT);
+#pragma unroll
+            for (int u = 0; u < PF; ++u)
+                if (x0 + u * NT < nrows * per) *dst(x0 + u * NT) = tmp[u];
+        }
+        __syncthreads();
+    }
+
     auto row_ptr = [&](int rr) -> const void* {
         if (rr <= k)
             return static_cast<const char*>(P.target) + (static_cast<size_t>(b) * (k + 1) + rr) * static_cast<size_t>(V) * ELT;
@@ -224,6 +257,8 @@ __global__ void __launch_bounds__(SEQ_NT, 3) sv_seq_kernel(const SeqParams P) {
             st.arg = bi;
             if (mx != mx || mx == POS_INF || bi < 0) st.err = 1;
         } else if (P.mode == MODE_SOFTMAX) {
+            // the draft-token logit load is issued before the partials are combined
+            if (d >= 0 && d < V) st.zd = load_elem<DT>(row_ptr(rr), d);
             float m = NEG_INF, s = 0.f;
             for (int q = lane; q < P.nseg; q += 32) {
                 const SegRec g = P.segs[r * P.nseg + q];
@@ -236,11 +271,14 @@ __global__ void __launch_bounds__(SEQ_NT, 3) sv_seq_kernel(const SeqParams P) {
             st.msc = m;
             st.invS = 1.f / s;
             if (m != m || m == POS_INF || m == NEG_INF || s != s) st.err = 1;
-            if (d >= 0 && d < V) st.zd = load_elem<DT>(row_ptr(rr), d);
         } else {
             // top-k: raw maximum over the chunks, then the kept set
             float mx = NEG_INF;
-            for (int q = lane; q < P.nch; q += 32) {
+            if (P.pre) {
+                const ChunkRec& g = prec[rr];
+                tmo |= g.flags & REC_TIMEOUT;
+                mx = g.m;
+            } else for (int q = lane; q < P.nch; q += 32) {
                 if (P.mode == MODE_TOPK) {
                     const ChunkRec g = P.chunks[r * P.nch + q];
                     tmo |= g.flags & REC_TIMEOUT;
@@ -260,7 +298,7 @@ __global__ void __launch_bounds__(SEQ_NT, 3) sv_seq_kernel(const SeqParams P) {
                 float G = NEG_INF;
                 int ovf = 0;
                 for (int ch = lane; ch < P.nch; ch += 32) {
-                    const ChunkRec cr = P.chunks[r * P.nch + ch];
+                    const ChunkRec cr = P.pre ? prec[rr] : P.chunks[r * P.nch + ch];
                     G = fmaxf(G, cr.tau);
                     tmo |= cr.flags & REC_TIMEOUT;
                     ovf |= cr.flags & REC_OVERFLOW;
@@ -272,7 +310,7 @@ __global__ void __launch_bounds__(SEQ_NT, 3) sv_seq_kernel(const SeqParams P) {
                 int ng = 0;
                 if (P.nch == 1 && !ovf) {
                     // one chunk: its header already holds tau, the sum and the draft logit
-                    const ChunkRec cr = P.chunks[r];
+                    const ChunkRec cr = P.pre ? prec[rr] : P.chunks[r];
                     st.tau = cr.tau;
                     st.invS = 1.f / cr.s;
                     st.zd = cr.zd;
@@ -387,46 +425,44 @@ __global__ void __launch_bounds__(SEQ_NT, 3) sv_seq_kernel(const SeqParams P) {
         }
     }
 
-    // ---- phase 2: decisions ----------------------------------------------------------
-    if (tid == 0) {
+    // ---- phase 2: decisions (warp 0, one lane per position) ----------------------------
+    if (warp == 0) {
         int err = S.err, tmo = 0;
-        for (int rr = 0; rr < nrows; ++rr) {
+        for (int rr = lane; rr < nrows; rr += 32) {
             if (rs[rr].err) err = 1;
             if (rs[rr].err == 2) tmo = 1;
         }
+        err = __any_sync(0xffffffffu, err);
+        tmo = __any_sync(0xffffffffu, tmo);
         int j = k;
-        if (!err) {
-            if (greedy) {
-                for (int i = 0; i < k; ++i)
-                    if (dtok[i] != rs[i].arg) {
-                        j = i;
-                        break;
-                    }
-                S.token = rs[j].arg;
-            } else {
-                bool found = false;
-                for (int i = 0; i < k; ++i) {
+        for (int i0 = 0; i0 < k; i0 += 32) {
+            const int i = i0 + lane;
+            bool rej = false;
+            if (i < k) {
+                if (greedy) {
+                    rej = !err && dtok[i] != rs[i].arg;
+                } else if (!err) {
                     const RowStat& t = rs[i];
                     const RowStat& dd = rs[k + 1 + i];
                     const float p = (t.zd >= t.tau) ? ex2(fmaf(t.zd, c, -t.msc)) * t.invS : 0.f;
                     const float q = (dd.zd >= dd.tau) ? ex2(fmaf(dd.zd, c, -dd.msc)) * dd.invS : 0.f;
                     if (P.out_p) P.out_p[b * k + i] = p;
                     if (P.out_q) P.out_q[b * k + i] = q;
-                    if (!found && !(uu[i] * q < p)) {
-                        j = i;
-                        found = true;
-                    }
+                    rej = !(uu[i] * q < p);
+                } else {
+                    if (P.out_p) P.out_p[b * k + i] = __int_as_float(0x7fc00000);
+                    if (P.out_q) P.out_q[b * k + i] = __int_as_float(0x7fc00000);
                 }
             }
-        } else if (!greedy) {
-            for (int i = 0; i < k; ++i) {
-                if (P.out_p) P.out_p[b * k + i] = __int_as_float(0x7fc00000);
-                if (P.out_q) P.out_q[b * k + i] = __int_as_float(0x7fc00000);
-            }
+            const unsigned m = __ballot_sync(0xffffffffu, rej);
+            if (m && j == k) j = i0 + __ffs(m) - 1;  // the first rejection
         }
-        if (tmo && P.out_status) atomicExch(P.out_status, -4);
-        S.err = err;
-        S.j = j;
+        if (lane == 0) {
+            if (!err && greedy) S.token = rs[j].arg;
+            if (tmo && P.out_status) atomicExch(P.out_status, -4);
+            S.err = err;
+            S.j = j;
+        }
     }
     __syncthreads();
 
@@ -442,46 +478,68 @@ __global__ void __launch_bounds__(SEQ_NT, 3) sv_seq_kernel(const SeqParams P) {
             Cand* lt = gbuf;
             Cand* ld = gbuf + P.mg;
             int nt = 0, nd = 0;
-            if (warp == 0) nt = gather(row_index(j), tst.tau, lt, P.mg);
-            if (warp == 1 && use_q0) nd = gather(row_index(k + 1 + j), dst.tau, ld, P.mg);
-            if (warp == 1 && lane == 0) S.red_i[1] = nd;
-            __syncthreads();
-            nd = S.red_i[1];
-            if (warp == 0) {
-                auto find = [&](int v) {
-                    int a = 0, z = nd - 1;
-                    while (a <= z) {
-                        const int mid = (a + z) >> 1;
-                        const int x = ld[mid].i;
-                        if (x == v) return mid;
-                        if (x < v) a = mid + 1; else z = mid - 1;
-                    }
-                    return -1;
-                };
-                bool use_q = use_q0;
-                auto weight = [&](int e) {
+            if (P.pre) {
+                // one chunk per row: the kept lists are complete, index-sorted and in shared memory
+                lt = plist + static_cast<size_t>(j) * P.kcap;
+                nt = prec[j].n;
+                if (use_q0) {
+                    ld = plist + static_cast<size_t>(k + 1 + j) * P.kcap;
+                    nd = prec[k + 1 + j].n;
+                }
+            } else {
+                if (warp == 0) nt = gather(row_index(j), tst.tau, lt, P.mg);
+                if (warp == 1 && use_q0) nd = gather(row_index(k + 1 + j), dst.tau, ld, P.mg);
+                if (warp == 0 && lane == 0) S.red_i[0] = nt;
+                if (warp == 1 && lane == 0) S.red_i[1] = nd;
+                __syncthreads();
+                nt = S.red_i[0];  // every thread takes part in the weights below
+                nd = S.red_i[1];
+            }
+            // weights of the target entries, computed once by all threads
+            float* wv = reinterpret_cast<float*>(P.pre ? gbuf : gbuf + 2 * P.mg);
+            auto find = [&](int v) {
+                int a = 0, z = nd - 1;
+                while (a <= z) {
+                    const int mid = (a + z) >> 1;
+                    const int x = ld[mid].i;
+                    if (x == v) return mid;
+                    if (x < v) a = mid + 1; else z = mid - 1;
+                }
+                return -1;
+            };
+            bool use_q = use_q0;
+            for (int attempt = 0; attempt < 2; ++attempt) {
+                for (int e = tid; e < nt; e += NT) {
                     const float pt = ex2(fmaf(lt[e].v, c, -tst.msc)) * tst.invS;
-                    if (!use_q) return pt;
-                    const int pd = find(lt[e].i);
-                    const float q = pd >= 0 ? ex2(fmaf(ld[pd].v, c, -dst.msc)) * dst.invS : 0.f;
-                    return fmaxf(pt - q, 0.f);
-                };
-                float W = 0.f;
-                for (int attempt = 0; attempt < 2; ++attempt) {
-                    W = 0.f;
+                    float w = pt;
+                    if (use_q) {
+                        const int pd = find(lt[e].i);
+                        const float q = pd >= 0 ? ex2(fmaf(ld[pd].v, c, -dst.msc)) * dst.invS : 0.f;
+                        w = fmaxf(pt - q, 0.f);
+                    }
+                    wv[e] = w;
+                }
+                __syncthreads();
+                if (warp == 0) {
+                    float W = 0.f;
                     for (int base = 0; base < nt; base += 32) {
-                        const float w = (base + lane < nt) ? weight(base + lane) : 0.f;
+                        const float w = (base + lane < nt) ? wv[base + lane] : 0.f;
                         const float incl = warp_incl_scan(w, lane);
                         W += __shfl_sync(0xffffffffu, incl, 31);
                     }
-                    if (W > 0.f || !use_q) break;
-                    use_q = false;  // zero residual mass: redraw from p at this position
+                    if (lane == 0) S.W = W;
                 }
-                const float x = u * W;
+                __syncthreads();
+                if (S.W > 0.f || !use_q) break;
+                use_q = false;  // zero residual mass: redraw from p at this position
+                __syncthreads();
+            }
+            if (warp == 0) {
+                const float x = u * S.W;
                 float carry = 0.f;
                 int token = -1;
                 for (int base = 0; base < nt; base += 32) {
-                    const float w = (base + lane < nt) ? weight(base + lane) : 0.f;
+                    const float w = (base + lane < nt) ? wv[base + lane] : 0.f;
                     const float incl = warp_incl_scan(w, lane);
                     const unsigned hit = __ballot_sync(0xffffffffu, base + lane < nt && carry + incl > x);
                     if (hit) {
@@ -493,7 +551,7 @@ __global__ void __launch_bounds__(SEQ_NT, 3) sv_seq_kernel(const SeqParams P) {
                 if (token < 0) {  // rounding: the last entry with positive weight
                     int lastp = -1;
                     for (int base = 0; base < nt; base += 32) {
-                        const float w = (base + lane < nt) ? weight(base + lane) : 0.f;
+                        const float w = (base + lane < nt) ? wv[base + lane] : 0.f;
                         const unsigned pos = __ballot_sync(0xffffffffu, w > 0.f);
                         if (pos) lastp = base + 31 - __clz(pos);
                     }
