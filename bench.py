@@ -36,8 +36,9 @@ FALLBACK_HBM_GBS = 6650.0
 PROFILE_DIR = os.path.join(ROOT, "profiles")
 KSAMPLE = 8  # timed steps per streaming-kernel event sample
 
+# sources that define the streaming kernel (the one the roofline figures describe)
 KERNEL_SOURCES = [os.path.join(ROOT, "draft_token_verification_verify_b200", "csrc", f)
-                  for f in ("sv_common.cuh", "sv_rows.cuh", "sv_seq.cuh", "sv_resid.cuh", "sv_ptx.cuh", "spec_verify.cu")]
+                  for f in ("sv_rows.cuh", "sv_common.cuh", "sv_ptx.cuh")]
 
 DESCR = {
     "tiny": "tiny stochastic verify B=1 k=4 V=32 fp32 T=1",
@@ -53,6 +54,28 @@ def dist_env():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     return world, rank, local
+
+
+def rank_seed(rank: int) -> int:
+    """Seed of a rank's batch: every rank verifies its own, independent batch."""
+    return 1000 + rank
+
+
+def max_over_ranks(ms: float, device=None) -> float:
+    """The slowest rank's time (MAX all-reduce); unchanged without a process group."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return ms
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(units_per_rank: float, world: int, ms: float) -> float:
+    """Whole-job throughput: the units of all ranks over the slowest rank's time."""
+    return units_per_rank * world / (ms / 1000.0)
 
 
 def measured_peak():
@@ -245,7 +268,7 @@ def run_ours(args):
 
     name = args.workload
     w = workloads.WORKLOADS[name]
-    case = workloads.make_case(name, seed=1000 + rank)
+    case = workloads.make_case(name, seed=rank_seed(rank))
     B, k, V = case.B, case.k, case.V
     greedy = case.mode == "greedy"
     mode = (sv.SV_MODE_GREEDY if greedy else sv.SV_MODE_STOCHASTIC) | (
@@ -326,18 +349,13 @@ def run_ours(args):
     if world > 1:
         torch.distributed.barrier()
     clocks = sampler.stop()
-    elapsed_ms = t_start.elapsed_time(t_stop)
+    elapsed_ms = max_over_ranks(t_start.elapsed_time(t_stop), dev)
     kern_ms = [a.elapsed_time(b) for a, b in evk]
-    if world > 1:
-        t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
     if int(status.item()) != 0:
         raise SystemExit(f"device status {int(status.item())} in the timed region")
 
-    units = B * k * args.steps * world
-    value = units / (elapsed_ms / 1000.0)
-    gbs = logit_bytes * args.steps * world / (elapsed_ms / 1000.0) / 1e9
+    value = job_rate(B * k * args.steps, world, elapsed_ms)
+    gbs = job_rate(logit_bytes * args.steps, world, elapsed_ms) / 1e9
     kmean = sum(kern_ms) / len(kern_ms)
     peak, peak_src = measured_peak()
     achieved = logit_bytes / (kmean / 1000.0) / 1e9
@@ -387,12 +405,8 @@ def run_ours(args):
             e2e_step()
         b.record(stream)
         torch.cuda.synchronize()
-        e_ms = a.elapsed_time(b)
-        if world > 1:
-            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": B * k * n_e2e * world / (e_ms / 1000.0), "unit": "positions/s",
+        e_ms = max_over_ranks(a.elapsed_time(b), dev)
+        e2e = {"value": job_rate(B * k * n_e2e, world, e_ms), "unit": "positions/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": n_e2e}
 
     cpu = None
