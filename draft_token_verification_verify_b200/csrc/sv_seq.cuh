@@ -218,6 +218,117 @@ __global__ void __launch_bounds__(SEQ_NT, 3) sv_seq_kernel(const SeqParams P) {
         return base;
     };
 
+    // ---- fast path: top-k, one chunk per row, every row clean ---------------------------
+    // Warp 0 alone finishes the sequence: lane r holds row r's statistics, the
+    // decisions come from shuffles and a ballot, and the draw reads the kept
+    // lists already in shared memory.  Same arithmetic as the block path below.
+    if (P.pre && nrows <= 32) {
+        const bool clean = tid >= nrows || (prec[tid].flags == 0 && prec[tid].m == prec[tid].m &&
+                                            prec[tid].m != POS_INF && prec[tid].m != NEG_INF);
+        if (__syncthreads_and(clean) && !S.err) {
+            if (warp != 0) return;
+            const ChunkRec rec = prec[lane < nrows ? lane : 0];
+            const float msc = rec.m * c, invS = 1.f / rec.s, tau = rec.tau, zd = rec.zd;
+            // decisions: lane i < k holds target row i; draft row i is lane k+1+i
+            int j = k;
+            for (int i0 = 0; i0 < k; i0 += 32) {
+                const int i = i0 + lane;
+                const int src_t = i < k ? i : 0, src_d = i < k ? k + 1 + i : 0;
+                const float t_msc = __shfl_sync(0xffffffffu, msc, src_t & 31), t_inv = __shfl_sync(0xffffffffu, invS, src_t & 31);
+                const float t_tau = __shfl_sync(0xffffffffu, tau, src_t & 31), t_zd = __shfl_sync(0xffffffffu, zd, src_t & 31);
+                const float d_msc = __shfl_sync(0xffffffffu, msc, src_d & 31), d_inv = __shfl_sync(0xffffffffu, invS, src_d & 31);
+                const float d_tau = __shfl_sync(0xffffffffu, tau, src_d & 31), d_zd = __shfl_sync(0xffffffffu, zd, src_d & 31);
+                bool rej = false;
+                if (i < k) {
+                    const float p = (t_zd >= t_tau) ? ex2(fmaf(t_zd, c, -t_msc)) * t_inv : 0.f;
+                    const float q = (d_zd >= d_tau) ? ex2(fmaf(d_zd, c, -d_msc)) * d_inv : 0.f;
+                    if (P.out_p) P.out_p[b * k + i] = p;
+                    if (P.out_q) P.out_q[b * k + i] = q;
+                    rej = !(uu[i] * q < p);
+                }
+                const unsigned m = __ballot_sync(0xffffffffu, rej);
+                if (m && j == k) j = i0 + __ffs(m) - 1;  // the first rejection
+            }
+            // draw from the kept lists of position j
+            const bool use_q0 = j < k;
+            const float t_msc = __shfl_sync(0xffffffffu, msc, j), t_inv = __shfl_sync(0xffffffffu, invS, j);
+            const int nt = __shfl_sync(0xffffffffu, rec.n, j);
+            const int jd = use_q0 ? k + 1 + j : 0;
+            const float d_msc = __shfl_sync(0xffffffffu, msc, jd), d_inv = __shfl_sync(0xffffffffu, invS, jd);
+            const int nd = use_q0 ? __shfl_sync(0xffffffffu, rec.n, jd) : 0;
+            const Cand* lt = plist + static_cast<size_t>(j) * P.kcap;
+            const Cand* ld = plist + static_cast<size_t>(jd) * P.kcap;
+            float* wv = reinterpret_cast<float*>(gbuf);
+            const float u = uu[k];
+            auto find = [&](int v) {
+                int a = 0, z = nd - 1;
+                while (a <= z) {
+                    const int mid = (a + z) >> 1;
+                    const int x = ld[mid].i;
+                    if (x == v) return mid;
+                    if (x < v) a = mid + 1; else z = mid - 1;
+                }
+                return -1;
+            };
+            bool use_q = use_q0;
+            float W = 0.f;
+            for (int attempt = 0; attempt < 2; ++attempt) {
+                for (int e = lane; e < nt; e += 32) {
+                    const float pt = ex2(fmaf(lt[e].v, c, -t_msc)) * t_inv;
+                    float w = pt;
+                    if (use_q) {
+                        const int pd = find(lt[e].i);
+                        const float q = pd >= 0 ? ex2(fmaf(ld[pd].v, c, -d_msc)) * d_inv : 0.f;
+                        w = fmaxf(pt - q, 0.f);
+                    }
+                    wv[e] = w;
+                }
+                __syncwarp();
+                W = 0.f;
+                for (int base = 0; base < nt; base += 32) {
+                    const float w = (base + lane < nt) ? wv[base + lane] : 0.f;
+                    const float incl = warp_incl_scan(w, lane);
+                    W += __shfl_sync(0xffffffffu, incl, 31);
+                }
+                if (W > 0.f || !use_q) break;
+                use_q = false;  // zero residual mass: redraw from p at this position
+                __syncwarp();
+            }
+            const float x = u * W;
+            float carry = 0.f;
+            int token = -1;
+            for (int base = 0; base < nt; base += 32) {
+                const float w = (base + lane < nt) ? wv[base + lane] : 0.f;
+                const float incl = warp_incl_scan(w, lane);
+                const unsigned hit = __ballot_sync(0xffffffffu, base + lane < nt && carry + incl > x);
+                if (hit) {
+                    token = lt[base + __ffs(hit) - 1].i;
+                    break;
+                }
+                carry += __shfl_sync(0xffffffffu, incl, 31);
+            }
+            if (token < 0) {  // rounding: the last entry with positive weight
+                int lastp = -1;
+                for (int base = 0; base < nt; base += 32) {
+                    const float w = (base + lane < nt) ? wv[base + lane] : 0.f;
+                    const unsigned pos = __ballot_sync(0xffffffffu, w > 0.f);
+                    if (pos) lastp = base + 31 - __clz(pos);
+                }
+                token = lastp >= 0 ? lt[lastp].i : -1;
+            }
+            // outputs
+            const bool err = token < 0;
+            if (P.sample_only) {
+                if (lane == 0) P.out_tokens[b] = err ? -1 : token;
+            } else {
+                int32_t* out = P.out_tokens + b * (k + 1);
+                for (int i = lane; i <= k; i += 32) out[i] = err ? -1 : (i < j ? dtok[i] : (i == j ? token : -1));
+                if (lane == 0) P.out_n[b] = err ? -1 : j;
+            }
+            return;
+        }
+    }
+
     // ---- phase 1: per-row statistics (one warp per row) ----------------------------
     for (int rr = warp; rr < nrows; rr += NW) {
         const long long r = row_index(rr);
