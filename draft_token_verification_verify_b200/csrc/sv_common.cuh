@@ -1,6 +1,5 @@
 // Shared device definitions of the verification kernels: workspace records,
-// element unpacking, order-preserving keys, warp and block reductions, and a
-// shared-memory bitonic sort.
+// element unpacking, order-preserving keys and warp reductions.
 #pragma once
 
 #include <cstdint>
@@ -143,11 +142,6 @@ __device__ __forceinline__ float warp_max_nan(float x) {
     for (int o = 16; o > 0; o >>= 1) x = fmax_nan(x, __shfl_xor_sync(0xffffffffu, x, o));
     return x;
 }
-__device__ __forceinline__ int warp_sum_i(int x) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-    return x;
-}
 __device__ __forceinline__ float warp_incl_scan(float x, int lane) {
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -172,37 +166,6 @@ __device__ __forceinline__ void ms_combine(float& m, float& s, float m2, float s
 // lower index (unsigned, so that -1 = "none" loses every tie).
 __device__ __forceinline__ bool arg_better(float v1, int i1, float v2, int i2) {
     return v1 > v2 || (v1 == v2 && static_cast<unsigned>(i1) < static_cast<unsigned>(i2));
-}
-
-// Block-wide bitonic sort of n (a power of two, >= 2) pairs in shared memory.
-// BY_VALUE: value descending; otherwise index ascending.  Every thread of the
-// block must call it.
-template <bool BY_VALUE>
-__device__ __forceinline__ void block_sort(float* key, int* idx, int n) {
-    for (int size = 2; size <= n; size <<= 1) {
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            for (int t = threadIdx.x; t < (n >> 1); t += blockDim.x) {
-                const int lo = 2 * stride * (t / stride) + (t % stride);
-                const int hi = lo + stride;
-                const bool up = (lo & size) == 0;  // this half sorts in the primary order
-                const float ka = key[lo], kb = key[hi];
-                const int ia = idx[lo], ib = idx[hi];
-                bool swap;
-                if constexpr (BY_VALUE) {
-                    swap = up ? (kb > ka) : (ka > kb);
-                } else {
-                    swap = up ? (ib < ia) : (ia < ib);
-                }
-                if (swap) {
-                    key[lo] = kb;
-                    key[hi] = ka;
-                    idx[lo] = ib;
-                    idx[hi] = ia;
-                }
-            }
-            __syncthreads();
-        }
-    }
 }
 
 __host__ __device__ constexpr int pow2_ceil(int n) {
