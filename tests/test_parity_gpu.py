@@ -99,6 +99,26 @@ def test_greedy_reduced_with_ties():
     check_case(case)
 
 
+def test_greedy_full_size_sampled():
+    """Full launch shape of the greedy workload (B=256, k=8, V=151936 bf16, ties
+    in 1 % of target rows); the oracle checks a sample, bit-exact."""
+    case = workloads.make_case("greedy", seed=6)
+    drafts = oracle.draft_tokens_for(case)
+    gpu = run_gpu(case.target, None, drafts, None, None, 0, greedy=True)
+    pick = np.unique(np.linspace(0, case.B - 1, 32).astype(int))
+    ref = oracle.verify(case.target[pick], None, drafts[pick], None, case.temperature[pick], 0, True)
+    assert np.array_equal(gpu.n_accepted[pick], ref.n_accepted)
+    assert np.array_equal(gpu.tokens[pick], ref.tokens)
+    # properties at any size: accepted prefix equals the drafts, one target token, then -1
+    for b in range(case.B):
+        n = gpu.n_accepted[b]
+        assert 0 <= n <= case.k
+        assert np.array_equal(gpu.tokens[b, :n], drafts[b, :n])
+        assert 0 <= gpu.tokens[b, n] < case.V and np.all(gpu.tokens[b, n + 1:] == -1)
+        if n < case.k:
+            assert gpu.tokens[b, n] != drafts[b, n]  # the first mismatch is replaced
+
+
 def test_large_reduced_mixed_temperature():
     case = workloads.make_case("large", seed=4, B=24)
     assert len(set(case.temperature.tolist())) > 1
