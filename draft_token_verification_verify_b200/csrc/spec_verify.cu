@@ -62,7 +62,7 @@ const DeviceInfo* device_info(int* dev_out) {
             d.ok = 0;
             return;
         }
-        d.ok = major >= 9 ? 1 : 0;
+        d.ok = major == 10 ? 1 : 0;  // the kernels are built for sm_100a only
         d.id = dev;
     });
     *dev_out = dev;

@@ -44,7 +44,8 @@
  *     launch (B <= 0, k < 1, V < 1, top_k < 0, unknown mode or dtype bits,
  *     a required pointer NULL or misaligned, sizes that overflow, a
  *     workspace that is too small or misaligned);
- *   - SV_ERR_UNSUPPORTED: no usable CUDA device of compute capability >= 9.0,
+ *   - SV_ERR_UNSUPPORTED: the current device is not of compute capability 10.0
+ *     (the kernels are built for sm_100a),
  *     or sizes whose per-sequence shared-memory needs exceed the device
  *     (about k > 1000);
  *   - SV_ERR_CUDA: a CUDA call failed while launching;
@@ -93,7 +94,7 @@ enum {
  * the library's own choices. */
 typedef struct sv_options {
     int chunks_per_row;        /* streaming tasks per logit row: 0 = auto, else >= 1 */
-    int threads;               /* threads per streaming CTA: 0 = auto (256), else 128, 256 or 512 */
+    int threads;               /* consumer threads per streaming CTA: 0 = auto, else 128, 256 or 512 */
     int topk_path;             /* 0 = auto, 1 = kept lists, 2 = radix select */
     void* event_start;         /* cudaEvent_t or NULL, recorded before the streaming kernel */
     void* event_stop;          /* cudaEvent_t or NULL, recorded right after it */
