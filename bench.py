@@ -298,11 +298,11 @@ def run_ours(args):
     wbytes = sv.spec_verify_workspace_size(B, k, V, case.top_k, mode)
     wsp = torch.empty((max(wbytes, 1),), dtype=torch.uint8, device=dev)
 
-    def step(i, ev0=None, ev1=None):
+    def step(i, ev0=None, ev1=None, on=None):
         opts = sv.make_options(event_start=ev0, event_stop=ev1) if ev0 is not None else None
         st = sv.spec_verify_ex(targets[i % nsets], drafts_l[i % nsets], drafts, unif, B, k, V, temp,
                                case.top_k, mode, out_tok, out_n, None, None, status, wsp, wbytes, opts,
-                               stream)
+                               stream if on is None else on)
         if st != sv.SV_OK:
             raise sv.SpecVerifyError(st, "spec_verify_ex")
 
@@ -409,6 +409,32 @@ def run_ours(args):
         e2e = {"value": job_rate(B * k * n_e2e, world, e_ms), "unit": "positions/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": n_e2e}
 
+    # ---- optional: the same steps replayed from a CUDA graph (launch-bound workloads) ---
+    graph = None
+    if args.graph:
+        gs = torch.cuda.Stream(device=dev)
+        gs.wait_stream(stream)
+        per_graph = 16
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=gs):
+            for i in range(per_graph):
+                step(i, on=gs)
+        rs = torch.cuda.current_stream()  # replay() launches the graph on the current stream
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        reps = max(3, args.steps // per_graph)
+        ga, gb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ga.record(rs)
+        for _ in range(reps):
+            g.replay()
+        gb.record(rs)
+        torch.cuda.synchronize()
+        g_ms = max_over_ranks(ga.elapsed_time(gb), dev) / (reps * per_graph)
+        graph = {"value": job_rate(B * k, world, g_ms), "unit": "positions/s", "ms_per_step": g_ms,
+                 "steps_per_graph": per_graph}
+        del g
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(name, case, drafts.cpu().numpy(), args.cpu_budget)
@@ -437,6 +463,7 @@ def run_ours(args):
         "gpu_launches": launches_per_step(case) * args.steps,
         "clocks": clocks,
         "e2e": e2e,
+        **({"graph": graph} if graph is not None else {}),
         "cpu_baseline": cpu,
     }
     print(json.dumps(line), flush=True)
@@ -454,6 +481,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--graph", action="store_true",
+                    help="also time the steps replayed from a CUDA graph (latency-bound workloads)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
