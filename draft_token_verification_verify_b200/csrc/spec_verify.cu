@@ -97,7 +97,7 @@ long long round_up(long long a, long long b) { return ceil_div(a, b) * b; }
 struct Plan {
     int mode = 0, elt = 2, seg = 0, nseg = 0, nch = 1, spc = 1, nt1 = 128, stages = kStages;
     int lcap = 0, kcap = 0, mg = 0;
-    long long R = 0, tasks = 0;
+    long long R = 0, tasks = 0, slots = 0;
     size_t smem1 = 0, smem2 = 0;
     size_t off_chunks = 0, off_cands = 0, ws_bytes = 0;
     bool defer = false;  // residual draws by the segment kernel
@@ -147,6 +147,7 @@ sv_status_t make_plan(const DeviceInfo& dev, long long seqs, int k, int V, int d
     long long occ = rows_occupancy(dev.id, dt, p.nt1, p.mode, p.smem1);
     if (occ < 1) return SV_ERR_CUDA;
     const long long slots = occ * dev.sms;
+    p.slots = slots;
     int nch;
     if (opts && opts->chunks_per_row) {
         nch = opts->chunks_per_row;
@@ -398,6 +399,17 @@ sv_status_t run(const Call& cl, void* workspace, size_t workspace_bytes, const s
         c1.blockDim = dim3(p.nt1 + 32, 1, 1);  // consumer warps + the producer warp
         c1.dynamicSmemBytes = p.smem1;
         c1.stream = st;
+        // programmatic dependent launch: the streaming pass may be placed while
+        // the preceding kernel finishes (it waits for that grid before any
+        // access).  Not for a single wave that fills more than half the device:
+        // CTAs placed early, as slots free up, spread unevenly over the SMs and
+        // such a grid has no later wave to even it out.
+        cudaLaunchAttribute a1[1];
+        a1[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        a1[0].val.programmaticStreamSerializationAllowed = 1;
+        const bool tight_wave = p.tasks > p.slots / 2 && p.tasks <= p.slots;
+        c1.attrs = tight_wave ? nullptr : a1;
+        c1.numAttrs = tight_wave ? 0 : 1;
         if (cudaLaunchKernelEx(&c1, f1, r) != cudaSuccess) {
             result = SV_ERR_CUDA;
             break;

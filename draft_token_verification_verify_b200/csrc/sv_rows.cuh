@@ -206,6 +206,11 @@ __global__ void __launch_bounds__(NT + 32, RowsOcc<NT>::value) sv_rows_kernel(co
         b = (r - Rt) / P.k;
         pos = static_cast<int>((r - Rt) - b * P.k);
     }
+    // Launched as a programmatic dependent of whatever precedes it on the
+    // stream (typically the previous call's per-sequence kernel, which lets its
+    // dependents start early): nothing is read or written before the
+    // preceding grid has completed.  A no-op when it did not start early.
+    pdl_wait_primary();
     if (task == 0 && tid == 0 && P.out_status) *P.out_status = 0;
     pdl_launch_dependents();
 
