@@ -1,8 +1,8 @@
 // Host side of the spec_verify C ABI: argument checks, launch planning,
-// workspace handling and the launches: the streaming pass, then the
-// per-sequence kernel as a programmatic dependent launch, then (softmax
-// verification only) the segment kernel of the residual draws, also as a
-// programmatic dependent launch.  Nothing here
+// workspace handling and the launches, each a programmatic dependent launch
+// of the one before it: the streaming pass (except for a single wave that
+// fills more than half the device), the per-sequence kernel, and for softmax
+// verification the segment kernel of the residual draws.  Nothing here
 // synchronises the caller's stream.
 #include <cuda_runtime.h>
 

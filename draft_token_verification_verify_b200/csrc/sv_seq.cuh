@@ -9,15 +9,17 @@
 // through the inverse CDF in index order.  Greedy mode compares d_i with the
 // lowest-index argmax of the target row.
 //
-// Draws: with top-k, from the kept lists gathered by the streaming pass (no
-// logit is read again); without top-k, the bonus draw locates its segment
-// from the streaming partials and rescans that segment only, while a
-// residual draw is handed to the segment kernel (one CTA per segment of the
-// rejected (target, draft) pair).  The rare cases left here (zero-mass
-// retries of top-k rows resolved by radix select) stream the pair in this
-// CTA.  Rows whose
-// kept list did not fit (massive ties) or top-k above the list capacity fall
-// back to an exact radix select over the row in global memory.
+// Paths: with top-k and one chunk per row, every row's chunk record and kept
+// list arrive in one round of loads, and a sequence whose rows are all clean
+// is finished by warp 0 alone (lane r holds row r; decisions by ballot; the
+// draw over the kept lists in shared memory).  Otherwise the block path
+// merges the partials with one warp per row.  Draws without top-k: a bonus
+// draw locates its segment from the streaming partials and rescans that
+// segment; a residual draw is handed to the segment kernel (one CTA per
+// segment of the rejected (target, draft) pair).  Rows whose kept list did
+// not fit (massive ties), or top-k resolved by radix select, get an exact
+// radix select over the row in global memory and a draw that streams the
+// row (pair) in this CTA.
 #pragma once
 
 #include <climits>
