@@ -36,6 +36,13 @@ def lib():
         _lib.oracle_verify.restype = I
         _lib.oracle_sample_rows.argtypes = [P, I, I, I, P, I, I, P, P, P, P]
         _lib.oracle_sample_rows.restype = I
+        _lib.oracle_process_row_procs.argtypes = [P, I, I, D, I, P, P, P, P]
+        _lib.oracle_process_row_procs.restype = I
+        _lib.oracle_verify_procs.argtypes = [P, P, P, P, I, I, I, P, I, I, P, P, P, I, P,
+                                             P, P, P, P, P, P, P]
+        _lib.oracle_verify_procs.restype = I
+        _lib.oracle_sample_rows_procs.argtypes = [P, I, I, I, I, P, I, P, P, P, I, P, P, P]
+        _lib.oracle_sample_rows_procs.restype = I
     return _lib
 
 
@@ -161,3 +168,97 @@ def draft_tokens_for(case) -> np.ndarray:
     temp = np.repeat(case.temperature, case.k)
     tok, _, _ = sample_rows(case.draft, case.draft_uniforms, temp, case.top_k)
     return tok.astype(np.int32)
+
+
+# ---- further logits processors (readings R12..R15 in spec_verify_oracle.c) -----------
+
+class _Procs(ctypes.Structure):
+    """Mirror of the oracle's ``or_procs_t``."""
+    _fields_ = [("top_p", ctypes.c_double), ("rep_penalty", ctypes.c_double),
+                ("rep_ids", ctypes.c_void_p), ("n_rep", ctypes.c_int), ("mask", ctypes.c_void_p)]
+
+
+def allow_mask(V: int, allowed) -> np.ndarray:
+    """Bitmask words (uint32, ceil(V/32)) allowing exactly the token ids in ``allowed``."""
+    words = np.zeros((V + 31) // 32, dtype=np.uint32)
+    for v in np.asarray(allowed, dtype=np.int64).ravel():
+        words[v // 32] |= np.uint32(1) << np.uint32(v % 32)
+    return words
+
+
+def process_row_procs(row: np.ndarray, temperature: float = 1.0, top_k: int = 0, top_p: float = 1.0,
+                      rep_penalty: float = 1.0, rep_ids=None, mask: Optional[np.ndarray] = None):
+    """Processed probabilities of one row with the further processors, or None on a row error."""
+    row = np.ascontiguousarray(row)
+    V = row.shape[-1]
+    ids = None if rep_ids is None else np.ascontiguousarray(rep_ids, dtype=np.int32).ravel()
+    msk = None if mask is None else np.ascontiguousarray(mask, dtype=np.uint32).ravel()
+    pr = _Procs(float(top_p), float(rep_penalty), None if ids is None else ids.ctypes.data,
+                0 if ids is None else ids.size, None if msk is None else msk.ctypes.data)
+    prob = np.zeros(V, dtype=np.float64)
+    work = np.zeros(V, dtype=np.float64)
+    pv = np.zeros(2 * V, dtype=np.float64)  # V (double, long) pairs
+    rc = lib().oracle_process_row_procs(_ptr(row), _dtype_code(row), V, float(temperature), int(top_k),
+                                        ctypes.byref(pr), _ptr(prob), _ptr(work), _ptr(pv))
+    return None if rc else prob
+
+
+def _seq_arrays(B, V, top_p, rep_penalty, rep_ids, mask):
+    tp = None if top_p is None else np.ascontiguousarray(np.broadcast_to(np.asarray(top_p, np.float32), (B,)))
+    rp = None if rep_penalty is None else np.ascontiguousarray(
+        np.broadcast_to(np.asarray(rep_penalty, np.float32), (B,)))
+    ids, n_rep = None, 0
+    if rep_ids is not None:
+        ids = np.ascontiguousarray(rep_ids, dtype=np.int32).reshape(B, -1)
+        n_rep = ids.shape[1]
+    msk = None if mask is None else np.ascontiguousarray(mask, dtype=np.uint32).reshape(B, (V + 31) // 32)
+    return tp, rp, ids, n_rep, msk
+
+
+def verify_procs(target, draft, draft_tokens, uniforms, temperature=None, top_k: int = 0, top_p=None,
+                 rep_penalty=None, rep_ids=None, mask=None) -> VerifyResult:
+    """``verify`` (stochastic) with per-sequence processors: top_p [B] or scalar,
+    rep_penalty [B] or scalar, rep_ids [B, n] (-1 = unused), mask [B, ceil(V/32)]."""
+    target = np.ascontiguousarray(target)
+    B, k1, V = target.shape
+    k = k1 - 1
+    draft = np.ascontiguousarray(draft)
+    assert draft.dtype == target.dtype and draft.shape == (B, k, V)
+    draft_tokens = np.ascontiguousarray(draft_tokens, dtype=np.int32).reshape(B, k)
+    uniforms = np.ascontiguousarray(uniforms, dtype=np.float32).reshape(B, k + 1)
+    if temperature is not None:
+        temperature = np.ascontiguousarray(temperature, dtype=np.float32).reshape(B)
+    tp, rp, ids, n_rep, msk = _seq_arrays(B, V, top_p, rep_penalty, rep_ids, mask)
+    tokens = np.empty((B, k + 1), dtype=np.int32)
+    n = np.empty(B, dtype=np.int32)
+    p = np.empty((B, k), dtype=np.float64)
+    q = np.empty_like(p)
+    ratio = np.empty_like(p)
+    lo = np.empty(B, dtype=np.float64)
+    hi = np.empty(B, dtype=np.float64)
+    errs = lib().oracle_verify_procs(_ptr(target), _ptr(draft), _ptr(draft_tokens), _ptr(uniforms), B, k,
+                                     V, _ptr(temperature), int(top_k), _dtype_code(target), _ptr(tp),
+                                     _ptr(rp), _ptr(ids), n_rep, _ptr(msk), _ptr(tokens), _ptr(n),
+                                     _ptr(p), _ptr(q), _ptr(ratio), _ptr(lo), _ptr(hi))
+    if errs < 0:
+        raise MemoryError("oracle_verify_procs could not allocate its work arrays")
+    return VerifyResult(tokens, n, p, q, ratio, lo, hi, errs)
+
+
+def sample_rows_procs(logits, u, temperature=None, top_k: int = 0, top_p=None, rep_penalty=None,
+                      rep_ids=None, mask=None) -> np.ndarray:
+    """The proposer's draw with processors: logits [B, rows_per_seq, V], u [B, rows_per_seq];
+    processors per sequence as in ``verify_procs``."""
+    logits = np.ascontiguousarray(logits)
+    B, rps, V = logits.shape
+    u = np.ascontiguousarray(u, dtype=np.float32).reshape(B * rps)
+    if temperature is not None:
+        temperature = np.ascontiguousarray(temperature, dtype=np.float32).reshape(B * rps)
+    tp, rp, ids, n_rep, msk = _seq_arrays(B, V, top_p, rep_penalty, rep_ids, mask)
+    out = np.empty(B * rps, dtype=np.int32)
+    errs = lib().oracle_sample_rows_procs(_ptr(logits), _dtype_code(logits), B * rps, rps, V,
+                                          _ptr(temperature), int(top_k), _ptr(tp), _ptr(rp), _ptr(ids),
+                                          n_rep, _ptr(msk), _ptr(u), _ptr(out))
+    if errs < 0:
+        raise MemoryError("oracle_sample_rows_procs could not allocate its work arrays")
+    return out.reshape(B, rps)

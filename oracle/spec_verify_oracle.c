@@ -305,3 +305,248 @@ int oracle_sample_rows(const void* logits, int dtype, int rows, int V, const flo
     free(prob); free(work);
     return errors;
 }
+
+/* ==== further logits processors ============================================
+ *
+ * Section "提议与核验的基本步骤", paragraph 4, names nucleus sampling,
+ * repetition penalties and vocabulary masks (with temperature and top-k) among
+ * the processing rules that must be applied to the target and the draft
+ * distributions alike, and kept consistent in the correction step.  The page
+ * does not define them; the readings taken here:
+ *   R12 order: repetition penalty and vocabulary mask act on the raw logits,
+ *       then top-k (R4) on the result, then temperature and the softmax (R5),
+ *       then the nucleus on the resulting probabilities;
+ *   R13 repetition penalty theta > 0 on the sequence's listed token ids (each
+ *       id once, ids outside [0, V) ignored): z -> z / theta if z > 0, else
+ *       z * theta;
+ *   R14 vocabulary mask: token v is allowed iff bit (v % 32) of word v / 32 is
+ *       set; a disallowed token gets the logit -inf (probability 0);
+ *   R15 nucleus 0 < top_p <= 1: order the tokens of positive probability by
+ *       probability descending (equal ones by index), take the first at which
+ *       the running sum reaches top_p, keep every token whose probability is
+ *       >= that token's (equal probabilities are all kept), renormalise;
+ *       top_p = 1 keeps every token.
+ * The same processors apply to every target and draft row of a sequence. */
+
+typedef struct {
+    double top_p;           /* R15, 1 disables */
+    double rep_penalty;     /* R13, 1 disables */
+    const int32_t* rep_ids; /* n_rep ids, or NULL */
+    int n_rep;
+    const uint32_t* mask;   /* ceil(V/32) words, or NULL (all allowed) */
+} or_procs_t;
+
+typedef struct {
+    double p;
+    long v;
+} or_pv_t;
+
+static int cmp_pv_desc(const void* a, const void* b) {
+    const or_pv_t* x = (const or_pv_t*)a;
+    const or_pv_t* y = (const or_pv_t*)b;
+    if (x->p > y->p) return -1;
+    if (x->p < y->p) return 1;
+    return (x->v > y->v) - (x->v < y->v);
+}
+
+/* Raw logit of token v after the repetition penalty and the mask (R13, R14). */
+static double or_logit_procs(const void* row, int dtype, long v, const or_procs_t* pr) {
+    double z = or_logit(row, dtype, v);
+    int i;
+    if (pr->mask && !((pr->mask[v / 32] >> (v % 32)) & 1u)) return -INFINITY;
+    if (pr->rep_ids && pr->rep_penalty != 1.0) {
+        for (i = 0; i < pr->n_rep; ++i) {
+            if (pr->rep_ids[i] == v) {
+                z = z > 0.0 ? z / pr->rep_penalty : z * pr->rep_penalty;
+                break; /* each id once */
+            }
+        }
+    }
+    return z;
+}
+
+/*
+ * oracle_process_row with the processors of R12..R15.  `work` holds V
+ * doubles, `pv` V pairs (only used when top_p < 1).  Returns 0, or 1 for a
+ * row error (R7; every token disallowed counts as "no finite kept logit").
+ */
+int oracle_process_row_procs(const void* row, int dtype, int V, double T, int top_k,
+                             const or_procs_t* pr, double* prob, double* work, void* pv_buf) {
+    long v, n = 0, i;
+    double tau = -INFINITY, m = -INFINITY, S = 0.0;
+    if (!(T > 0.0) || isinf(T)) return 1;
+    if (!(pr->top_p > 0.0 && pr->top_p <= 1.0) || !(pr->rep_penalty > 0.0)) return 1;
+    for (v = 0; v < V; ++v) {
+        double z0 = or_logit(row, dtype, v);
+        if (isnan(z0) || z0 == INFINITY) return 1;
+        work[v] = or_logit_procs(row, dtype, v, pr);
+    }
+    for (v = 0; v < V; ++v) prob[v] = work[v]; /* processed logits, kept for below */
+    if (top_k > 0 && top_k < V) {
+        qsort(work, (size_t)V, sizeof(double), cmp_desc);
+        tau = work[top_k - 1];
+    }
+    for (v = 0; v < V; ++v)
+        if (prob[v] >= tau && prob[v] / T > m) m = prob[v] / T;
+    if (m == -INFINITY) return 1;
+    for (v = 0; v < V; ++v) {
+        double z = prob[v];
+        prob[v] = (z >= tau) ? exp(z / T - m) : 0.0;
+        S += prob[v];
+    }
+    for (v = 0; v < V; ++v) prob[v] /= S;
+    if (pr->top_p < 1.0) {
+        or_pv_t* pv = (or_pv_t*)pv_buf;
+        double run = 0.0, cut = 0.0, K2 = 0.0;
+        for (v = 0; v < V; ++v)
+            if (prob[v] > 0.0) {
+                pv[n].p = prob[v];
+                pv[n].v = v;
+                ++n;
+            }
+        qsort(pv, (size_t)n, sizeof(or_pv_t), cmp_pv_desc);
+        cut = n > 0 ? pv[n - 1].p : 0.0;
+        for (i = 0; i < n; ++i) {
+            run += pv[i].p;
+            if (run >= pr->top_p) {
+                cut = pv[i].p;
+                break;
+            }
+        }
+        for (v = 0; v < V; ++v) {
+            if (!(prob[v] >= cut)) prob[v] = 0.0;
+            K2 += prob[v];
+        }
+        for (v = 0; v < V; ++v) prob[v] /= K2;
+    }
+    return 0;
+}
+
+/*
+ * oracle_verify with per-sequence processors (R12..R15): top_p [B] or NULL
+ * (all 1), rep_penalty [B] or NULL (all 1), rep_ids [B][n_rep] (entries < 0
+ * unused) or NULL, mask [B][ceil(V/32)] or NULL.  Same outputs and return
+ * value as oracle_verify, whose steps it follows.
+ */
+int oracle_verify_procs(const void* target, const void* draft, const int32_t* draft_tokens,
+                        const float* uniforms, int B, int k, int V, const float* temperature,
+                        int top_k, int dtype, const float* top_p, const float* rep_penalty,
+                        const int32_t* rep_ids, int n_rep, const uint32_t* mask,
+                        int32_t* out_tokens, int32_t* out_n, double* out_p, double* out_q,
+                        double* out_ratio, double* out_lo, double* out_hi) {
+    int b, i, errors = 0;
+    const long words = (V + 31) / 32;
+    double* pt = (double*)malloc(sizeof(double) * (size_t)(k + 1) * (size_t)V);
+    double* pd = (double*)malloc(sizeof(double) * (size_t)(k > 0 ? k : 1) * (size_t)V);
+    double* w = (double*)malloc(sizeof(double) * (size_t)V);
+    double* work = (double*)malloc(sizeof(double) * (size_t)V);
+    or_pv_t* pv = (or_pv_t*)malloc(sizeof(or_pv_t) * (size_t)V);
+    if (!pt || !pd || !w || !work || !pv) {
+        free(pt); free(pd); free(w); free(work); free(pv);
+        return -1;
+    }
+    for (b = 0; b < B; ++b) {
+        int32_t* tok = out_tokens + (size_t)b * (k + 1);
+        const int32_t* d = draft_tokens + (size_t)b * k;
+        const float* u = uniforms + (size_t)b * (k + 1);
+        double T = temperature ? (double)temperature[b] : 1.0;
+        or_procs_t pr;
+        int err = 0, j = k, y = -1;
+        double lo = NAN, hi = NAN;
+        pr.top_p = top_p ? (double)top_p[b] : 1.0;
+        pr.rep_penalty = rep_penalty ? (double)rep_penalty[b] : 1.0;
+        pr.rep_ids = rep_ids ? rep_ids + (size_t)b * n_rep : NULL;
+        pr.n_rep = rep_ids ? n_rep : 0;
+        pr.mask = mask ? mask + (size_t)b * words : NULL;
+        for (i = 0; i < k; ++i)
+            if (d[i] < 0 || d[i] >= V) err = 1;
+        for (i = 0; i <= k; ++i) tok[i] = -1;
+        if (out_p) for (i = 0; i < k; ++i) out_p[(size_t)b * k + i] = NAN;
+        if (out_q) for (i = 0; i < k; ++i) out_q[(size_t)b * k + i] = NAN;
+        if (out_ratio) for (i = 0; i < k; ++i) out_ratio[(size_t)b * k + i] = NAN;
+        if (!(T > 0.0) || isinf(T) || isnan(T)) err = 1;
+        for (i = 0; i <= k && !err; ++i)
+            if (!(u[i] >= 0.0f && u[i] < 1.0f)) err = 1;
+        for (i = 0; i <= k && !err; ++i)
+            err |= oracle_process_row_procs(or_row(target, dtype, (long)b * (k + 1) + i, V), dtype, V,
+                                            T, top_k, &pr, pt + (size_t)i * V, work, pv);
+        for (i = 0; i < k && !err; ++i)
+            err |= oracle_process_row_procs(or_row(draft, dtype, (long)b * k + i, V), dtype, V, T,
+                                            top_k, &pr, pd + (size_t)i * V, work, pv);
+        if (!err) {
+            long v;
+            int found = 0;
+            for (i = 0; i < k; ++i) {
+                double p = pt[(size_t)i * V + d[i]], q = pd[(size_t)i * V + d[i]];
+                if (out_p) out_p[(size_t)b * k + i] = p;
+                if (out_q) out_q[(size_t)b * k + i] = q;
+                if (out_ratio)
+                    out_ratio[(size_t)b * k + i] = q > 0.0 ? (p / q < 1.0 ? p / q : 1.0)
+                                                           : (p > 0.0 ? 1.0 : 0.0);
+                if (!found && !((double)u[i] * q < p)) {
+                    j = i;
+                    found = 1;
+                }
+            }
+            if (j < k) {
+                for (v = 0; v < V; ++v) {
+                    double r = pt[(size_t)j * V + v] - pd[(size_t)j * V + v];
+                    w[v] = r > 0.0 ? r : 0.0;
+                }
+                if (oracle_inverse_cdf(w, V, (double)u[k], &y, &lo, &hi))
+                    oracle_inverse_cdf(pt + (size_t)j * V, V, (double)u[k], &y, &lo, &hi);
+            } else {
+                oracle_inverse_cdf(pt + (size_t)k * V, V, (double)u[k], &y, &lo, &hi);
+            }
+        }
+        if (err) {
+            out_n[b] = -1;
+            errors++;
+        } else {
+            for (i = 0; i < j; ++i) tok[i] = d[i];
+            tok[j] = y;
+            out_n[b] = j;
+        }
+        if (out_lo) out_lo[b] = lo;
+        if (out_hi) out_hi[b] = hi;
+    }
+    free(pt); free(pd); free(w); free(work); free(pv);
+    return errors;
+}
+
+/* The proposer's draw (as oracle_sample_rows, stochastic) with processors:
+ * row r uses the processors of sequence r / rows_per_seq. */
+int oracle_sample_rows_procs(const void* logits, int dtype, int rows, int rows_per_seq, int V,
+                             const float* temperature, int top_k, const float* top_p,
+                             const float* rep_penalty, const int32_t* rep_ids, int n_rep,
+                             const uint32_t* mask, const float* u, int32_t* out_tokens) {
+    int r, errors = 0;
+    const long words = (V + 31) / 32;
+    double* prob = (double*)malloc(sizeof(double) * (size_t)V);
+    double* work = (double*)malloc(sizeof(double) * (size_t)V);
+    or_pv_t* pv = (or_pv_t*)malloc(sizeof(or_pv_t) * (size_t)V);
+    if (!prob || !work || !pv) {
+        free(prob); free(work); free(pv);
+        return -1;
+    }
+    for (r = 0; r < rows; ++r) {
+        const int s = r / rows_per_seq;
+        or_procs_t pr;
+        int y = -1;
+        double lo, hi, T = temperature ? (double)temperature[r] : 1.0;
+        pr.top_p = top_p ? (double)top_p[s] : 1.0;
+        pr.rep_penalty = rep_penalty ? (double)rep_penalty[s] : 1.0;
+        pr.rep_ids = rep_ids ? rep_ids + (size_t)s * n_rep : NULL;
+        pr.n_rep = rep_ids ? n_rep : 0;
+        pr.mask = mask ? mask + (size_t)s * words : NULL;
+        if ((u[r] >= 0.0f && u[r] < 1.0f) &&
+            oracle_process_row_procs(or_row(logits, dtype, r, V), dtype, V, T, top_k, &pr, prob, work,
+                                     pv) == 0) {
+            if (oracle_inverse_cdf(prob, V, (double)u[r], &y, &lo, &hi)) y = -1;
+        }
+        if (y < 0) errors++;
+        out_tokens[r] = y;
+    }
+    free(prob); free(work); free(pv);
+    return errors;
+}
