@@ -186,6 +186,27 @@ def test_k_values(k):
     check_case(workloads.make_case("tiny", seed=100 + k, B=40, k=k, V=2048, dtype="bf16"))
 
 
+@pytest.mark.parametrize("k", [15, 16])
+def test_top_k_many_positions(k):
+    """2k+1 = 31 rows take the single-warp path of the per-sequence kernel,
+    33 rows the block path."""
+    check_case(workloads.make_case("batched", seed=200 + k, B=3, k=k, V=30011, top_k=20))
+
+
+@pytest.mark.parametrize("k", [12, 20])
+def test_softmax_many_positions(k):
+    check_case(workloads.make_case("single", seed=300 + k, B=2, k=k, V=20000, dtype="f32"))
+
+
+def test_top_k_fp32_full_vocabulary():
+    check_case(workloads.make_case("large", seed=31, B=4, top_k=50))
+
+
+@pytest.mark.parametrize("K", [0, 7])
+def test_many_sequences_tiny_vocabulary(K):
+    check_case(workloads.make_case("tiny", seed=41 + K, B=3000, k=2, V=40, top_k=K))
+
+
 @pytest.mark.parametrize("T", [0.5, 1.5])
 def test_temperatures(T):
     check_case(workloads.make_case("single", seed=7, B=2, k=3, temperature=(T,)))
