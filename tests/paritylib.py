@@ -162,3 +162,17 @@ def check_case(case, drafts=None, opts=None, check_pq=True):
     print(rep)
     assert rep.flagged_accept <= max(1, 0.01 * rep.sequences), rep
     return rep
+
+
+def nucleus_near_cut(probs: np.ndarray, top_p: float, tol: float = DECISION_TOL) -> bool:
+    """True when the nucleus cut of the fp64 distribution ``probs`` (before the
+    nucleus) is a near-tie: the running sum in descending order reaches top_p
+    within ``tol`` of a step, so fp32 arithmetic may keep a different set.
+    Such rows are reported and counted, like near-threshold decisions."""
+    if top_p >= 1.0:
+        return False
+    p = np.sort(np.asarray(probs, dtype=np.float64)[probs > 0])[::-1]
+    run = np.cumsum(p)
+    i = int(np.argmax(run >= top_p))
+    before = run[i - 1] if i > 0 else 0.0
+    return abs(run[i] - top_p) < tol or abs(before - top_p) < tol

@@ -59,7 +59,7 @@ import numpy as np
 __all__ = [
     "GAMMA", "mix64", "splitmix64_stream", "stream_state", "uniform_f32",
     "normals_f64", "f64_to_bf16_bits", "bf16_bits_to_f32", "f64_to_f32",
-    "WORKLOADS", "Case", "make_case", "workload_bytes",
+    "WORKLOADS", "Case", "make_case", "workload_bytes", "Processors", "make_processors",
 ]
 
 M64 = (1 << 64) - 1
@@ -77,6 +77,9 @@ TAG_DRAFT_UNIFORMS = 5
 TAG_TEMPERATURE = 6
 TAG_TIES = 7
 TAG_PROXY_NOISE = 8
+TAG_TOP_P = 9
+TAG_REP_IDS = 10
+TAG_MASK = 11
 
 _U = np.uint64
 
@@ -309,3 +312,40 @@ def make_case(name: str, seed: int = 0, B: Optional[int] = None, k: Optional[int
     return Case(name=name, seed=seed, B=B, k=k, V=V, dtype=w.dtype, mode=w.mode, top_k=tk,
                 target=target, draft=draft, draft_proxy=proxy, uniforms=uniforms,
                 draft_uniforms=duni, temperature=temp)
+
+
+@dataclasses.dataclass
+class Processors:
+    """Per-sequence inputs of the further logits processors (repetition
+    penalty, vocabulary mask, nucleus): arrays only, no processing here."""
+    top_p: np.ndarray        # [B] fp32 in (0, 1]
+    rep_penalty: np.ndarray  # [B] fp32 > 0
+    rep_ids: np.ndarray      # [B, n_rep] int32 token ids (the sequence's history)
+    mask: np.ndarray         # [B, ceil(V/32)] uint32, bit v % 32 of word v // 32 = allowed
+
+
+def make_processors(seed: int, B: int, V: int, top_p=(0.7, 0.95), rep_penalty: float = 1.2,
+                    n_rep: int = 32, allowed_fraction: float = 0.5) -> Processors:
+    """Seeded processor inputs for B sequences: top_p uniform on the given
+    interval (or a fixed value), one penalty for every sequence, n_rep distinct
+    history ids per sequence, and a mask allowing each token with probability
+    ``allowed_fraction`` (always at least the sequence's first history id)."""
+    if isinstance(top_p, tuple):
+        lo, hi = top_p
+        tp = (lo + (hi - lo) * uniform_f32(seed, TAG_TOP_P, B, 1)[:, 0].astype(np.float64)).astype(np.float32)
+    else:
+        tp = np.full(B, top_p, dtype=np.float32)
+    rp = np.full(B, rep_penalty, dtype=np.float32)
+    n_rep = min(n_rep, V)
+    ids = np.stack([_distinct_ids(seed, TAG_REP_IDS, b, n_rep, V) for b in range(B)]).astype(np.int32)
+    allow = uniform_f32(seed, TAG_MASK, B, V) < np.float32(allowed_fraction)
+    if n_rep > 0:
+        allow[np.arange(B), ids[:, 0]] = True
+    else:
+        allow[:, 0] = True
+    words = (V + 31) // 32
+    bits = np.zeros((B, words * 32), dtype=np.uint64)
+    bits[:, :V] = allow
+    weights = (np.uint64(1) << np.arange(32, dtype=np.uint64))
+    mask = (bits.reshape(B, words, 32) * weights).sum(axis=2).astype(np.uint32)
+    return Processors(tp, rp, ids, mask)
