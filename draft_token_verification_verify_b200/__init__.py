@@ -51,6 +51,7 @@ class SvOptions(ctypes.Structure):
         ("event_stop", ctypes.c_void_p),
         ("wait_timeout_ns", ctypes.c_uint64),
         ("test_extra_tx", ctypes.c_uint32),
+        ("top_p", ctypes.c_void_p),
     ]
 
 
@@ -186,9 +187,11 @@ def spec_sample_ex(logits, uniforms, rows, V, temperature, top_k, mode, out_toke
 
 
 def make_options(chunks_per_row=0, threads=0, topk_path=0, event_start=None, event_stop=None,
-                 wait_timeout_ns=0, test_extra_tx=0) -> SvOptions:
+                 wait_timeout_ns=0, test_extra_tx=0, top_p=None) -> SvOptions:
+    """``sv_options_t``; ``top_p`` is a [B] fp32 device tensor (nucleus per
+    sequence, top-k path only) or None.  Keep it alive until the call completes."""
     return SvOptions(chunks_per_row, threads, topk_path, _event(event_start), _event(event_stop),
-                     wait_timeout_ns, test_extra_tx)
+                     wait_timeout_ns, test_extra_tx, None if top_p is None else _p(top_p).value)
 
 
 def _dtype_code(t) -> int:

@@ -300,6 +300,7 @@ sv_status_t run(const Call& cl, void* workspace, size_t workspace_bytes, const s
     sv_status_t s = make_plan(*info, cl.seqs, cl.k, cl.V, cl.dt, cl.greedy, cl.top_k, opts, &p);
     if (s != SV_OK) return s;
     if (workspace && (workspace_bytes < p.ws_bytes || !aligned(workspace, 16))) return SV_ERR_INVALID_ARG;
+    if (opts && opts->top_p && p.mode != sv::MODE_TOPK) return SV_ERR_UNSUPPORTED;  // nucleus needs the kept lists
     if ((s = set_attrs(dev, cl.dt, p.nt1, p.mode)) != SV_OK) return s;
 
     void* ws = workspace;
@@ -365,6 +366,7 @@ sv_status_t run(const Call& cl, void* workspace, size_t workspace_bytes, const s
     q.out_q = cl.out_q;
     q.out_status = cl.sample ? nullptr : cl.out_status;
     q.defer = p.defer ? 1 : 0;
+    q.top_p = opts ? opts->top_p : nullptr;
     q.pre = p.pre ? 1 : 0;
     q.pre_off = static_cast<int>(p.pre_off);
     q.req = p.defer ? reinterpret_cast<sv::DrawReq*>(base + p.off_req) : nullptr;
@@ -465,6 +467,7 @@ sv_status_t check_options(const sv_options_t* o) {
     if (!(o->threads == 0 || o->threads == 128 || o->threads == 256 || o->threads == 512))
         return SV_ERR_INVALID_ARG;
     if (o->topk_path < 0 || o->topk_path > 2) return SV_ERR_INVALID_ARG;
+    if (o->top_p && !aligned(o->top_p, 4)) return SV_ERR_INVALID_ARG;
     return SV_OK;
 }
 

@@ -57,6 +57,7 @@ struct SeqParams {
                                  // list is loaded into shared memory at offset pre_off
     int pre_off;
     int defer;                   // residual draws go to the segment kernel (softmax, verify)
+    const float* top_p;          // [B] nucleus thresholds (top-k path only) or null
     DrawReq* req;                // [B] when defer
     int* counter;                // [B] when defer: zeroed here for the segment kernel
 };
@@ -136,6 +137,7 @@ __global__ void __launch_bounds__(SEQ_NT, 3) sv_seq_kernel(const SeqParams P) {
     // ---- inputs that do not depend on the streaming pass -----------------------
     float T = 1.f;
     if (!greedy && P.temperature) T = P.temperature[b];
+    const float tp = (!greedy && P.top_p) ? P.top_p[b] : 1.f;  // nucleus threshold
     const float c = (T > 0.f && T != POS_INF) ? LOG2E / T : 1.f;
     for (int i = tid; i < k; i += NT) dtok[i] = P.draft_tokens[b * k + i];
     if (!greedy)
@@ -151,6 +153,7 @@ __global__ void __launch_bounds__(SEQ_NT, 3) sv_seq_kernel(const SeqParams P) {
             if (dtok[i] < 0 || dtok[i] >= V) bad = 1;
         if (!greedy) {
             if (!(T > 0.f) || T == POS_INF) bad = 1;
+            if (!(tp > 0.f && tp <= 1.f)) bad = 1;
             for (int i = 0; i <= k; ++i)
                 if (!(uu[i] >= 0.f && uu[i] < 1.f)) bad = 1;
         }
@@ -224,7 +227,7 @@ __global__ void __launch_bounds__(SEQ_NT, 3) sv_seq_kernel(const SeqParams P) {
     // Warp 0 alone finishes the sequence: lane r holds row r's statistics, the
     // decisions come from shuffles and a ballot, and the draw reads the kept
     // lists already in shared memory.  Same arithmetic as the block path below.
-    if (P.pre && nrows <= 32) {
+    if (P.pre && nrows <= 32 && tp >= 1.f) {
         const bool clean = tid >= nrows || (prec[tid].flags == 0 && prec[tid].m == prec[tid].m &&
                                             prec[tid].m != POS_INF && prec[tid].m != NEG_INF);
         if (__syncthreads_and(clean) && !S.err) {
@@ -468,6 +471,44 @@ __global__ void __launch_bounds__(SEQ_NT, 3) sv_seq_kernel(const SeqParams P) {
                     st.invS = 1.f / acc;
                     st.zd = zd;  // -inf: the draft token is not kept (probability 0)
                 }
+                if (tp < 1.f && !st.err) {
+                    if (st.slow) {
+                        st.err = 1;  // the nucleus needs the kept list of the row
+                    } else {
+                        // Nucleus over the kept set: the cut is the largest kept value
+                        // x whose tail mass (probabilities of the values >= x) reaches
+                        // top_p; every value >= x is kept and renormalised.
+                        const Cand* L = buf;
+                        int n = ng;
+                        if (P.pre) {
+                            L = plist + static_cast<size_t>(rr) * P.kcap;
+                            n = prec[rr].n;
+                        } else if (P.nch == 1) {
+                            n = min(gather(r, st.tau, buf, P.mg), P.mg);
+                            __syncwarp();
+                        }
+                        float cand = NEG_INF;
+                        for (int e = lane; e < n; e += 32) {
+                            const float x = L[e].v;
+                            if (!(x >= st.tau)) continue;
+                            float mass = 0.f;
+                            for (int f = 0; f < n; ++f) {
+                                const float y = L[f].v;
+                                if (y >= x && y >= st.tau) mass += ex2(fmaf(y, c, -st.msc)) * st.invS;
+                            }
+                            if (mass >= tp) cand = fmaxf(cand, x);
+                        }
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1) cand = fmaxf(cand, __shfl_xor_sync(0xffffffffu, cand, o));
+                        const float cut = fmaxf(cand, st.tau);
+                        float acc = 0.f;
+                        for (int e = lane; e < n; e += 32)
+                            if (L[e].v >= cut) acc += ex2(fmaf(L[e].v, c, -st.msc));
+                        acc = warp_sum(acc);
+                        st.tau = cut;
+                        st.invS = 1.f / acc;
+                    }
+                }
             }
         }
         tmo = __any_sync(0xffffffffu, tmo);
@@ -623,11 +664,13 @@ __global__ void __launch_bounds__(SEQ_NT, 3) sv_seq_kernel(const SeqParams P) {
             bool use_q = use_q0;
             for (int attempt = 0; attempt < 2; ++attempt) {
                 for (int e = tid; e < nt; e += NT) {
-                    const float pt = ex2(fmaf(lt[e].v, c, -tst.msc)) * tst.invS;
+                    // entries below a row's threshold (a nucleus cut) weigh nothing
+                    const float pt = lt[e].v >= tst.tau ? ex2(fmaf(lt[e].v, c, -tst.msc)) * tst.invS : 0.f;
                     float w = pt;
                     if (use_q) {
                         const int pd = find(lt[e].i);
-                        const float q = pd >= 0 ? ex2(fmaf(ld[pd].v, c, -dst.msc)) * dst.invS : 0.f;
+                        const float q = (pd >= 0 && ld[pd].v >= dst.tau) ? ex2(fmaf(ld[pd].v, c, -dst.msc)) * dst.invS
+                                                                          : 0.f;
                         w = fmaxf(pt - q, 0.f);
                     }
                     wv[e] = w;

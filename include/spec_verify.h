@@ -101,6 +101,15 @@ typedef struct sv_options {
     uint64_t wait_timeout_ns;  /* bound of every device-side wait: 0 = 1e9 ns */
     uint32_t test_extra_tx;    /* test hook: bytes added to each bulk-copy wait so that
                                   the bounded wait runs out (0 in normal use) */
+    const float* top_p;        /* [B] fp32 or NULL: nucleus threshold per sequence, applied
+                                  to p and q alike after top-k and temperature: the most
+                                  probable kept tokens whose probabilities first sum to
+                                  >= top_p are kept, every token as probable as the last one
+                                  included, then renormalised (1 keeps all).  Values outside
+                                  (0, 1] make the sequence a row error.  Needs the top-k
+                                  kept-list path (0 < top_k < V, topk_path 0 or 1), else the
+                                  call returns SV_ERR_UNSUPPORTED; a row whose kept list
+                                  overflowed (massive ties at tau) becomes a row error. */
 } sv_options_t;
 
 /*

@@ -57,11 +57,11 @@ def test_options_struct_layout_matches_c(tmp_path):
 #include <stdio.h>
 #include "spec_verify.h"
 int main(void) {
-  printf("%zu %zu %zu %zu %zu %zu %zu %zu\n", sizeof(sv_options_t),
+  printf("%zu %zu %zu %zu %zu %zu %zu %zu %zu\n", sizeof(sv_options_t),
          offsetof(sv_options_t, chunks_per_row), offsetof(sv_options_t, threads),
          offsetof(sv_options_t, topk_path), offsetof(sv_options_t, event_start),
          offsetof(sv_options_t, event_stop), offsetof(sv_options_t, wait_timeout_ns),
-         offsetof(sv_options_t, test_extra_tx));
+         offsetof(sv_options_t, test_extra_tx), offsetof(sv_options_t, top_p));
   return 0;
 }
 """)
