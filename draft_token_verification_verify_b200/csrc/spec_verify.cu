@@ -532,6 +532,7 @@ sv_status_t sample_args(const void* logits, const float* uniforms, int rows, int
     if (rows <= 0 || V < 1 || top_k < 0) return SV_ERR_INVALID_ARG;
     if (!decode_mode(mode, &greedy, &dt)) return SV_ERR_INVALID_ARG;
     if (check_options(opts) != SV_OK) return SV_ERR_INVALID_ARG;
+    if (opts && opts->top_p) return SV_ERR_UNSUPPORTED;  // the nucleus is offered for verification only
     const int elt = dt ? 4 : 2;
     if (static_cast<unsigned long long>(rows) > (1ULL << 62) / (static_cast<unsigned long long>(V) * 4ULL))
         return SV_ERR_INVALID_ARG;

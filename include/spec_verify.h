@@ -109,7 +109,9 @@ typedef struct sv_options {
                                   (0, 1] make the sequence a row error.  Needs the top-k
                                   kept-list path (0 < top_k < V, topk_path 0 or 1), else the
                                   call returns SV_ERR_UNSUPPORTED; a row whose kept list
-                                  overflowed (massive ties at tau) becomes a row error. */
+                                  overflowed (massive ties at tau) becomes a row error.
+                                  Verification only: spec_sample_ex returns
+                                  SV_ERR_UNSUPPORTED when it is set. */
 } sv_options_t;
 
 /*

@@ -121,6 +121,20 @@ def test_invalid_options_rejected(L, field, val):
     assert sv.spec_verify_workspace_size(2, 3, 100, 0, 0, o) == 0
 
 
+def test_misaligned_top_p_rejected(L):
+    o = sv.make_options()
+    o.top_p = 0x1002  # not 4-byte aligned
+    st = sv.spec_verify_ex(P, P, P, P, 2, 3, 100, None, 50, 0, P, P, None, None, None, None, 0, o, 0)
+    assert st == sv.SV_ERR_INVALID_ARG
+
+
+def test_sampler_refuses_top_p(L):
+    o = sv.make_options()
+    o.top_p = 0x1000
+    st = sv.spec_sample_ex(P, P, 4, 50, None, 5, 0, P, None, 0, o, 0)
+    assert st == sv.SV_ERR_UNSUPPORTED
+
+
 @pytest.mark.parametrize("kw", [dict(B=0), dict(k=0), dict(V=0), dict(top_k=-1), dict(mode=7)])
 def test_workspace_size_invalid_arguments(L, kw):
     a = dict(B=2, k=3, V=100, top_k=0, mode=0)
