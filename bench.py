@@ -309,27 +309,49 @@ def run_reference(args):
         return 0
     name = args.workload
     k = workloads.WORKLOADS[name].k
-    run = OracleRunner(name, host_cores())
     try:
+        run = OracleRunner(name, host_cores())
+        try:
+            for _ in range(args.warmup):
+                run.step()
+            t0 = time.perf_counter()
+            for _ in range(args.steps):
+                run.step()
+            dt = time.perf_counter() - t0
+        finally:
+            run.close()
+        per_step, cores = run.sequences_per_step(), run.workers
+        sample = (f"{per_step} sequence(s) of the {name} workload shape per step, one per core on "
+                  f"{cores} processes")
+    except Exception as exc:  # the multi-process run failed: the same steps on one thread
+        import oracle
+
+        case = workloads.make_case(name, seed=7000, B=1)
+        drafts = oracle.draft_tokens_for(case)
+        greedy = case.mode == "greedy"
+        per_step, cores = ORACLE_REPS[name], 1
+
+        def one_step():
+            for _ in range(per_step):
+                oracle.verify(case.target, None if greedy else case.draft, drafts,
+                              None if greedy else case.uniforms, case.temperature, case.top_k, greedy)
+
         for _ in range(args.warmup):
-            run.step()
+            one_step()
         t0 = time.perf_counter()
         for _ in range(args.steps):
-            run.step()
+            one_step()
         dt = time.perf_counter() - t0
-    finally:
-        run.close()
-    per_step = run.sequences_per_step()
+        sample = (f"{per_step} sequence(s) of the {name} workload shape per step, single thread "
+                  f"(multi-process run failed: {type(exc).__name__})")
     value = args.steps * per_step * k / dt
-    sample = (f"{per_step} sequence(s) of the {name} workload shape per step, one per core on "
-              f"{run.workers} processes")
     line = {
         "impl": "reference", "metric": "verified draft positions/sec", "value": value,
         "unit": "positions/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1000 * dt / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": DESCR[name], "sample_per_step": f"{per_step} sequence(s)"},
-        "cpu_baseline": {"value": value, "unit": "positions/s", "cores": run.workers, "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": "positions/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "positions/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
