@@ -157,7 +157,9 @@ def test_argmax_lowest_index(row, expect):
 
 def test_greedy_verify_rule():
     target = np.array([[[1, 5, 5, 2], [0, 0, 9, 9], [-0.0, 0.0, -1, -2]]], np.float32)
-    cases = [([1, 2], 2, [1, 2, 0]), ([2, 2], 0, [1, -1, -1]), ([1, 3], 1, [1, 2, -1])]
+    # argmaxes 1, 2, 0; the first mismatch decides, a later one changes nothing
+    cases = [([1, 2], 2, [1, 2, 0]), ([2, 2], 0, [1, -1, -1]), ([1, 3], 1, [1, 2, -1]),
+             ([2, 3], 0, [1, -1, -1])]
     for d, n, toks in cases:
         r = oracle.verify(target, None, np.array([d]), None, greedy=True)
         assert r.n_accepted.tolist() == [n] and r.tokens[0].tolist() == toks
@@ -167,17 +169,20 @@ def test_greedy_verify_rule():
 # inverse CDF
 # --------------------------------------------------------------------------
 
-@pytest.mark.parametrize("w,u,expect", [
-    ([0, 1, 0, 3], 0.0, 1),            # zero-weight entries are never drawn
-    ([0, 1, 0, 3], 0.2499, 1),
-    ([0, 1, 0, 3], 0.25, 3),           # C_v > u*W is strict
-    ([0, 1, 0, 3], 0.999, 3),
-    ([1, 2, 0], 1.0 - 2 ** -53, 1),    # u just below 1: the last positive entry
-    ([5], 0.5, 0),
+@pytest.mark.parametrize("w,u,expect,lo_hi", [
+    ([0, 1, 0, 3], 0.0, 1, (0.0, 0.25)),           # zero-weight entries are never drawn
+    ([0, 1, 0, 3], 0.2499, 1, (0.0, 0.25)),
+    ([0, 1, 0, 3], 0.25, 3, (0.25, 1.0)),          # C_v > u*W is strict
+    ([0, 1, 0, 3], 0.999, 3, (0.25, 1.0)),
+    ([1, 2, 0], 1.0 - 2 ** -53, 1, (1 / 3, 1.0)),  # u just below 1: the last positive entry
+    ([5], 0.5, 0, (0.0, 1.0)),
+    ([2, 1, 1], 0.6, 1, (0.5, 0.75)),
 ])
-def test_inverse_cdf_hand_cases(w, u, expect):
+def test_inverse_cdf_hand_cases(w, u, expect, lo_hi):
+    """Token and the CDF points C_{y-1}/W, C_y/W around it (reading R3)."""
     tok, lo, hi = oracle.inverse_cdf(np.array(w, np.float64), u)
-    assert tok == expect and lo <= hi
+    assert tok == expect
+    assert lo == pytest.approx(lo_hi[0], abs=1e-15) and hi == pytest.approx(lo_hi[1], abs=1e-15)
 
 
 def test_inverse_cdf_zero_mass():
@@ -344,6 +349,16 @@ def test_chi_square_emitted_law():
     a = reached[1] / n_total
     alpha = np.minimum(p[0], q0).sum()
     assert abs(a - alpha) < 5 * math.sqrt(alpha * (1 - alpha) / n_total)
+
+
+@pytest.mark.parametrize("u,expect", [(0.0, 0), (0.1, 0), (0.25, 1), (0.3, 1), (0.5, 2), (0.9, 3)])
+def test_sampler_token_for_each_uniform(u, expect):
+    """Four equal logits give 1/4 each, so the draw is the smallest v with
+    (v + 1)/4 > u (reading R3): the map from u to the token is fixed, not only
+    its law."""
+    row = np.zeros((1, 4), np.float32)
+    tok, lo, hi = oracle.sample_rows(row, np.array([u], np.float32), np.ones(1, np.float32))
+    assert tok[0] == expect and lo[0] == expect / 4 and hi[0] == (expect + 1) / 4
 
 
 def test_sampler_law_by_midpoint_grid():

@@ -176,6 +176,66 @@ def test_verify_without_processors_equals_plain_verify():
         assert np.array_equal(getattr(a, f), getattr(b, f), equal_nan=True), f
 
 
+def test_verify_rejects_a_draft_token_the_target_nucleus_drops():
+    """Reading R1 (accept iff u*q < p) with the nucleus in effect: the target
+    keeps only token 0 (p(1) = 0), the draft only token 1 (q(1) = 1), so even
+    u = 0 rejects token 1, and the residual max(0, p - q) is all on token 0."""
+    target = f32([[[5, 0, 0], [0, 0, 0]]])
+    draft = f32([[[0, 5, 0]]])
+    r = oracle.verify_procs(target, draft, np.array([[1]]), f32([[0.0, 0.5]]), top_p=0.5)
+    assert r.p[0, 0] == 0.0 and r.q[0, 0] == 1.0
+    assert r.n_accepted[0] == 0 and r.tokens[0].tolist() == [0, -1]
+
+
+@pytest.mark.parametrize("where", ["accept", "final", "negative"])
+def test_verify_procs_uniform_out_of_range_is_a_row_error(where):
+    """Reading R7: a uniform outside [0, 1) makes its sequence a row error; the
+    other sequence is unaffected."""
+    V, k = 5, 2
+    target = np.zeros((2, k + 1, V), np.float32)
+    draft = np.zeros((2, k, V), np.float32)
+    u = np.full((2, k + 1), 0.5, np.float32)
+    u[0, {"accept": 0, "final": k, "negative": 1}[where]] = -0.1 if where == "negative" else 1.0
+    r = oracle.verify_procs(target, draft, np.ones((2, k), np.int32), u, top_p=0.9)
+    assert r.n_accepted[0] == -1 and np.all(r.tokens[0] == -1)
+    assert r.n_accepted[1] == k and r.errors == 1
+
+
+def test_each_sequence_uses_its_own_processors():
+    """Sequences are verified independently: a batch with different top_p,
+    penalties and masks per sequence gives, for every sequence, what that
+    sequence gives alone."""
+    rng = np.random.default_rng(21)
+    B, k, V = 5, 3, 70
+    target = f32(rng.normal(0, 2, (B, k + 1, V)))
+    draft = f32(target[:, :k] + rng.normal(0, 1, (B, k, V)))
+    temp = f32(rng.uniform(0.6, 1.4, B))
+    u = f32(rng.uniform(0, 1, (B, k + 1)))
+    top_p = f32(rng.uniform(0.5, 0.95, B))
+    pen = f32(rng.uniform(0.5, 2.0, B))
+    ids = rng.integers(0, V, (B, 6)).astype(np.int32)
+    mask = np.stack([oracle.allow_mask(V, rng.choice(V, 40, replace=False)) for _ in range(B)])
+    drafts = np.stack([oracle.sample_rows_procs(draft[b:b + 1], u[b:b + 1, :k], np.full(k, temp[b]), 0,
+                                                top_p=top_p[b:b + 1], rep_penalty=pen[b:b + 1],
+                                                rep_ids=ids[b:b + 1], mask=mask[b:b + 1])[0]
+                       for b in range(B)]).astype(np.int32)
+    both = oracle.verify_procs(target, draft, drafts, u, temp, 0, top_p=top_p, rep_penalty=pen,
+                               rep_ids=ids, mask=mask)
+    assert both.errors == 0
+
+    def alone(b, s):
+        return oracle.verify_procs(target[b:b + 1], draft[b:b + 1], drafts[b:b + 1], u[b:b + 1],
+                                   temp[b:b + 1], 0, top_p=top_p[s:s + 1], rep_penalty=pen[s:s + 1],
+                                   rep_ids=ids[s:s + 1], mask=mask[s:s + 1])
+
+    for b in range(B):
+        one = alone(b, b)
+        for f in ("tokens", "n_accepted", "p", "q", "cdf_lo", "cdf_hi"):
+            assert np.array_equal(getattr(both, f)[b], getattr(one, f)[0], equal_nan=True), (b, f)
+    # the processors differ enough between sequences to change the results
+    assert any(not np.array_equal(alone(b, 0).p, alone(b, b).p, equal_nan=True) for b in range(1, B))
+
+
 def _pieces(points):
     pts = sorted(set([0.0, 1.0] + [float(x) for x in points if 0.0 < x < 1.0]))
     return [(a, b) for a, b in zip(pts[:-1], pts[1:]) if b - a > 1e-6]
