@@ -39,6 +39,7 @@ DeviceInfo g_dev[kMaxDevices];
 std::once_flag g_dev_once[kMaxDevices];
 std::once_flag g_pool_once[kMaxDevices];
 std::once_flag g_attr_once[kMaxDevices][26];
+cudaError_t g_attr_err[kMaxDevices][26];  // result of each one-time attribute call
 std::once_flag g_occ_once[kMaxDevices][24];
 int g_occ[kMaxDevices][24];
 
@@ -52,8 +53,9 @@ const DeviceInfo* device_info(int* dev_out) {
     }
     std::call_once(g_dev_once[dev], [dev] {
         DeviceInfo& d = g_dev[dev];
-        int major = 0;
+        int major = 0, minor = 0;
         if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&d.smem_per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) !=
@@ -62,7 +64,8 @@ const DeviceInfo* device_info(int* dev_out) {
             d.ok = 0;
             return;
         }
-        d.ok = major == 10 ? 1 : 0;  // the kernels are built for sm_100a only
+        // sm_100a code runs on compute capability 10.0 only (not on other 10.x parts)
+        d.ok = (major == 10 && minor == 0) ? 1 : 0;
         d.id = dev;
     });
     *dev_out = dev;
@@ -243,18 +246,18 @@ sv_status_t set_attrs(int dev, int dt, int nt, int mode) {
     int slot = 0;
     RowsFn f1 = pick_rows(dt, nt, mode, &slot);
     SeqFn f2 = dt ? sv::sv_seq_kernel<1> : sv::sv_seq_kernel<0>;
-    cudaError_t e = cudaSuccess;
     std::call_once(g_attr_once[dev][slot], [&] {
-        e = cudaFuncSetAttribute(f1, cudaFuncAttributeMaxDynamicSharedMemorySize, g_dev[dev].smem_optin);
+        g_attr_err[dev][slot] =
+            cudaFuncSetAttribute(f1, cudaFuncAttributeMaxDynamicSharedMemorySize, g_dev[dev].smem_optin);
+        if (g_attr_err[dev][slot] != cudaSuccess) cudaGetLastError();
     });
     std::call_once(g_attr_once[dev][24 + dt], [&] {
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(f2, cudaFuncAttributeMaxDynamicSharedMemorySize, g_dev[dev].smem_optin);
+        g_attr_err[dev][24 + dt] =
+            cudaFuncSetAttribute(f2, cudaFuncAttributeMaxDynamicSharedMemorySize, g_dev[dev].smem_optin);
+        if (g_attr_err[dev][24 + dt] != cudaSuccess) cudaGetLastError();
     });
-    if (e != cudaSuccess) {
-        cudaGetLastError();
-        return SV_ERR_CUDA;
-    }
+    // a failed attribute call fails every later call for that kernel too
+    if (g_attr_err[dev][slot] != cudaSuccess || g_attr_err[dev][24 + dt] != cudaSuccess) return SV_ERR_CUDA;
     return SV_OK;
 }
 
