@@ -204,6 +204,28 @@ def _dtype_code(t) -> int:
     raise TypeError(f"logits must be bfloat16 or float32, got {t.dtype}")
 
 
+def _check(t, name, dtypes, numel, device):
+    """Raise unless tensor ``t`` has the layout the C ABI reads: one of
+    ``dtypes``, ``numel`` elements, contiguous, on ``device``."""
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if not hasattr(t, "data_ptr"):
+        raise TypeError(f"{name} must be a torch tensor (use the spec_* functions for raw pointers)")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name} must be {' or '.join(str(d) for d in dtypes)}, got {t.dtype}")
+    if t.numel() != numel:
+        raise ValueError(f"{name} must have {numel} elements, got {t.numel()} (shape {tuple(t.shape)})")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, the logits on {device}")
+
+
+def _check_cuda(device):
+    if device.type != "cuda":
+        raise ValueError(f"tensors must be on a CUDA device, got {device}")
+
+
 def verify(target, draft, draft_tokens, uniforms=None, temperature=None, top_k: int = 0,
            greedy: bool = False, out_tokens=None, out_n_accepted=None, out_p=None, out_q=None,
            out_status=None, workspace=None, opts: Optional[SvOptions] = None, stream=None):
@@ -213,18 +235,42 @@ def verify(target, draft, draft_tokens, uniforms=None, temperature=None, top_k: 
     GPU), draft_tokens [B, k] int32, uniforms [B, k+1] fp32, temperature [B]
     fp32 or None.  Output tensors are allocated with torch when not given; the
     workspace (a uint8 tensor) is taken from the library pool when None.
-    Returns (out_tokens [B, k+1], out_n_accepted [B]).
+    Every tensor is checked for dtype, element count, contiguity and device
+    before the call (TypeError / ValueError); greedy mode ignores draft,
+    uniforms and temperature.  Returns (out_tokens [B, k+1], out_n_accepted [B]).
     """
     import torch
 
+    if target.dim() != 3:
+        raise ValueError(f"target must be [B, k+1, V], got shape {tuple(target.shape)}")
     B, k1, V = target.shape
     k = k1 - 1
     dev = target.device
+    f32, i32 = (torch.float32,), (torch.int32,)
+    mode = (SV_MODE_GREEDY if greedy else SV_MODE_STOCHASTIC) | _dtype_code(target)
+    _check(target, "target", (target.dtype,), B * k1 * V, dev)
+    _check(draft_tokens, "draft_tokens", i32, B * k, dev)
+    if not greedy:  # greedy reads neither the draft logits, the uniforms nor the temperature
+        _check(draft, "draft", (target.dtype,), B * k * V, dev)
+        _check(uniforms, "uniforms", f32, B * k1, dev)
+        if temperature is not None:
+            _check(temperature, "temperature", f32, B, dev)
+        for t, name in ((out_p, "out_p"), (out_q, "out_q")):
+            if t is not None:
+                _check(t, name, f32, B * k, dev)
+    if out_tokens is not None:
+        _check(out_tokens, "out_tokens", i32, B * k1, dev)
+    if out_n_accepted is not None:
+        _check(out_n_accepted, "out_n_accepted", i32, B, dev)
+    if out_status is not None:
+        _check(out_status, "out_status", i32, 1, dev)
+    if workspace is not None:
+        _check(workspace, "workspace", (workspace.dtype,), workspace.numel(), dev)
+    _check_cuda(dev)
     if out_tokens is None:
         out_tokens = torch.empty((B, k + 1), dtype=torch.int32, device=dev)
     if out_n_accepted is None:
         out_n_accepted = torch.empty((B,), dtype=torch.int32, device=dev)
-    mode = (SV_MODE_GREEDY if greedy else SV_MODE_STOCHASTIC) | _dtype_code(target)
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = spec_verify_ex(target, draft, draft_tokens, uniforms, B, k, V, temperature, top_k, mode,
                         out_tokens, out_n_accepted, out_p, out_q, out_status, workspace, wbytes, opts,
@@ -236,14 +282,25 @@ def verify(target, draft, draft_tokens, uniforms=None, temperature=None, top_k: 
 
 def sample(logits, uniforms=None, temperature=None, top_k: int = 0, greedy: bool = False,
            out_tokens=None, opts: Optional[SvOptions] = None, stream=None):
-    """Tensor convenience wrapper around ``spec_sample_ex``: logits [..., V]."""
+    """Tensor convenience wrapper around ``spec_sample_ex``: logits [..., V]
+    (bf16 or fp32), uniforms and temperature fp32 with one entry per row,
+    checked like the arguments of ``verify``."""
     import torch
 
     V = logits.shape[-1]
     rows = logits.numel() // V
-    if out_tokens is None:
-        out_tokens = torch.empty(logits.shape[:-1], dtype=torch.int32, device=logits.device)
+    dev = logits.device
     mode = (SV_MODE_GREEDY if greedy else SV_MODE_STOCHASTIC) | _dtype_code(logits)
+    _check(logits, "logits", (logits.dtype,), rows * V, dev)
+    if not greedy:
+        _check(uniforms, "uniforms", (torch.float32,), rows, dev)
+        if temperature is not None:
+            _check(temperature, "temperature", (torch.float32,), rows, dev)
+    if out_tokens is not None:
+        _check(out_tokens, "out_tokens", (torch.int32,), rows, dev)
+    _check_cuda(dev)
+    if out_tokens is None:
+        out_tokens = torch.empty(logits.shape[:-1], dtype=torch.int32, device=dev)
     st = spec_sample_ex(logits, uniforms, rows, V, temperature, top_k, mode, out_tokens, None, 0, opts,
                         stream)
     if st != SV_OK:

@@ -168,3 +168,96 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     with pytest.raises(ImportError):
         sv.lib()
     importlib.reload(sv)
+
+
+# --------------------------------------------------------------------------
+# tensor wrappers: layout checks before the call (CPU tensors, no GPU needed)
+# --------------------------------------------------------------------------
+
+def _verify_args(B=3, k=2, V=17):
+    import torch
+
+    return dict(target=torch.zeros(B, k + 1, V, dtype=torch.bfloat16),
+                draft=torch.zeros(B, k, V, dtype=torch.bfloat16),
+                draft_tokens=torch.zeros(B, k, dtype=torch.int32),
+                uniforms=torch.zeros(B, k + 1, dtype=torch.float32),
+                temperature=torch.ones(B, dtype=torch.float32))
+
+
+def _bad_verify_cases():
+    import torch
+
+    def t(**kw):
+        a = _verify_args()
+        a.update(kw)
+        return a
+
+    return [
+        (t(draft_tokens=torch.zeros(3, 2, dtype=torch.int64)), TypeError, "draft_tokens"),
+        (t(uniforms=torch.zeros(3, 3, dtype=torch.float64)), TypeError, "uniforms"),
+        (t(draft=torch.zeros(3, 2, 17, dtype=torch.float32)), TypeError, "draft"),
+        (t(target=torch.zeros(3, 3, 17, dtype=torch.float16)), TypeError, "bfloat16 or float32"),
+        (t(draft_tokens=torch.zeros(3, 3, dtype=torch.int32)), ValueError, "draft_tokens"),
+        (t(temperature=torch.ones(4, dtype=torch.float32)), ValueError, "temperature"),
+        (t(uniforms=torch.zeros(3, 3, dtype=torch.float32).t()), ValueError, "contiguous"),
+        (t(draft=torch.zeros(3, 17, 2, dtype=torch.bfloat16).transpose(1, 2)), ValueError, "contiguous"),
+        (t(uniforms=None), ValueError, "uniforms is required"),
+        (t(target=torch.zeros(3, 17, dtype=torch.bfloat16)), ValueError, "target must be"),
+        (t(draft_tokens=[[0, 0]] * 3), TypeError, "torch tensor"),
+        (t(), ValueError, "CUDA device"),
+    ]
+
+
+@pytest.mark.parametrize("i", range(12))
+def test_verify_wrapper_checks_layout(i):
+    import draft_token_verification_verify_b200 as sv
+
+    args, exc, msg = _bad_verify_cases()[i]
+    with pytest.raises(exc, match=msg):
+        sv.verify(args["target"], args["draft"], args["draft_tokens"], args["uniforms"], args["temperature"], 5)
+
+
+def test_verify_wrapper_greedy_ignores_stochastic_inputs():
+    import torch
+
+    import draft_token_verification_verify_b200 as sv
+
+    a = _verify_args()
+    # draft, uniforms and temperature of the wrong kind are not read in greedy mode
+    with pytest.raises(ValueError, match="CUDA device"):
+        sv.verify(a["target"], None, a["draft_tokens"], torch.zeros(1, dtype=torch.float64), None, greedy=True)
+
+
+def test_verify_wrapper_checks_outputs():
+    import torch
+
+    import draft_token_verification_verify_b200 as sv
+
+    a = _verify_args()
+    with pytest.raises(ValueError, match="out_tokens"):
+        sv.verify(**a, out_tokens=torch.zeros(3, 2, dtype=torch.int32))
+    with pytest.raises(TypeError, match="out_p"):
+        sv.verify(**a, out_p=torch.zeros(3, 2, dtype=torch.float64))
+    with pytest.raises(ValueError, match="out_status"):
+        sv.verify(**a, out_status=torch.zeros(2, dtype=torch.int32))
+
+
+def test_sample_wrapper_checks_layout():
+    import torch
+
+    import draft_token_verification_verify_b200 as sv
+
+    logits = torch.zeros(4, 3, 11, dtype=torch.float32)
+    u = torch.zeros(4, 3, dtype=torch.float32)
+    with pytest.raises(TypeError, match="uniforms"):
+        sv.sample(logits, u.double())
+    with pytest.raises(ValueError, match="uniforms"):
+        sv.sample(logits, torch.zeros(4, dtype=torch.float32))
+    with pytest.raises(ValueError, match="temperature"):
+        sv.sample(logits, u, torch.ones(4, dtype=torch.float32))
+    with pytest.raises(ValueError, match="contiguous"):
+        sv.sample(torch.zeros(4, 11, 3).transpose(1, 2), u)
+    with pytest.raises(ValueError, match="CUDA device"):
+        sv.sample(logits, u, torch.ones(12, dtype=torch.float32))   # one temperature per row: valid
+    with pytest.raises(ValueError, match="CUDA device"):
+        sv.sample(logits, greedy=True)
