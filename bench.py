@@ -17,6 +17,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -33,6 +34,7 @@ import workloads  # noqa: E402
 
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
+SPEC_HBM_GBS = 8000.0  # B200 HBM3e data-sheet bandwidth, for the fraction of the spec figure
 PROFILE_DIR = os.path.join(ROOT, "profiles")
 KSAMPLE = 8  # timed steps per streaming-kernel event sample
 
@@ -160,6 +162,12 @@ class ClockSampler:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
                 "reasons": sorted(reasons)}
+
+
+def pctl(xs, q: float) -> float:
+    """Nearest-rank percentile ``q`` (0..100) of a non-empty sequence."""
+    s = sorted(xs)
+    return s[min(len(s) - 1, max(0, math.ceil(q / 100.0 * len(s)) - 1))]
 
 
 def launches_per_step(case) -> int:
@@ -553,6 +561,13 @@ def run_ours(args):
         except Exception as exc:  # the multi-process leg failed: one thread instead
             cpu = cpu_baseline_single(name, case, drafts.cpu().numpy(), args.cpu_budget,
                                       f"multi-process run failed: {type(exc).__name__}")
+        if cpu.get("cores", 1) > 1:  # the one-core figure beside the all-core one
+            try:
+                one = cpu_baseline_single(name, case, drafts.cpu().numpy(), args.cpu_budget / 3,
+                                          "one core, beside the all-core figure")
+                cpu["single_core"] = {"value": one["value"], "unit": one["unit"], "sample": one["sample"]}
+            except Exception as exc:
+                cpu["single_core"] = {"unavailable": f"{type(exc).__name__}: {exc}"[:200]}
 
     if world > 1:
         torch.distributed.barrier()
@@ -574,7 +589,10 @@ def run_ours(args):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
                      "kernel": "sv_rows_kernel", "kernel_ms_mean": kmean,
-                     "kernel_ms_median": statistics.median(kern_ms)},
+                     "kernel_ms_median": statistics.median(kern_ms),
+                     "kernel_ms_p10": pctl(kern_ms, 10), "kernel_ms_p90": pctl(kern_ms, 90),
+                     "kernel_samples": len(kern_ms),
+                     "frac_of_spec": achieved / SPEC_HBM_GBS, "spec_gbs": SPEC_HBM_GBS},
         "gpu_launches": launches_per_step(case) * args.steps,
         "clocks": clocks,
         "e2e": e2e,

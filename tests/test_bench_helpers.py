@@ -47,3 +47,19 @@ def test_oracle_runner_two_processes():
         run.close()
     assert run.sequences_per_step() == 2 * bench.ORACLE_REPS["tiny"]
     assert all(not p.is_alive() for p in run.procs)
+
+
+def test_nearest_rank_percentiles():
+    xs = [5.0, 1.0, 3.0, 2.0, 4.0]
+    assert bench.pctl(xs, 10) == 1.0 and bench.pctl(xs, 50) == 3.0 and bench.pctl(xs, 90) == 5.0
+    assert bench.pctl([7.0], 10) == 7.0 == bench.pctl([7.0], 90)
+
+
+def test_single_core_oracle_leg():
+    import oracle
+
+    case = workloads.make_case("tiny", seed=3, B=6)
+    drafts = oracle.draft_tokens_for(case)
+    out = bench.cpu_baseline_single("tiny", case, drafts, 0.5, "test")
+    assert out["cores"] == 1 and out["kind"] == "oracle" and out["value"] > 0
+    assert "single thread" in out["sample"]
