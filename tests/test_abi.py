@@ -83,6 +83,37 @@ def test_header_compiles_as_c_and_cpp(tmp_path):
                         "-o", str(tmp_path / "h.o"), str(src)], check=True)
 
 
+def test_c_program_links_and_calls_the_library(tmp_path, L):
+    """A plain C consumer: compiled with gcc against the header, linked against the
+    in-tree library, calling only what is safe on any machine (version, status
+    strings, calls rejected before any CUDA work)."""
+    src = tmp_path / "consumer.c"
+    src.write_text(r"""
+#include <stdio.h>
+#include "spec_verify.h"
+int main(void) {
+    sv_options_t o = {0};
+    sv_status_t bad_b = spec_verify(NULL, NULL, NULL, NULL, 0, 1, 10, NULL, 0,
+                                    SV_MODE_STOCHASTIC | SV_DTYPE_BF16, NULL, NULL, NULL);
+    sv_status_t bad_mode = spec_verify_ex(NULL, NULL, NULL, NULL, 1, 1, 10, NULL, 0, 7, NULL, NULL,
+                                          NULL, NULL, NULL, NULL, 0, &o, NULL);
+    size_t ws = spec_verify_workspace_size(0, 1, 10, 0, 0, NULL);
+    sv_status_t bad_rows = spec_sample(NULL, NULL, 0, 10, NULL, 0, SV_MODE_GREEDY, NULL, NULL);
+    printf("%d %d %d %zu %d %s\n", spec_verify_version(), (int)bad_b, (int)bad_mode, ws, (int)bad_rows,
+           spec_verify_status_string(SV_ERR_UNSUPPORTED));
+    return 0;
+}
+""")
+    libdir = os.path.dirname(sv.LIB_PATH)
+    exe = tmp_path / "consumer"
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(src),
+                    "-L", libdir, "-lspec_verify", f"-Wl,-rpath,{libdir}", "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split(maxsplit=5)
+    assert int(out[0]) == sv.spec_verify_version()
+    assert [int(x) for x in out[1:5]] == [sv.SV_ERR_INVALID_ARG, sv.SV_ERR_INVALID_ARG, 0, sv.SV_ERR_INVALID_ARG]
+    assert out[5].strip() == sv.spec_verify_status_string(sv.SV_ERR_UNSUPPORTED)
+
+
 # fake but aligned device pointers: argument checks run before any CUDA call
 P = 0x7f0000000000
 
