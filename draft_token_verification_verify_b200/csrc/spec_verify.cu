@@ -573,7 +573,7 @@ size_t workspace_for(const Call& cl, const sv_options_t* opts) {
 
 // One fixed buffer per device, part of the library's device image: calls that
 // must not allocate take their scratch from here.
-std::once_flag g_static_once[kMaxDevices];
+std::mutex g_static_mu[kMaxDevices];
 void* g_static_ptr[kMaxDevices];
 
 }  // namespace
@@ -583,16 +583,19 @@ static __device__ __align__(256) unsigned char g_sv_static_scratch[SV_STATIC_WOR
 namespace {
 
 // Device address of the static buffer on `dev`, which must be the current
-// device; looked up once per device.  NULL if the lookup failed.
+// device.  Only a successful lookup is cached, so a lookup that failed (for
+// example one made during a stream capture) is tried again by the next call.
+// NULL if the lookup failed.
 void* static_scratch(int dev) {
-    std::call_once(g_static_once[dev], [dev] {
+    std::lock_guard<std::mutex> lock(g_static_mu[dev]);
+    if (!g_static_ptr[dev]) {
         void* ptr = nullptr;
         if (cudaGetSymbolAddress(&ptr, g_sv_static_scratch) != cudaSuccess) {
             cudaGetLastError();
-            ptr = nullptr;
+            return nullptr;
         }
         g_static_ptr[dev] = ptr;
-    });
+    }
     return g_static_ptr[dev];
 }
 

@@ -182,8 +182,9 @@ SV_API sv_status_t spec_verify_ex(const void* target_logits, const void* draft_l
  * Arguments and outputs are those of spec_verify_ex without the workspace.
  *
  * Set-up: the first call on a device, with that device current, looks up the
- * buffer's device address once and caches it.  Make that first call before
- * any stream capture on that device.
+ * buffer's device address and caches it; a lookup that fails is not cached
+ * and the next call tries again.  Make that first call before any stream
+ * capture on that device.
  *
  * Limit: a problem whose scratch need (spec_verify_workspace_size with the
  * same arguments and options) exceeds SV_STATIC_WORKSPACE_BYTES is rejected

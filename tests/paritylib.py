@@ -176,3 +176,74 @@ def nucleus_near_cut(probs: np.ndarray, top_p: float, tol: float = DECISION_TOL)
     i = int(np.argmax(run >= top_p))
     before = run[i - 1] if i > 0 else 0.0
     return abs(run[i] - top_p) < tol or abs(before - top_p) < tol
+
+
+def flag_probability(w: np.ndarray, tol: float = DECISION_TOL) -> float:
+    """Probability, for u uniform on [0, 1), that an inverse-CDF draw from the
+    weights ``w`` is flagged as near-threshold: u lies within ``tol`` of one of
+    the two CDF points that bracket the drawn token.  Token v owns the interval
+    [C_{v-1}/W, C_v/W) of length w_v/W; the flagged part of it is its first and
+    its last ``tol`` (all of it when shorter than 2*tol)."""
+    w = np.asarray(w, dtype=np.float64)
+    W = w.sum()
+    if not W > 0:
+        return 0.0
+    return float(np.minimum(w[w > 0] / W, 2.0 * tol).sum())
+
+
+def flag_bound(expected: float) -> float:
+    """Largest flagged count accepted when ``expected`` flags are due: a sum of
+    independent Bernoulli trials has variance at most its mean, so five
+    standard deviations plus a small constant."""
+    return expected + 5.0 * np.sqrt(expected) + 3.0
+
+
+@dataclasses.dataclass
+class SampleReport:
+    rows: int
+    exact: int
+    flagged: int
+    expected_flagged: float
+    errors: int
+
+
+def compare_samples(logits, u, temperature, top_k, got, ref, lo, hi, greedy=False) -> SampleReport:
+    """GPU proposer draws vs the oracle's, one token per row of ``logits``.
+
+    Greedy: bit-exact.  Stochastic: bit-exact, except rows whose uniform lies
+    within DECISION_TOL of one of the two CDF points bracketing the oracle's
+    token.  Those rows are counted, and the GPU token must have positive
+    weight and a CDF interval (under the oracle's fp64 distribution) within
+    DECISION_TOL of u.  The flagged count must stay within ``flag_bound`` of
+    the count the rule predicts from the oracle's distributions."""
+    rows = got.shape[0]
+    exact = flagged = errors = 0
+    expected = 0.0
+    for r in range(rows):
+        if ref[r] < 0:
+            assert got[r] == -1, (r, got[r])
+            errors += 1
+            continue
+        if greedy:
+            assert got[r] == ref[r], (r, got[r], ref[r])
+            exact += 1
+            continue
+        T = 1.0 if temperature is None else float(temperature[r])
+        w = oracle.process_row(logits[r], T, top_k)
+        expected += flag_probability(w)
+        ur = float(u[r])
+        if abs(ur - lo[r]) < DECISION_TOL or abs(ur - hi[r]) < DECISION_TOL:
+            y = int(got[r])
+            assert 0 <= y < w.size, (r, y)
+            C = np.cumsum(w)
+            W = C[-1]
+            ylo = (C[y - 1] if y > 0 else 0.0) / W
+            yhi = C[y] / W
+            assert w[y] > 0 and ylo - DECISION_TOL <= ur <= yhi + DECISION_TOL, (r, y, ylo, yhi, ur)
+            flagged += 1
+            continue
+        assert got[r] == ref[r], (r, got[r], ref[r], ur, lo[r], hi[r])
+        exact += 1
+    rep = SampleReport(rows, exact, flagged, expected, errors)
+    assert flagged <= flag_bound(expected), rep
+    return rep

@@ -8,7 +8,8 @@ import numpy as np
 import pytest
 
 import oracle
-from paritylib import DECISION_TOL, GpuResult, compare, nucleus_near_cut
+from paritylib import (DECISION_TOL, GpuResult, compare, compare_samples, flag_probability,
+                       nucleus_near_cut)
 
 
 def _case(seed=0, B=12, k=3, V=40, top_k=0):
@@ -171,3 +172,69 @@ def test_greedy_is_bit_exact():
 ])
 def test_nucleus_near_cut_hand_cases(probs, top_p, near):
     assert bool(nucleus_near_cut(np.array(probs), top_p)) == near
+
+
+# ---- the proposer-sampler comparison ------------------------------------------------
+
+def _sample_case(seed=3, rows=60, V=400, top_k=0):
+    rng = np.random.default_rng(seed)
+    logits = rng.normal(0, 2, (rows, V)).astype(np.float32)
+    temp = np.asarray([0.5, 1.0, 1.5], np.float32)[np.arange(rows) % 3]
+    u = rng.uniform(0, 1, rows).astype(np.float32)
+    ref, lo, hi = oracle.sample_rows(logits, u, temp, top_k)
+    return logits, u, temp, top_k, ref, lo, hi
+
+
+def test_flag_probability_matches_a_fine_grid():
+    """The flagged measure of [0, 1) under the rule, counted on a grid of u."""
+    w = np.array([0.5, 1e-6, 0.0, 3e-6, 0.25, 0.25 - 4e-6])
+    G = 2_000_000
+    u = (np.arange(G) + 0.5) / G
+    C = np.cumsum(w) / w.sum()
+    tok = np.searchsorted(C, u, side="right")
+    lo = np.where(tok > 0, C[np.maximum(tok - 1, 0)], 0.0)
+    hi = C[tok]
+    flagged = (np.abs(u - lo) < DECISION_TOL) | (np.abs(u - hi) < DECISION_TOL)
+    assert abs(flagged.mean() - flag_probability(w)) < 2.0 / G * 8
+
+
+def test_sampler_oracle_output_passes_and_counts():
+    logits, u, temp, top_k, ref, lo, hi = _sample_case()
+    rep = compare_samples(logits, u, temp, top_k, ref.copy(), ref, lo, hi)
+    assert rep.exact + rep.flagged == rep.rows
+
+
+def test_sampler_wrong_token_fails():
+    logits, u, temp, top_k, ref, lo, hi = _sample_case()
+    near = (np.abs(u - lo) < DECISION_TOL) | (np.abs(u - hi) < DECISION_TOL)
+    r = int(np.flatnonzero(~near)[0])
+    got = ref.copy()
+    got[r] = (got[r] + 1) % logits.shape[1]
+    with pytest.raises(AssertionError):
+        compare_samples(logits, u, temp, top_k, got, ref, lo, hi)
+
+
+def test_sampler_flagged_row_checks_the_window():
+    """A flagged row whose GPU token lies far from u in the CDF fails."""
+    logits, u, temp, top_k, ref, lo, hi = _sample_case(rows=3)
+    u = u.copy()
+    u[0] = np.float32(hi[0])  # on the CDF point above the oracle's token: flagged
+    ref2, lo2, hi2 = oracle.sample_rows(logits, u, temp, top_k)
+    got = ref2.copy()
+    w = oracle.process_row(logits[0], float(temp[0]), top_k)
+    C = np.cumsum(w) / w.sum()
+    far = int(np.argmax(np.abs(C - u[0]) > 0.1))
+    got[0] = far
+    with pytest.raises(AssertionError):
+        compare_samples(logits, u, temp, top_k, got, ref2, lo2, hi2)
+    got[0] = ref2[0]
+    assert compare_samples(logits, u, temp, top_k, got, ref2, lo2, hi2).flagged >= 1
+
+
+def test_sampler_flag_count_is_bounded():
+    """More flagged rows than the rule predicts fails: uniforms planted on CDF points."""
+    logits, u, temp, top_k, ref, lo, hi = _sample_case(rows=40)
+    u = hi.astype(np.float32)  # every row on a CDF point
+    ref2, lo2, hi2 = oracle.sample_rows(logits, u, temp, top_k)
+    with pytest.raises(AssertionError):
+        compare_samples(logits, u, temp, top_k, ref2.copy(), ref2, lo2, hi2)
