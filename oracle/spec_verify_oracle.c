@@ -318,7 +318,11 @@ int oracle_sample_rows(const void* logits, int dtype, int rows, int V, const flo
  *       then the nucleus on the resulting probabilities;
  *   R13 repetition penalty theta > 0 on the sequence's listed token ids (each
  *       id once, ids outside [0, V) ignored): z -> z / theta if z > 0, else
- *       z * theta;
+ *       z * theta, the result rounded to fp32 (the logit's quotient or product
+ *       of two fp32 values, correctly rounded: computing it in double and
+ *       rounding once gives exactly that, as 53 >= 2 * 24 + 2 bits).  The
+ *       penalised logit decides the top-k set, so both sides take that
+ *       decision on the same fp32 value;
  *   R14 vocabulary mask: token v is allowed iff bit (v % 32) of word v / 32 is
  *       set; a disallowed token gets the logit -inf (probability 0);
  *   R15 nucleus 0 < top_p <= 1: order the tokens of positive probability by
@@ -357,7 +361,8 @@ static double or_logit_procs(const void* row, int dtype, long v, const or_procs_
     if (pr->rep_ids && pr->rep_penalty != 1.0) {
         for (i = 0; i < pr->n_rep; ++i) {
             if (pr->rep_ids[i] == v) {
-                z = z > 0.0 ? z / pr->rep_penalty : z * pr->rep_penalty;
+                /* rounded to fp32, the precision the kernels rank and exponentiate in */
+                z = z > 0.0 ? (double)(float)(z / pr->rep_penalty) : (double)(float)(z * pr->rep_penalty);
                 break; /* each id once */
             }
         }

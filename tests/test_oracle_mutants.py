@@ -76,7 +76,10 @@ MUTANTS = [
     ("out_p_is_q", "if (out_p) out_p[(size_t)b * k + i] = p;", "if (out_p) out_p[(size_t)b * k + i] = q;", 0),
     ("f32_row_stride", "size_t elt = dtype == OR_DTYPE_BF16 ? 2 : 4;", "size_t elt = 2;", 0),
     # R13 repetition penalty
-    ("penalty_ignores_sign", "z = z > 0.0 ? z / pr->rep_penalty : z * pr->rep_penalty;", "z = z / pr->rep_penalty;", 0),
+    ("penalty_ignores_sign", "z = z > 0.0 ? (double)(float)(z / pr->rep_penalty) : (double)(float)(z * pr->rep_penalty);",
+     "z = (double)(float)(z / pr->rep_penalty);", 0),
+    ("penalty_not_rounded", "z = z > 0.0 ? (double)(float)(z / pr->rep_penalty) : (double)(float)(z * pr->rep_penalty);",
+     "z = z > 0.0 ? z / pr->rep_penalty : z * pr->rep_penalty;", 0),
     ("penalty_per_listing", "break; /* each id once */", "/* every listing */", 0),
     ("penalty_ids_of_first_sequence", "pr.rep_ids = rep_ids ? rep_ids + (size_t)b * n_rep : NULL;",
      "pr.rep_ids = rep_ids;", 0),

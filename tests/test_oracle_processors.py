@@ -42,7 +42,25 @@ def test_repetition_penalty_each_id_once_and_out_of_range_ignored():
     once = oracle.process_row_procs(z, rep_penalty=1.7, rep_ids=[2])
     many = oracle.process_row_procs(z, rep_penalty=1.7, rep_ids=[2, 2, 9, -1, 2])
     assert np.array_equal(once, many)
-    assert np.allclose(once, softmax([1.5, 0.25, -0.75 * 1.7, 3.0]), rtol=0, atol=1e-15)
+    penalised = float(np.float32(-0.75 * 1.7))  # the exact product, rounded once to fp32
+    assert np.allclose(once, softmax([1.5, 0.25, penalised, 3.0]), rtol=0, atol=1e-15)
+
+
+def test_repetition_penalty_rounds_to_fp32():
+    """The penalised logit is the correctly rounded fp32 quotient (product):
+    1.5 / 1.2f rounds up to exactly 1.25 in fp32 while its fp64 value lies just
+    below, so a competitor at 1.25 ties with the penalised token at top-1 and
+    both are kept; unrounded, top-1 would keep the competitor alone.  Likewise
+    -1.5 * 1.2f against its own fp32 rounding."""
+    theta = np.float32(1.2)
+    c = np.float32(1.5) / theta                      # numpy fp32 division is IEEE round-to-nearest
+    assert float(c) == 1.25 and 1.5 / float(theta) < 1.25  # the rounding matters for this pair
+    z = f32([1.5, c, -3.0])
+    got = oracle.process_row_procs(z, top_k=1, rep_penalty=float(theta), rep_ids=[0])
+    assert np.allclose(got, [0.5, 0.5, 0.0], rtol=0, atol=1e-15)
+    neg = oracle.process_row_procs(f32([-1.5, np.float32(-1.5) * theta, -9.0]), top_k=1,
+                                   rep_penalty=float(theta), rep_ids=[0])
+    assert np.allclose(neg, [0.5, 0.5, 0.0], rtol=0, atol=1e-15)
 
 
 def test_unit_penalty_and_no_processor_equal_plain_processing():
