@@ -316,7 +316,8 @@ int oracle_sample_rows(const void* logits, int dtype, int rows, int V, const flo
  *   R12 order: repetition penalty and vocabulary mask act on the raw logits,
  *       then top-k (R4) on the result, then temperature and the softmax (R5),
  *       then the nucleus on the resulting probabilities;
- *   R13 repetition penalty theta > 0 on the sequence's listed token ids (each
+ *   R13 repetition penalty theta > 0 and finite (else a row error) on the
+ *       sequence's listed token ids (each
  *       id once, ids outside [0, V) ignored): z -> z / theta if z > 0, else
  *       z * theta, the result rounded to fp32 (the logit's quotient or product
  *       of two fp32 values, correctly rounded: computing it in double and
@@ -380,7 +381,8 @@ int oracle_process_row_procs(const void* row, int dtype, int V, double T, int to
     long v, n = 0, i;
     double tau = -INFINITY, m = -INFINITY, S = 0.0;
     if (!(T > 0.0) || isinf(T)) return 1;
-    if (!(pr->top_p > 0.0 && pr->top_p <= 1.0) || !(pr->rep_penalty > 0.0)) return 1;
+    if (!(pr->top_p > 0.0 && pr->top_p <= 1.0) || !(pr->rep_penalty > 0.0) || isinf(pr->rep_penalty))
+        return 1;
     for (v = 0; v < V; ++v) {
         double z0 = or_logit(row, dtype, v);
         if (isnan(z0) || z0 == INFINITY) return 1;

@@ -80,6 +80,7 @@ MUTANTS = [
      "z = (double)(float)(z / pr->rep_penalty);", 0),
     ("penalty_not_rounded", "z = z > 0.0 ? (double)(float)(z / pr->rep_penalty) : (double)(float)(z * pr->rep_penalty);",
      "z = z > 0.0 ? z / pr->rep_penalty : z * pr->rep_penalty;", 0),
+    ("penalty_infinite_accepted", "!(pr->rep_penalty > 0.0) || isinf(pr->rep_penalty)", "!(pr->rep_penalty > 0.0)", 0),
     ("penalty_per_listing", "break; /* each id once */", "/* every listing */", 0),
     ("penalty_ids_of_first_sequence", "pr.rep_ids = rep_ids ? rep_ids + (size_t)b * n_rep : NULL;",
      "pr.rep_ids = rep_ids;", 0),

@@ -94,6 +94,15 @@ def test_mask_bit_layout_word_boundaries():
         assert got[v] == 1.0 and got.sum() == 1.0
 
 
+@pytest.mark.parametrize("theta", [0.0, -1.5, float("nan"), float("inf")])
+def test_penalty_not_positive_and_finite_is_a_row_error(theta):
+    """Reading R13: theta must be finite and > 0, listed ids or not."""
+    z = f32([0.5, 1.0, 2.0])
+    assert oracle.process_row_procs(z, rep_penalty=theta, rep_ids=[1]) is None
+    assert oracle.process_row_procs(z, rep_penalty=theta) is None
+    assert oracle.process_row_procs(z, rep_penalty=2.0, rep_ids=[1]) is not None
+
+
 def test_everything_masked_is_a_row_error():
     assert oracle.process_row_procs(f32([0.0, 1.0, 2.0]), mask=oracle.allow_mask(3, [])) is None
 
