@@ -36,12 +36,14 @@ L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
 SPEC_HBM_GBS = 8000.0  # B200 HBM3e data-sheet bandwidth, for the fraction of the spec figure
 PROFILE_DIR = os.path.join(ROOT, "profiles")
-KSAMPLE = 8  # timed steps per streaming-kernel event sample
+KSAMPLES = 40  # event-bracketed launches of the streaming kernel per workload
 
 # sources that define the streaming kernel (the one the roofline figures describe)
 KERNEL_SOURCES = [os.path.join(ROOT, "draft_token_verification_verify_b200", "csrc", f)
                   for f in ("sv_rows.cuh", "sv_common.cuh", "sv_ptx.cuh")]
 
+WORKLOAD_ORDER = ("batched", "greedy", "large", "single", "tiny")
+GRAPH_WORKLOADS = ("single", "tiny")  # launch-bound: also timed from a CUDA-graph replay
 DESCR = {
     "tiny": "tiny stochastic verify B=1 k=4 V=32 fp32 T=1",
     "single": "single-sequence stochastic verify B=1 k=8 V=151936 bf16 T=1",
@@ -367,26 +369,13 @@ def run_reference(args):
     return 0
 
 
-def run_ours(args):
+def measure_workload(name, args, sv, dev, world, rank, local, e2e_leg=False):
+    """Time one workload: K steps bracketed by synchronize (and a barrier plus
+    the max over ranks under torchrun), the streaming kernel alone from CUDA
+    events over its own KSAMPLES launches, clocks sampled while the same steps
+    run, and optionally the end-to-end leg and a CUDA-graph replay."""
     import torch
 
-    import draft_token_verification_verify_b200 as sv
-
-    world, rank, local = dist_env()
-    if not torch.cuda.is_available():
-        raise SystemExit("bench.py needs a CUDA device")
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-
-        import torch.distributed as dist
-
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-    sv.lib()
-
-    name = args.workload
-    w = workloads.WORKLOADS[name]
     case = workloads.make_case(name, seed=rank_seed(rank))
     B, k, V = case.B, case.k, case.V
     greedy = case.mode == "greedy"
@@ -429,7 +418,7 @@ def run_ours(args):
         step(i)
     torch.cuda.synchronize()
     if int(status.item()) != 0:
-        raise SystemExit(f"device status {int(status.item())} during warm-up")
+        raise SystemExit(f"{name}: device status {int(status.item())} during warm-up")
 
     # clock window: the same work back to back while nvidia-smi samples
     sampler = ClockSampler(local)
@@ -437,52 +426,69 @@ def run_ours(args):
     t_end = time.perf_counter() + args.clock_window
     i = 0
     while time.perf_counter() < t_end:
-        for _ in range(64):
+        for _ in range(32):
             step(i)
             i += 1
         torch.cuda.synchronize()
 
-    # ---- timed region: exactly K steps --------------------------------------------
-    # The streaming kernel is timed with a CUDA event pair on one timed step in
-    # KSAMPLE; an event between the two launches of a step stops the second
-    # from starting early, so the other steps run without one.
-    sampled = list(range(0, args.steps, KSAMPLE))
-    evk = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in sampled]
+    # ---- timed region: exactly K steps, no event between the launches ---------------
     t_start = torch.cuda.Event(enable_timing=True)
     t_stop = torch.cuda.Event(enable_timing=True)
-    for a, b in evk:  # torch creates the CUDA event on first record
-        a.record(stream)
-        b.record(stream)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
     t_start.record(stream)
-    for s in range(args.steps):
-        if s % KSAMPLE == 0:
-            step(s, *evk[s // KSAMPLE])
-        else:
-            step(s)
+    for s_ in range(args.steps):
+        step(s_)
     t_stop.record(stream)
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
-    clocks = sampler.stop()
     elapsed_ms = max_over_ranks(t_start.elapsed_time(t_stop), dev)
+    if int(status.item()) != 0:
+        raise SystemExit(f"{name}: device status {int(status.item())} in the timed region")
+
+    # ---- the streaming kernel alone: an event pair around it on KSAMPLES steps ------
+    # (an event between the two launches of a step stops the second from starting
+    # early, so these steps are timed apart from the K above)
+    evk = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(KSAMPLES)]
+    for a, b in evk:  # torch creates the CUDA event on first record
+        a.record(stream)
+        b.record(stream)
+    torch.cuda.synchronize()
+    for j_, (a, b) in enumerate(evk):
+        step(args.steps + j_, a, b)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
     kern_ms = [a.elapsed_time(b) for a, b in evk]
     if int(status.item()) != 0:
-        raise SystemExit(f"device status {int(status.item())} in the timed region")
+        raise SystemExit(f"{name}: device status {int(status.item())} in the kernel samples")
 
     value = job_rate(B * k * args.steps, world, elapsed_ms)
     gbs = job_rate(logit_bytes * args.steps, world, elapsed_ms) / 1e9
     kmean = sum(kern_ms) / len(kern_ms)
     peak, peak_src = measured_peak()
     achieved = logit_bytes / (kmean / 1000.0) / 1e9
-    traffic = profiled_traffic(name)
+    out = {
+        "workload": DESCR[name], "B": B, "k": k, "V": V, "top_k": case.top_k, "mode": case.mode,
+        "dtype": case.dtype, "value": value, "unit": "positions/s", "steps": args.steps,
+        "ms_per_step": elapsed_ms / args.steps, "logit_gbs": gbs, "logit_bytes_per_step": logit_bytes,
+        "l2": f"{nsets} rotating input set(s) of {logit_bytes / 1e6:.1f} MB"
+              + (" (> 126 MB L2 in rotation)" if nsets * logit_bytes > L2_BYTES else ""),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": profiled_traffic(name), "peak_source": peak_src,
+                     "kernel": "sv_rows_kernel", "kernel_ms_mean": kmean,
+                     "kernel_ms_median": statistics.median(kern_ms),
+                     "kernel_ms_p10": pctl(kern_ms, 10), "kernel_ms_p90": pctl(kern_ms, 90),
+                     "kernel_samples": len(kern_ms),
+                     "frac_of_spec": achieved / SPEC_HBM_GBS, "spec_gbs": SPEC_HBM_GBS},
+        "gpu_launches": launches_per_step(case) * args.steps,
+        "clocks": clocks,
+    }
 
     # ---- end to end through the public API, host (pinned) buffers -------------------
-    e2e = None
-    if not args.no_e2e:
+    if e2e_leg:
         h_target = to_pinned(case.target)
         h_draft = None if greedy else to_pinned(case.draft)
         h_tok = drafts.cpu().pin_memory()
@@ -525,12 +531,11 @@ def run_ours(args):
         b.record(stream)
         torch.cuda.synchronize()
         e_ms = max_over_ranks(a.elapsed_time(b), dev)
-        e2e = {"value": job_rate(B * k * n_e2e, world, e_ms), "unit": "positions/s",
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": n_e2e}
+        out["e2e"] = {"value": job_rate(B * k * n_e2e, world, e_ms), "unit": "positions/s",
+                      "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": n_e2e}
 
-    # ---- optional: the same steps replayed from a CUDA graph (launch-bound workloads) ---
-    graph = None
-    if args.graph:
+    # ---- the same steps replayed from a CUDA graph (launch-bound workloads) ---------
+    if args.graph or name in GRAPH_WORKLOADS:
         gs = torch.cuda.Stream(device=dev)
         gs.wait_stream(stream)
         per_graph = 16
@@ -550,20 +555,57 @@ def run_ours(args):
         gb.record(rs)
         torch.cuda.synchronize()
         g_ms = max_over_ranks(ga.elapsed_time(gb), dev) / (reps * per_graph)
-        graph = {"value": job_rate(B * k, world, g_ms), "unit": "positions/s", "ms_per_step": g_ms,
-                 "steps_per_graph": per_graph}
+        out["graph"] = {"value": job_rate(B * k, world, g_ms), "unit": "positions/s", "ms_per_step": g_ms,
+                        "steps_per_graph": per_graph}
         del g
+    out["_drafts"] = drafts.cpu().numpy()
+    out["_case"] = case
+    del targets, drafts_l, target0, draft0, wsp
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_ours(args):
+    import torch
+
+    import draft_token_verification_verify_b200 as sv
+
+    world, rank, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    sv.lib()
+
+    name = args.workload
+    head = measure_workload(name, args, sv, dev, world, rank, local, e2e_leg=not args.no_e2e)
+    others = {}
+    if not args.headline_only:
+        for other in WORKLOAD_ORDER:
+            if other == name:
+                continue
+            r = measure_workload(other, args, sv, dev, world, rank, local)
+            r.pop("_drafts")
+            r.pop("_case")
+            others[other] = r
+    case, drafts = head.pop("_case"), head.pop("_drafts")
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         try:
             cpu = cpu_baseline(name, args.cpu_budget)
         except Exception as exc:  # the multi-process leg failed: one thread instead
-            cpu = cpu_baseline_single(name, case, drafts.cpu().numpy(), args.cpu_budget,
+            cpu = cpu_baseline_single(name, case, drafts, args.cpu_budget,
                                       f"multi-process run failed: {type(exc).__name__}")
         if cpu.get("cores", 1) > 1:  # the one-core figure beside the all-core one
             try:
-                one = cpu_baseline_single(name, case, drafts.cpu().numpy(), args.cpu_budget / 3,
+                one = cpu_baseline_single(name, case, drafts, args.cpu_budget / 3,
                                           "one core, beside the all-core figure")
                 cpu["single_core"] = {"value": one["value"], "unit": one["unit"], "sample": one["sample"]}
             except Exception as exc:
@@ -575,29 +617,24 @@ def run_ours(args):
     if rank != 0:
         return 0
     line = {
-        "metric": "verified draft positions/sec", "value": value, "unit": "positions/s",
+        "metric": "verified draft positions/sec", "value": head["value"], "unit": "positions/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": case.dtype, "data": "synthetic",
-        "config": {"workload": DESCR[name], "B": B, "k": k, "V": V, "top_k": case.top_k,
-                   "mode": case.mode, "per_rank_batch": B, "parallelism": f"replicas x{world}",
-                   "l2": f"{nsets} rotating input sets of {logit_bytes / 1e6:.1f} MB (> 126 MB L2)",
+        "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": head["dtype"], "data": "synthetic",
+        "config": {"workload": head["workload"], "B": head["B"], "k": head["k"], "V": head["V"],
+                   "top_k": head["top_k"], "mode": head["mode"], "per_rank_batch": head["B"],
+                   "parallelism": f"replicas x{world}", "l2": head["l2"],
                    "clocks_window": f"sampled over a {args.clock_window:.1f} s window of the same "
-                                    "steps right before the timed region"},
-        "logit_gbs": gbs,
-        "logit_bytes_per_step": logit_bytes,
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
-                     "kernel": "sv_rows_kernel", "kernel_ms_mean": kmean,
-                     "kernel_ms_median": statistics.median(kern_ms),
-                     "kernel_ms_p10": pctl(kern_ms, 10), "kernel_ms_p90": pctl(kern_ms, 90),
-                     "kernel_samples": len(kern_ms),
-                     "frac_of_spec": achieved / SPEC_HBM_GBS, "spec_gbs": SPEC_HBM_GBS},
-        "gpu_launches": launches_per_step(case) * args.steps,
-        "clocks": clocks,
-        "e2e": e2e,
-        **({"graph": graph} if graph is not None else {}),
+                                    "steps right before the timed region and during the kernel samples"},
+        "logit_gbs": head["logit_gbs"],
+        "logit_bytes_per_step": head["logit_bytes_per_step"],
+        "roofline": head["roofline"],
+        "gpu_launches": head["gpu_launches"],
+        "clocks": head["clocks"],
+        "e2e": head.get("e2e"),
+        **({"graph": head["graph"]} if "graph" in head else {}),
         "cpu_baseline": cpu,
+        "workloads": others,
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -610,12 +647,14 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(workloads.WORKLOADS), default="batched")
-    ap.add_argument("--clock-window", type=float, default=1.5)
+    ap.add_argument("--clock-window", type=float, default=1.0)
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--graph", action="store_true",
-                    help="also time the steps replayed from a CUDA graph (latency-bound workloads)")
+                    help="also time the headline's steps replayed from a CUDA graph")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="measure only --workload (default: every workload, the headline first)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

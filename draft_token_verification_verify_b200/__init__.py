@@ -52,6 +52,11 @@ class SvOptions(ctypes.Structure):
         ("wait_timeout_ns", ctypes.c_uint64),
         ("test_extra_tx", ctypes.c_uint32),
         ("top_p", ctypes.c_void_p),
+        ("vocab_mask", ctypes.c_void_p),
+        ("rep_ids", ctypes.c_void_p),
+        ("n_rep", ctypes.c_int),
+        ("rep_penalty", ctypes.c_void_p),
+        ("rows_per_sequence", ctypes.c_int),
     ]
 
 
@@ -187,11 +192,19 @@ def spec_sample_ex(logits, uniforms, rows, V, temperature, top_k, mode, out_toke
 
 
 def make_options(chunks_per_row=0, threads=0, topk_path=0, event_start=None, event_stop=None,
-                 wait_timeout_ns=0, test_extra_tx=0, top_p=None) -> SvOptions:
-    """``sv_options_t``; ``top_p`` is a [B] fp32 device tensor (nucleus per
-    sequence, top-k path only) or None.  Keep it alive until the call completes."""
+                 wait_timeout_ns=0, test_extra_tx=0, top_p=None, vocab_mask=None, rep_ids=None,
+                 rep_penalty=None, rows_per_sequence=0) -> SvOptions:
+    """``sv_options_t``.  Per-sequence processor inputs are device tensors or
+    None: ``top_p`` [S] fp32 (nucleus), ``vocab_mask`` [S, ceil(V/32)] uint32
+    bit words (passed as int32), ``rep_ids`` [S, n_rep] int32 and
+    ``rep_penalty`` [S] fp32.  Keep them alive until the call completes."""
+    n_rep = 0
+    if rep_ids is not None:
+        n_rep = rep_ids.shape[-1] if rep_ids.dim() > 1 else rep_ids.numel()
+    ptr = lambda t: None if t is None else _p(t).value
     return SvOptions(chunks_per_row, threads, topk_path, _event(event_start), _event(event_stop),
-                     wait_timeout_ns, test_extra_tx, None if top_p is None else _p(top_p).value)
+                     wait_timeout_ns, test_extra_tx, ptr(top_p), ptr(vocab_mask), ptr(rep_ids), n_rep,
+                     ptr(rep_penalty), rows_per_sequence)
 
 
 def _dtype_code(t) -> int:

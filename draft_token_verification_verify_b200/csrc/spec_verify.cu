@@ -24,7 +24,6 @@ constexpr uint64_t kDefaultTimeoutNs = 1000000000ull;
 constexpr int kSegBytes = sv::TILE_BYTES;  // bytes per segment (one ring stage)
 constexpr int kStages = 2;                 // ring stages of the streaming kernel
 constexpr int kTopkMax = 256;         // largest K on the kept-list path (<= threads)
-constexpr int kListCap = 1024;        // shared candidate list of a streaming CTA
 
 struct DeviceInfo {
     int ok = 0;
@@ -38,10 +37,14 @@ struct DeviceInfo {
 DeviceInfo g_dev[kMaxDevices];
 std::once_flag g_dev_once[kMaxDevices];
 std::once_flag g_pool_once[kMaxDevices];
-std::once_flag g_attr_once[kMaxDevices][26];
-cudaError_t g_attr_err[kMaxDevices][26];  // result of each one-time attribute call
-std::once_flag g_occ_once[kMaxDevices][24];
-int g_occ[kMaxDevices][24];
+// streaming-kernel instantiations: 24 plain (dtype x threads x mode) and 12 with
+// processors (dtype x 128/256 threads x softmax/top-k/max-only); then the two
+// per-sequence kernels
+constexpr int kRowsSlots = 36;
+std::once_flag g_attr_once[kMaxDevices][kRowsSlots + 2];
+cudaError_t g_attr_err[kMaxDevices][kRowsSlots + 2];  // result of each one-time attribute call
+std::once_flag g_occ_once[kMaxDevices][kRowsSlots];
+int g_occ[kMaxDevices][kRowsSlots];
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -98,6 +101,10 @@ long long ceil_div(long long a, long long b) { return (a + b - 1) / b; }
 long long round_up(long long a, long long b) { return ceil_div(a, b) * b; }
 
 struct Plan {
+    bool proc = false;  // processors: K0 builds the bitmaps, K1 runs its PROC variant
+    int W4 = 0;         // words per bitmap row
+    long long nprocs = 0;  // processor rows (sequences)
+    size_t off_allow = 0, off_pen = 0;
     int mode = 0, elt = 2, seg = 0, nseg = 0, nch = 1, spc = 1, nt1 = 128, stages = kStages;
     int lcap = 0, kcap = 0, mg = 0;
     long long R = 0, tasks = 0, slots = 0;
@@ -109,13 +116,16 @@ struct Plan {
     size_t off_req = 0, off_mass = 0, off_counter = 0;
 };
 
-int rows_occupancy(int dev, int dt, int nt, int mode, size_t smem);
+int rows_occupancy(int dev, int dt, int nt, int mode, bool proc, size_t smem);
 
 // Plan the launches for `seqs` sequences of draft length k (rows = k+1 target
-// rows per sequence, plus k draft rows when stochastic).
+// rows per sequence, plus k draft rows when stochastic); `nprocs` > 0 when the
+// processors are in use (their rows: one per sequence).
 sv_status_t make_plan(const DeviceInfo& dev, long long seqs, int k, int V, int dt, bool greedy, int top_k,
-                      const sv_options_t* opts, Plan* out) {
+                      const sv_options_t* opts, long long nprocs, Plan* out) {
     Plan p;
+    p.proc = nprocs > 0;
+    p.nprocs = nprocs;
     p.elt = dt ? 4 : 2;
     const int vec = 16 / p.elt;
     p.nt1 = (opts && opts->threads) ? opts->threads : 128;
@@ -132,6 +142,7 @@ sv_status_t make_plan(const DeviceInfo& dev, long long seqs, int k, int V, int d
     else
         p.mode = sv::MODE_MAXONLY;
     if (opts && opts->topk_path == 1 && top_k > 0 && p.mode != sv::MODE_TOPK) return SV_ERR_UNSUPPORTED;
+    if (p.proc && (greedy || p.nt1 == 512)) return SV_ERR_UNSUPPORTED;
     if (p.mode == sv::MODE_TOPK) {
         // the running bound needs K <= threads (each warp contributes <= 32 ranks)
         if (top_k > p.nt1) {
@@ -142,12 +153,13 @@ sv_status_t make_plan(const DeviceInfo& dev, long long seqs, int k, int V, int d
                 p.nt1 = 256;
             }
         }
-        if (p.mode == sv::MODE_TOPK) p.lcap = kListCap;
+        if (p.mode == sv::MODE_TOPK) p.lcap = (p.nt1 / 32) * sv::TOPK_WCAP;
     }
-    p.smem1 = static_cast<size_t>(sv::rows_smem_bytes(p.mode, p.nt1, p.stages, p.lcap));
+    if (p.proc && p.nt1 == 512) return SV_ERR_UNSUPPORTED;
+    p.smem1 = static_cast<size_t>(sv::rows_smem_bytes(p.mode, p.nt1, p.stages, p.lcap, p.proc));
     if (p.smem1 > static_cast<size_t>(dev.smem_optin)) return SV_ERR_UNSUPPORTED;
     // chunks per row: one when there are enough rows to fill the device
-    long long occ = rows_occupancy(dev.id, dt, p.nt1, p.mode, p.smem1);
+    long long occ = rows_occupancy(dev.id, dt, p.nt1, p.mode, p.proc, p.smem1);
     if (occ < 1) return SV_ERR_CUDA;
     const long long slots = occ * dev.sms;
     p.slots = slots;
@@ -175,16 +187,24 @@ sv_status_t make_plan(const DeviceInfo& dev, long long seqs, int k, int V, int d
         p.kcap = 0;
         p.mg = 64;  // also holds the two draw lists of the top-k path
     }
-    // workspace: segment partials, chunk headers, kept lists
-    const size_t segs = static_cast<size_t>(p.R) * p.nseg * sizeof(sv::SegRec);
-    p.off_chunks = round_up(segs, 256);
+    // workspace: segment partials (not in top-k mode), chunk headers, kept lists
+    const size_t segs = p.mode == sv::MODE_TOPK ? 0 : static_cast<size_t>(p.R) * p.nseg * sizeof(sv::SegRec);
     size_t chunks = 0, cands = 0;
     if (p.mode == sv::MODE_TOPK) {
         chunks = static_cast<size_t>(p.R) * p.nch * sizeof(sv::ChunkRec);
         cands = static_cast<size_t>(p.R) * p.nch * p.kcap * sizeof(sv::Cand);
     }
+    p.off_chunks = round_up(segs, 256);
     p.off_cands = round_up(p.off_chunks + chunks, 256);
     p.ws_bytes = round_up(p.off_cands + cands, 256);
+    // processors: allow and penalty bitmaps, rows of W4 words (a multiple of 4)
+    if (p.proc) {
+        p.W4 = static_cast<int>(4 * ceil_div(V, 128));
+        const size_t bm = static_cast<size_t>(nprocs) * p.W4 * sizeof(uint32_t);
+        p.off_allow = p.ws_bytes;
+        p.off_pen = round_up(p.off_allow + bm, 256);
+        p.ws_bytes = round_up(p.off_pen + bm, 256);
+    }
     // softmax verification: residual draws by the segment kernel
     p.defer = p.mode == sv::MODE_SOFTMAX && k > 0;
     if (p.defer) {
@@ -217,56 +237,71 @@ sv_status_t make_plan(const DeviceInfo& dev, long long seqs, int k, int V, int d
 using RowsFn = void (*)(sv::RowsParams);
 using SeqFn = void (*)(sv::SeqParams);
 using ResFn = void (*)(sv::ResidParams);
+using ProcsFn = void (*)(sv::ProcsParams);
 
-template <int DT, int NT>
+template <int DT, int NT, bool PROC>
 RowsFn rows_for_mode(int mode) {
-    switch (mode) {
-        case sv::MODE_GREEDY: return sv::sv_rows_kernel<DT, NT, sv::MODE_GREEDY>;
-        case sv::MODE_SOFTMAX: return sv::sv_rows_kernel<DT, NT, sv::MODE_SOFTMAX>;
-        case sv::MODE_TOPK: return sv::sv_rows_kernel<DT, NT, sv::MODE_TOPK>;
-        default: return sv::sv_rows_kernel<DT, NT, sv::MODE_MAXONLY>;
+    if constexpr (PROC) {  // the processors have no greedy variant (rejected by the plan)
+        switch (mode) {
+            case sv::MODE_SOFTMAX: return sv::sv_rows_kernel<DT, NT, sv::MODE_SOFTMAX, true>;
+            case sv::MODE_TOPK: return sv::sv_rows_kernel<DT, NT, sv::MODE_TOPK, true>;
+            default: return sv::sv_rows_kernel<DT, NT, sv::MODE_MAXONLY, true>;
+        }
+    } else {
+        switch (mode) {
+            case sv::MODE_GREEDY: return sv::sv_rows_kernel<DT, NT, sv::MODE_GREEDY, false>;
+            case sv::MODE_SOFTMAX: return sv::sv_rows_kernel<DT, NT, sv::MODE_SOFTMAX, false>;
+            case sv::MODE_TOPK: return sv::sv_rows_kernel<DT, NT, sv::MODE_TOPK, false>;
+            default: return sv::sv_rows_kernel<DT, NT, sv::MODE_MAXONLY, false>;
+        }
     }
 }
 
-// slot = dtype * 12 + threads-class * 4 + mode (24 instantiations)
-RowsFn pick_rows(int dt, int nt, int mode, int* slot) {
+// slot = dtype * 12 + threads-class * 4 + mode (24 plain instantiations), then
+// 24 + dtype * 6 + threads-class * 3 + (mode - 1) with processors (12 more)
+RowsFn pick_rows(int dt, int nt, int mode, bool proc, int* slot) {
     const int ntc = nt == 128 ? 0 : (nt == 512 ? 2 : 1);
-    *slot = dt * 12 + ntc * 4 + mode;
-    if (dt == 0) {
-        if (nt == 128) return rows_for_mode<0, 128>(mode);
-        if (nt == 512) return rows_for_mode<0, 512>(mode);
-        return rows_for_mode<0, 256>(mode);
+    *slot = proc ? 24 + dt * 6 + ntc * 3 + (mode - 1) : dt * 12 + ntc * 4 + mode;
+    if (proc) {
+        if (dt == 0) return nt == 128 ? rows_for_mode<0, 128, true>(mode) : rows_for_mode<0, 256, true>(mode);
+        return nt == 128 ? rows_for_mode<1, 128, true>(mode) : rows_for_mode<1, 256, true>(mode);
     }
-    if (nt == 128) return rows_for_mode<1, 128>(mode);
-    if (nt == 512) return rows_for_mode<1, 512>(mode);
-    return rows_for_mode<1, 256>(mode);
+    if (dt == 0) {
+        if (nt == 128) return rows_for_mode<0, 128, false>(mode);
+        if (nt == 512) return rows_for_mode<0, 512, false>(mode);
+        return rows_for_mode<0, 256, false>(mode);
+    }
+    if (nt == 128) return rows_for_mode<1, 128, false>(mode);
+    if (nt == 512) return rows_for_mode<1, 512, false>(mode);
+    return rows_for_mode<1, 256, false>(mode);
 }
 
-sv_status_t set_attrs(int dev, int dt, int nt, int mode) {
+sv_status_t set_attrs(int dev, int dt, int nt, int mode, bool proc) {
     int slot = 0;
-    RowsFn f1 = pick_rows(dt, nt, mode, &slot);
+    RowsFn f1 = pick_rows(dt, nt, mode, proc, &slot);
     SeqFn f2 = dt ? sv::sv_seq_kernel<1> : sv::sv_seq_kernel<0>;
     std::call_once(g_attr_once[dev][slot], [&] {
         g_attr_err[dev][slot] =
             cudaFuncSetAttribute(f1, cudaFuncAttributeMaxDynamicSharedMemorySize, g_dev[dev].smem_optin);
         if (g_attr_err[dev][slot] != cudaSuccess) cudaGetLastError();
     });
-    std::call_once(g_attr_once[dev][24 + dt], [&] {
-        g_attr_err[dev][24 + dt] =
+    const int s2 = kRowsSlots + dt;
+    std::call_once(g_attr_once[dev][s2], [&] {
+        g_attr_err[dev][s2] =
             cudaFuncSetAttribute(f2, cudaFuncAttributeMaxDynamicSharedMemorySize, g_dev[dev].smem_optin);
-        if (g_attr_err[dev][24 + dt] != cudaSuccess) cudaGetLastError();
+        if (g_attr_err[dev][s2] != cudaSuccess) cudaGetLastError();
     });
     // a failed attribute call fails every later call for that kernel too
-    if (g_attr_err[dev][slot] != cudaSuccess || g_attr_err[dev][24 + dt] != cudaSuccess) return SV_ERR_CUDA;
+    if (g_attr_err[dev][slot] != cudaSuccess || g_attr_err[dev][s2] != cudaSuccess) return SV_ERR_CUDA;
     return SV_OK;
 }
 
 // Resident streaming CTAs per SM for one instantiation (its shared memory
 // depends only on the slot), from the occupancy calculator; 0 on failure.
-int rows_occupancy(int dev, int dt, int nt, int mode, size_t smem) {
-    if (set_attrs(dev, dt, nt, mode) != SV_OK) return 0;
+int rows_occupancy(int dev, int dt, int nt, int mode, bool proc, size_t smem) {
+    if (set_attrs(dev, dt, nt, mode, proc) != SV_OK) return 0;
     int slot = 0;
-    RowsFn f1 = pick_rows(dt, nt, mode, &slot);
+    RowsFn f1 = pick_rows(dt, nt, mode, proc, &slot);
     std::call_once(g_occ_once[dev][slot], [&] {
         int n = 0;
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, f1, nt + 32, smem) != cudaSuccess) {
@@ -279,6 +314,13 @@ int rows_occupancy(int dev, int dt, int nt, int mode, size_t smem) {
 }
 
 struct Call {
+    // processors (options): mask [S][ceil(V/32)], rep_ids [S][n_rep], rep_penalty [S]
+    const uint32_t* mask = nullptr;
+    const int32_t* rep_ids = nullptr;
+    int n_rep = 0;
+    const float* rep_penalty = nullptr;
+    long long rows_per_seq = 1;  // sampler: rows per processor sequence
+    long long nprocs = 0;        // processor rows (0: no processors)
     const void* target = nullptr;
     const void* draft = nullptr;
     const int32_t* draft_tokens = nullptr;
@@ -300,11 +342,11 @@ sv_status_t run(const Call& cl, void* workspace, size_t workspace_bytes, const s
     const DeviceInfo* info = device_info(&dev);
     if (!info) return SV_ERR_UNSUPPORTED;
     Plan p;
-    sv_status_t s = make_plan(*info, cl.seqs, cl.k, cl.V, cl.dt, cl.greedy, cl.top_k, opts, &p);
+    sv_status_t s = make_plan(*info, cl.seqs, cl.k, cl.V, cl.dt, cl.greedy, cl.top_k, opts, cl.nprocs, &p);
     if (s != SV_OK) return s;
     if (workspace && (workspace_bytes < p.ws_bytes || !aligned(workspace, 16))) return SV_ERR_INVALID_ARG;
     if (opts && opts->top_p && p.mode != sv::MODE_TOPK) return SV_ERR_UNSUPPORTED;  // nucleus needs the kept lists
-    if ((s = set_attrs(dev, cl.dt, p.nt1, p.mode)) != SV_OK) return s;
+    if ((s = set_attrs(dev, cl.dt, p.nt1, p.mode, p.proc)) != SV_OK) return s;
 
     void* ws = workspace;
     bool owned = false;
@@ -340,6 +382,24 @@ sv_status_t run(const Call& cl, void* workspace, size_t workspace_bytes, const s
     r.out_status = cl.sample ? nullptr : cl.out_status;
     r.timeout_ns = (opts && opts->wait_timeout_ns) ? opts->wait_timeout_ns : kDefaultTimeoutNs;
     r.test_extra_tx = opts ? opts->test_extra_tx : 0u;
+    sv::ProcsParams pp;
+    std::memset(&pp, 0, sizeof pp);
+    if (p.proc) {
+        pp.mask = cl.mask;
+        pp.rep_ids = cl.rep_ids;
+        pp.n_rep = cl.n_rep;
+        pp.rep_penalty = cl.rep_penalty;
+        pp.V = cl.V;
+        pp.words = static_cast<int>(ceil_div(cl.V, 32));
+        pp.W4 = p.W4;
+        pp.allow = reinterpret_cast<uint32_t*>(base + p.off_allow);
+        pp.pen = reinterpret_cast<uint32_t*>(base + p.off_pen);
+        r.allow = pp.allow;
+        r.pen = pp.pen;
+        r.theta = cl.rep_penalty;
+        r.W4 = p.W4;
+    }
+    r.procs_div = static_cast<int>(cl.rows_per_seq);
 
     sv::SeqParams q;
     std::memset(&q, 0, sizeof q);
@@ -363,6 +423,7 @@ sv_status_t run(const Call& cl, void* workspace, size_t workspace_bytes, const s
     q.segs = r.segs;
     q.chunks = r.chunks;
     q.cands = r.cands;
+
     q.out_tokens = cl.out_tokens;
     q.out_n = cl.out_n;
     q.out_p = cl.out_p;
@@ -374,6 +435,11 @@ sv_status_t run(const Call& cl, void* workspace, size_t workspace_bytes, const s
     q.pre_off = static_cast<int>(p.pre_off);
     q.req = p.defer ? reinterpret_cast<sv::DrawReq*>(base + p.off_req) : nullptr;
     q.counter = p.defer ? reinterpret_cast<int*>(base + p.off_counter) : nullptr;
+    q.allow = r.allow;
+    q.pen = r.pen;
+    q.theta = r.theta;
+    q.W4 = r.W4;
+    q.procs_div = r.procs_div;
 
     sv::ResidParams rp;
     std::memset(&rp, 0, sizeof rp);
@@ -388,6 +454,10 @@ sv_status_t run(const Call& cl, void* workspace, size_t workspace_bytes, const s
     rp.counter = q.counter;
     rp.out_tokens = cl.out_tokens;
     rp.out_n = cl.out_n;
+    rp.allow = r.allow;
+    rp.pen = r.pen;
+    rp.theta = r.theta;
+    rp.W4 = r.W4;
 
     sv_status_t result = SV_OK;
     do {
@@ -396,8 +466,22 @@ sv_status_t run(const Call& cl, void* workspace, size_t workspace_bytes, const s
             result = SV_ERR_CUDA;
             break;
         }
+        if (p.proc) {
+            // K0: the processors' bitmaps, in plain stream order after the
+            // previous call's kernels (which may still read them)
+            cudaLaunchConfig_t c0;
+            std::memset(&c0, 0, sizeof c0);
+            c0.gridDim = dim3(static_cast<unsigned>(p.nprocs), 1, 1);
+            c0.blockDim = dim3(sv::PROCS_NT, 1, 1);
+            c0.stream = st;
+            ProcsFn f0 = sv::sv_procs_kernel;
+            if (cudaLaunchKernelEx(&c0, f0, pp) != cudaSuccess) {
+                result = SV_ERR_CUDA;
+                break;
+            }
+        }
         int slot = 0;
-        RowsFn f1 = pick_rows(cl.dt, p.nt1, p.mode, &slot);
+        RowsFn f1 = pick_rows(cl.dt, p.nt1, p.mode, p.proc, &slot);
         cudaLaunchConfig_t c1;
         std::memset(&c1, 0, sizeof c1);
         c1.gridDim = dim3(static_cast<unsigned>(p.tasks), 1, 1);
@@ -407,8 +491,9 @@ sv_status_t run(const Call& cl, void* workspace, size_t workspace_bytes, const s
         // programmatic dependent launch: the streaming pass may be placed while
         // the preceding kernel finishes (it waits for that grid before any
         // access).  Not for a single wave that fills more than half the device:
-        // CTAs placed early, as slots free up, spread unevenly over the SMs and
-        // such a grid has no later wave to even it out.
+        // CTAs placed early, as slots free up (the preceding kernels are
+        // themselves placed early), land unevenly, and a few can miss the wave
+        // altogether and run after it (measured: +20 us per step).
         cudaLaunchAttribute a1[1];
         a1[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
         a1[0].val.programmaticStreamSerializationAllowed = 1;
@@ -424,15 +509,15 @@ sv_status_t run(const Call& cl, void* workspace, size_t workspace_bytes, const s
             result = SV_ERR_CUDA;
             break;
         }
+        cudaLaunchAttribute a2[1];
+        a2[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        a2[0].val.programmaticStreamSerializationAllowed = 1;
         cudaLaunchConfig_t c2;
         std::memset(&c2, 0, sizeof c2);
         c2.gridDim = dim3(static_cast<unsigned>(cl.seqs), 1, 1);
         c2.blockDim = dim3(sv::SEQ_NT, 1, 1);
         c2.dynamicSmemBytes = p.smem2;
         c2.stream = st;
-        cudaLaunchAttribute a2[1];
-        a2[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        a2[0].val.programmaticStreamSerializationAllowed = 1;
         c2.attrs = a2;
         c2.numAttrs = 1;
         SeqFn f2 = cl.dt ? sv::sv_seq_kernel<1> : sv::sv_seq_kernel<0>;
@@ -471,6 +556,24 @@ sv_status_t check_options(const sv_options_t* o) {
         return SV_ERR_INVALID_ARG;
     if (o->topk_path < 0 || o->topk_path > 2) return SV_ERR_INVALID_ARG;
     if (o->top_p && !aligned(o->top_p, 4)) return SV_ERR_INVALID_ARG;
+    if (o->n_rep < 0 || o->rows_per_sequence < 0) return SV_ERR_INVALID_ARG;
+    if ((o->vocab_mask && !aligned(o->vocab_mask, 4)) || (o->rep_ids && !aligned(o->rep_ids, 4)) ||
+        (o->rep_penalty && !aligned(o->rep_penalty, 4)))
+        return SV_ERR_INVALID_ARG;
+    return SV_OK;
+}
+
+// The processor inputs of the options, for `nseq` processor rows; greedy
+// verification takes none.
+sv_status_t take_procs(const sv_options_t* o, bool greedy, long long nseq, long long rows_per_seq, Call* cl) {
+    cl->rows_per_seq = rows_per_seq;
+    if (!o || !(o->vocab_mask || (o->rep_ids && o->n_rep > 0) || o->rep_penalty)) return SV_OK;
+    if (greedy) return SV_ERR_UNSUPPORTED;
+    cl->mask = o->vocab_mask;
+    cl->rep_ids = o->n_rep > 0 ? o->rep_ids : nullptr;
+    cl->n_rep = o->n_rep > 0 && o->rep_ids ? o->n_rep : 0;
+    cl->rep_penalty = o->rep_penalty;
+    cl->nprocs = nseq;
     return SV_OK;
 }
 
@@ -524,7 +627,7 @@ sv_status_t verify_args(const void* target_logits, const void* draft_logits, con
     cl->out_p = greedy ? nullptr : out_p;
     cl->out_q = greedy ? nullptr : out_q;
     cl->out_status = out_status;
-    return SV_OK;
+    return take_procs(opts, greedy, B, 1, cl);
 }
 
 sv_status_t sample_args(const void* logits, const float* uniforms, int rows, int V, const float* temperature,
@@ -535,7 +638,6 @@ sv_status_t sample_args(const void* logits, const float* uniforms, int rows, int
     if (rows <= 0 || V < 1 || top_k < 0) return SV_ERR_INVALID_ARG;
     if (!decode_mode(mode, &greedy, &dt)) return SV_ERR_INVALID_ARG;
     if (check_options(opts) != SV_OK) return SV_ERR_INVALID_ARG;
-    if (opts && opts->top_p) return SV_ERR_UNSUPPORTED;  // the nucleus is offered for verification only
     const int elt = dt ? 4 : 2;
     if (static_cast<unsigned long long>(rows) > (1ULL << 62) / (static_cast<unsigned long long>(V) * 4ULL))
         return SV_ERR_INVALID_ARG;
@@ -557,7 +659,8 @@ sv_status_t sample_args(const void* logits, const float* uniforms, int rows, int
     cl->greedy = greedy;
     cl->sample = true;
     cl->out_tokens = out_tokens;
-    return SV_OK;
+    const long long rps = (opts && opts->rows_per_sequence > 0) ? opts->rows_per_sequence : 1;
+    return take_procs(opts, greedy, ceil_div(rows, rps), rps, cl);
 }
 
 size_t workspace_for(const Call& cl, const sv_options_t* opts) {
@@ -565,7 +668,7 @@ size_t workspace_for(const Call& cl, const sv_options_t* opts) {
     const DeviceInfo* info = device_info(&dev);
     if (!info) return 0;
     Plan p;
-    if (make_plan(*info, cl.seqs, cl.k, cl.V, cl.dt, cl.greedy, cl.top_k, opts, &p) != SV_OK) return 0;
+    if (make_plan(*info, cl.seqs, cl.k, cl.V, cl.dt, cl.greedy, cl.top_k, opts, cl.nprocs, &p) != SV_OK) return 0;
     return p.ws_bytes;
 }
 
@@ -628,7 +731,7 @@ sv_status_t spec_verify_static(const void* target_logits, const void* draft_logi
     const DeviceInfo* info = device_info(&dev);
     if (!info) return SV_ERR_UNSUPPORTED;
     Plan p;
-    if ((s = make_plan(*info, cl.seqs, cl.k, cl.V, cl.dt, cl.greedy, cl.top_k, opts, &p)) != SV_OK) return s;
+    if ((s = make_plan(*info, cl.seqs, cl.k, cl.V, cl.dt, cl.greedy, cl.top_k, opts, cl.nprocs, &p)) != SV_OK) return s;
     if (p.ws_bytes > SV_STATIC_WORKSPACE_BYTES) return SV_ERR_UNSUPPORTED;  // beyond the static buffer
     void* ws = static_scratch(dev);
     if (!ws) return SV_ERR_CUDA;

@@ -49,6 +49,7 @@ struct Cand {
     int i;
 };
 
+
 // A final draw handed from the per-sequence kernel to the segment kernel
 // (64 bytes): weights w(v) = max(0, p(v) - q(v)) over the row pair of position
 // j, or p(v) alone, with p(v) = [z_t(v) >= t_tau] 2^(z_t(v)*c - t_msc) * t_invS

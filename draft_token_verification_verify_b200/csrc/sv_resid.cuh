@@ -13,6 +13,7 @@
 #pragma once
 
 #include "sv_common.cuh"
+#include "sv_procs.cuh"
 
 namespace sv {
 
@@ -31,10 +32,16 @@ struct ResidParams {
     int* counter;         // [B], zeroed by the per-sequence kernel
     int32_t* out_tokens;  // [B][k+1]
     int32_t* out_n;       // [B]
+    // processors (mask, repetition penalty) or null
+    const uint32_t* allow;
+    const uint32_t* pen;
+    const float* theta;
+    int W4;
 };
 
 template <int DT>
-__device__ __forceinline__ void res_load_vec(const void* row, bool aligned, int q, int V, float* v) {
+__device__ __forceinline__ void res_load_vec(const void* row, bool aligned, int q, int V, float* v,
+                                             const ProcView& pv) {
     constexpr int VEC = VT<DT>::VEC;
     const long long e = static_cast<long long>(q) * VEC;
     if (aligned && e + VEC <= V) {
@@ -42,6 +49,11 @@ __device__ __forceinline__ void res_load_vec(const void* row, bool aligned, int 
     } else {
 #pragma unroll
         for (int t = 0; t < VEC; ++t) v[t] = (e + t < V) ? load_elem<DT>(row, e + t) : NEG_INF;
+    }
+    if (pv.allow) {
+#pragma unroll
+        for (int t = 0; t < VEC; ++t)
+            if (e + t < V) v[t] = proc_logit(v[t], e + t, pv);
     }
 }
 
@@ -62,6 +74,7 @@ __global__ void __launch_bounds__(RES_NT) sv_resid_kernel(const ResidParams P) {
     if (!R.need) return;
 
     const int V = P.V;
+    const ProcView pv = proc_view(P.allow, P.pen, P.theta, P.W4, b);
     const void* rowt = static_cast<const char*>(P.target) + static_cast<size_t>(R.rowt) * V * ELT;
     const void* rowd = static_cast<const char*>(P.draft) + static_cast<size_t>(R.rowd) * V * ELT;
     const bool alt = (reinterpret_cast<uintptr_t>(rowt) & 15u) == 0;
@@ -70,8 +83,8 @@ __global__ void __launch_bounds__(RES_NT) sv_resid_kernel(const ResidParams P) {
     const int nvec = (V + VEC - 1) / VEC;
     auto weights = [&](int q, bool use_q, float* w) {
         float vt[VEC], vd[VEC];
-        res_load_vec<DT>(rowt, alt, q, V, vt);
-        if (use_q) res_load_vec<DT>(rowd, ald, q, V, vd);
+        res_load_vec<DT>(rowt, alt, q, V, vt, pv);
+        if (use_q) res_load_vec<DT>(rowd, ald, q, V, vd, pv);
 #pragma unroll
         for (int t = 0; t < VEC; ++t) {
             const float pt = (vt[t] >= R.t_tau) ? ex2(fmaf(vt[t], R.c, -R.t_msc)) * R.t_invS : 0.f;
@@ -89,8 +102,8 @@ __global__ void __launch_bounds__(RES_NT) sv_resid_kernel(const ResidParams P) {
         float ar = 0.f, ap = 0.f;
         for (int q = s * vps + tid; q < min(nvec, (s + 1) * vps); q += RES_NT) {
             float vt[VEC], vd[VEC];
-            res_load_vec<DT>(rowt, alt, q, V, vt);
-            if (R.use_q) res_load_vec<DT>(rowd, ald, q, V, vd);
+            res_load_vec<DT>(rowt, alt, q, V, vt, pv);
+            if (R.use_q) res_load_vec<DT>(rowd, ald, q, V, vd, pv);
 #pragma unroll
             for (int t = 0; t < VEC; ++t) {
                 const float pt = (vt[t] >= R.t_tau) ? ex2(fmaf(vt[t], R.c, -R.t_msc)) * R.t_invS : 0.f;

@@ -21,31 +21,36 @@
 //            Warp w publishes a value b_w such that at least rsel =
 //            ceil(K / NW) distinct vectors it has seen have a maximum >= b_w
 //            (the rsel-th largest of its lanes' running maxima, or the
-//            rsel-th largest entry of its own candidate list).  Then at least
+//            rsel-th largest key of its own candidate list).  Then at least
 //            NW * rsel >= K vector maxima are >= min_w b_w, so that minimum
-//            never exceeds the K-th largest vector maximum tau_v — whatever mix
-//            of older and newer published values a warp reads — and vectors
-//            whose maximum reaches it go to the warp's private list (one
-//            ballot per vector slot, no per-element work).  At the end tau_v is
-//            taken exactly from the list; the chunk's K-th largest logit is
-//            >= tau_v and every element >= it lies in a vector whose maximum
-//            is >= tau_v, so only those ~K vectors are read again (from L2 or
-//            HBM) and expanded to elements.
+//            never exceeds the K-th largest vector maximum — whatever mix of
+//            older and newer published values a warp reads — and vectors
+//            whose maximum reaches it are copied, whole, into the warp's
+//            private list in shared memory (one ballot per vector slot, no
+//            per-element work).  A consumer hands its stage back as soon as
+//            the maxima are taken and the candidates copied; publishing the
+//            bounds works on registers only and overlaps the next copy.  At
+//            the end the listed vectors are expanded to their elements >= the
+//            final bound (the chunk's K-th largest logit is >= it, and every
+//            element >= that lies in a listed vector), and the exact
+//            threshold and kept entries are taken from those few elements.
 // Rows are read from HBM exactly once; no CTA waits for another.
 #pragma once
 
 #include <climits>
 
 #include "sv_common.cuh"
+#include "sv_procs.cuh"
 
 namespace sv {
 
 constexpr int MAX_STAGES = 8;
 constexpr int MAX_TILES_K1 = 64;   // segments per chunk
-constexpr int RANK_MAX = 256;      // expanded top-k elements ranked per chunk (more: exact fallback)
 constexpr int TILE_BYTES = 16384;  // bytes per segment (one ring stage)
 constexpr int REC_DIAG = 4;        // a device-side consistency check failed
+constexpr int RANK_MAX = 256;      // expanded top-k elements ranked per chunk (more: exact fallback)
 constexpr int MAX_CONSUMER_WARPS = 16;
+constexpr int TOPK_WCAP = 256;     // candidate vectors per consumer warp (top-k)
 
 struct RowsParams {
     const void* target;          // [B][k+1][V] (sampler: [rows][V])
@@ -60,27 +65,35 @@ struct RowsParams {
     int spc;                     // segments per chunk (<= MAX_TILES_K1)
     int nch;                     // chunks per row
     int stages;                  // ring stages (2..MAX_STAGES)
-    int lcap;                    // top-k candidate entries per CTA (NW segments)
-    int kcap;                    // stored kept entries per chunk
+    int lcap;                    // top-k candidate vectors per CTA (NW segments of TOPK_WCAP)
+    int kcap;                    // stored kept entries per chunk (top-k)
     SegRec* segs;                // [R][nseg]
-    ChunkRec* chunks;            // [R][nch]
-    Cand* cands;                 // [R][nch][kcap]
+    ChunkRec* chunks;            // [R][nch] (top-k)
+    Cand* cands;                 // [R][nch][kcap] (top-k)
     int32_t* out_status;         // reset to 0 by CTA 0 (or null)
     unsigned long long timeout_ns;
     unsigned int test_extra_tx;
+    // processors (the PROC variants): per-sequence bitmaps built by K0
+    const uint32_t* allow;       // [S][W4]
+    const uint32_t* pen;         // [S][W4]
+    const float* theta;          // [S] or null
+    int W4;
+    int procs_div;               // the processors' sequence of row-owner b is b / procs_div
 };
 
 struct __align__(16) RowsCtl {
     uint64_t full[MAX_STAGES];
     uint64_t empty[MAX_STAGES];
     int issued;   // tiles the producer issued
+    int copied;   // bit q: the last issue into stage q carried a bulk copy
     int tmo;      // a wait ran out
+    int rawbad;   // a raw logit is NaN or +inf (processors: the row is an error even if masked)
     int diag;     // a copy failed its self-check (skipped)
     int cnt2;
     int nkept;
     float tau;
     int ne;     // expanded elements (top-k)
-    float tauv; // K-th largest candidate-vector maximum (top-k)
+    float thf;  // K-th largest candidate-vector maximum (top-k finish)
     float wbound[MAX_CONSUMER_WARPS];  // published per-warp bounds (top-k)
     float wmax[MAX_CONSUMER_WARPS];
     float wbest[MAX_CONSUMER_WARPS];
@@ -93,12 +106,15 @@ struct __align__(16) RowsCtl {
 
 constexpr int ROWS_CTL_BYTES = (int)((sizeof(RowsCtl) + 127) / 128 * 128);
 constexpr int STAGE_BYTES = (TILE_BYTES + 32 + 127) / 128 * 128;  // one segment plus one spare vector
+// processors: each stage also holds the segment's allow and penalty bitmap words
+constexpr int MASK_STAGE_BYTES = (TILE_BYTES / 2 / 32 * 4 + 32 + 127) / 128 * 128;
+constexpr int STAGE_BYTES_PROC = STAGE_BYTES + 2 * MASK_STAGE_BYTES;
 
 // Dynamic shared memory of one streaming CTA.
-__host__ __device__ constexpr int rows_smem_bytes(int mode, int nt, int stages, int lcap) {
-    return ROWS_CTL_BYTES + stages * STAGE_BYTES +
+__host__ __device__ constexpr int rows_smem_bytes(int mode, int nt, int stages, int lcap, bool proc) {
+    return ROWS_CTL_BYTES + stages * (proc ? STAGE_BYTES_PROC : STAGE_BYTES) +
            (mode == MODE_SOFTMAX ? 2 * MAX_TILES_K1 * (nt / 32) * 4 : 0) +
-           (mode == MODE_TOPK ? lcap * 8 : 0);
+           (mode == MODE_TOPK ? lcap * (4 + 4) : 0);
 }
 
 // Geometry of one segment in the ring: the stage mirrors the 16-byte aligned
@@ -139,37 +155,16 @@ __device__ __forceinline__ void consumer_sync() {
     asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory");
 }
 
-// Sort n (<= 32 * 16) (key, index) pairs of one warp's shared segment by key,
-// descending; entries past n are padded by the caller up to the power of two
-// `np2`.  Warp-synchronous.
-__device__ __forceinline__ void warp_sort_desc(float* key, int* idx, int np2, int lane) {
-    for (int size = 2; size <= np2; size <<= 1) {
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            for (int t = lane; t < (np2 >> 1); t += 32) {
-                const int lo = 2 * stride * (t / stride) + (t % stride);
-                const int hi = lo + stride;
-                const bool up = (lo & size) == 0;
-                const float ka = key[lo], kb = key[hi];
-                if (up ? (kb > ka) : (ka > kb)) {
-                    const int ia = idx[lo];
-                    key[lo] = kb;
-                    key[hi] = ka;
-                    idx[lo] = idx[hi];
-                    idx[hi] = ia;
-                }
-            }
-            __syncwarp();
-        }
-    }
-}
-
-template <int NT>
+template <int NT, int MODE>
 struct RowsOcc {  // CTAs per SM the register budget is sized for
-    static constexpr int value = NT <= 128 ? 6 : (NT <= 256 ? 4 : 2);
+    // top-k CTAs hold their candidate lists in shared memory, which caps them
+    // at 4 / 3 / 2 per SM; the other modes fit 6 / 4 / 2
+    static constexpr int value = MODE == MODE_TOPK ? (NT <= 128 ? 4 : (NT <= 256 ? 3 : 2))
+                                                   : (NT <= 128 ? 6 : (NT <= 256 ? 4 : 2));
 };
 
-template <int DT, int NT, int MODE>
-__global__ void __launch_bounds__(NT + 32, RowsOcc<NT>::value) sv_rows_kernel(const RowsParams P) {
+template <int DT, int NT, int MODE, bool PROC>
+__global__ void __launch_bounds__(NT + 32, RowsOcc<NT, MODE>::value) sv_rows_kernel(const RowsParams P) {
     constexpr int ELT = VT<DT>::ELT;
     constexpr int VEC = VT<DT>::VEC;
     constexpr int NW = NT / 32;             // consumer warps; warp NW is the producer
@@ -177,17 +172,19 @@ __global__ void __launch_bounds__(NT + 32, RowsOcc<NT>::value) sv_rows_kernel(co
     constexpr int TV = TILE_BYTES / 16;     // vectors per tile
     constexpr int VPT = TV / NT;            // vectors per consumer thread per tile
     constexpr int SEG = TILE_BYTES / ELT;   // elements per segment
+    constexpr int SSTRIDE = PROC ? STAGE_BYTES_PROC : STAGE_BYTES;  // bytes per ring stage
+    constexpr uint32_t VMASK = (1u << VEC) - 1u;
     static_assert(VPT * NT == TV, "tile must split evenly over the consumer threads");
+    static_assert(!PROC || MODE != MODE_GREEDY, "greedy verification takes no processors");
     static_assert(NW <= MAX_CONSUMER_WARPS, "too many consumer warps");
-    static_assert(VPT * VEC <= 64, "candidate mask");
     extern __shared__ __align__(128) unsigned char smem[];
     RowsCtl& S = *reinterpret_cast<RowsCtl*>(smem);
     unsigned char* const ring = smem + ROWS_CTL_BYTES;
-    unsigned char* const tail = ring + static_cast<size_t>(P.stages) * STAGE_BYTES;
-    float* const red_m = reinterpret_cast<float*>(tail);      // softmax: [MAX_TILES_K1][NW]
+    unsigned char* const tail = ring + static_cast<size_t>(P.stages) * SSTRIDE;
+    float* const red_m = reinterpret_cast<float*>(tail);          // softmax: [MAX_TILES_K1][NW]
     float* const red_s = red_m + MAX_TILES_K1 * NW;
-    float* const lkey = reinterpret_cast<float*>(tail);       // top-k: [lcap]
-    int* const lidx = reinterpret_cast<int*>(lkey + P.lcap);  //        [lcap]
+    float* const lkey = reinterpret_cast<float*>(tail);           // top-k: [lcap] candidate-vector maxima
+    int* const lidx = reinterpret_cast<int*>(lkey + P.lcap);      //        [lcap] their place: t*(TV+1) + j
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const long long task = blockIdx.x;
@@ -214,6 +211,14 @@ __global__ void __launch_bounds__(NT + 32, RowsOcc<NT>::value) sv_rows_kernel(co
     if (task == 0 && tid == 0 && P.out_status) *P.out_status = 0;
     pdl_launch_dependents();
 
+    // processors of the row's sequence (PROC only)
+    const long long pseq = PROC ? b / P.procs_div : 0;
+    const float pen_theta = (PROC && P.theta) ? P.theta[pseq] : 1.f;  // repetition penalty
+    const uint32_t* const gallow = PROC ? P.allow + pseq * P.W4 : nullptr;
+    const uint32_t* const gpen = PROC ? P.pen + pseq * P.W4 : nullptr;
+    (void)pen_theta;
+    (void)gallow;
+    (void)gpen;
     float cscale = 1.f;  // log2(e) / T
     if constexpr (MODE == MODE_SOFTMAX || MODE == MODE_TOPK) {
         const float T = P.temperature ? P.temperature[b] : 1.f;
@@ -222,7 +227,7 @@ __global__ void __launch_bounds__(NT + 32, RowsOcc<NT>::value) sv_rows_kernel(co
     const int s0 = c * P.spc;
     const int ntiles = min(P.spc, P.nseg - s0);
     const int K = P.top_k;
-    const int wcap = P.lcap / NW;  // top-k entries per warp segment
+    const int wcap = P.lcap / NW;  // top-k candidate vectors per warp segment
     auto geom = [&](int t) {
         const int lo = (s0 + t) * SEG;
         const int hi = min(P.V, lo + SEG);
@@ -236,7 +241,9 @@ __global__ void __launch_bounds__(NT + 32, RowsOcc<NT>::value) sv_rows_kernel(co
         }
         fence_mbar_init();
         S.issued = 0;
+        S.copied = 0;
         S.tmo = 0;
+        S.rawbad = 0;
         S.diag = 0;
     }
     if (tid < MAX_CONSUMER_WARPS) S.wbound[tid] = NEG_INF;
@@ -245,7 +252,7 @@ __global__ void __launch_bounds__(NT + 32, RowsOcc<NT>::value) sv_rows_kernel(co
     if (warp == NW) {
         // ================= producer: lane 0 fills the ring =================
         if (lane == 0) {
-            int t = 0;
+            int t = 0, copied = 0;
             for (; t < ntiles; ++t) {
                 const int st = t % P.stages;
                 if (*reinterpret_cast<volatile int*>(&S.tmo)) break;
@@ -255,7 +262,7 @@ __global__ void __launch_bounds__(NT + 32, RowsOcc<NT>::value) sv_rows_kernel(co
                     break;
                 }
                 const TileGeom g = geom(t);
-                unsigned char* buf = ring + static_cast<size_t>(st) * STAGE_BYTES;
+                unsigned char* buf = ring + static_cast<size_t>(st) * SSTRIDE;
                 uint32_t bytes = 0;
                 int nh = 0, ntl = 0;
                 if (g.hi > g.lo) {
@@ -276,6 +283,28 @@ __global__ void __launch_bounds__(NT + 32, RowsOcc<NT>::value) sv_rows_kernel(co
                     bytes = 0;
                     nh = ntl = 0;
                 }
+                // processors: the segment's bitmap words, a 16-byte aligned span
+                // (rows padded to a multiple of 4 words, segments start at a
+                // multiple of 128 elements) of whole words covering [lo, hi)
+                uint32_t mbytes = 0;
+                const uint32_t* asrc = nullptr;
+                const uint32_t* psrc = nullptr;
+                if constexpr (PROC) {
+                    if (g.hi > g.lo) {
+                        mbytes = static_cast<uint32_t>(((g.hi - g.lo + 127) / 128) * 16);
+                        asrc = gallow + g.lo / 32;
+                        psrc = gpen + g.lo / 32;
+                        if (((reinterpret_cast<uintptr_t>(asrc) | reinterpret_cast<uintptr_t>(psrc) | mbytes) & 15u) != 0 ||
+                            mbytes > static_cast<uint32_t>(MASK_STAGE_BYTES - 32) || g.lo % 128 != 0 ||
+                            g.lo / 32 + static_cast<int>(mbytes / 4) > P.W4) {
+                            atomicOr(&S.diag, 1);
+                            mbytes = 0;
+                        }
+                    }
+                }
+                // Test hook: the stage expects test_extra_tx bytes that no copy
+                // delivers (no bulk copy is issued), so its wait runs out.
+                if (P.test_extra_tx) bytes = mbytes = 0;
                 // elements outside the aligned interior: plain loads, published by the arrive
                 for (int q = 0; q < nh + ntl; ++q) {
                     const int e = q < nh ? g.lo + q : g.hi - ntl + (q - nh);
@@ -284,24 +313,32 @@ __global__ void __launch_bounds__(NT + 32, RowsOcc<NT>::value) sv_rows_kernel(co
                     else
                         reinterpret_cast<float*>(buf)[e - g.e0] = reinterpret_cast<const float*>(row)[e];
                 }
-                mbar_arrive_expect_tx(&S.full[st], bytes + P.test_extra_tx);
+                mbar_arrive_expect_tx(&S.full[st], bytes + 2 * mbytes + P.test_extra_tx);
                 if (bytes) bulk_g2s(buf + doff, reinterpret_cast<const void*>(g.ga16), bytes, &S.full[st]);
+                if (mbytes) {
+                    bulk_g2s(buf + STAGE_BYTES, asrc, mbytes, &S.full[st]);
+                    bulk_g2s(buf + STAGE_BYTES + MASK_STAGE_BYTES, psrc, mbytes, &S.full[st]);
+                }
+                copied = (bytes | mbytes) ? (copied | (1 << st)) : (copied & ~(1 << st));
             }
             S.issued = t;
+            S.copied = copied;
         }
         __syncwarp();
     } else {
         // ================= consumers =================
-        float run = NEG_INF;    // running NaN-propagating maximum of this thread's elements
+        float run = NEG_INF;    // running NaN-propagating maximum of this thread's (processed) elements
+        bool rawbad = false;    // processors: a raw NaN or +inf was seen
         float wbest = NEG_INF;  // greedy: best value of this warp and its lowest index
         int widx = -1;
         const int rsel = (K + NW - 1) / NW;  // <= 32 on the top-k path (K <= NT)
         float* const wkey = lkey + warp * wcap;
         int* const widxs = lidx + warp * wcap;
-        int wcnt = 0;       // entries in this warp's segment (warp-uniform)
-        bool wovf = false;  // the segment lost entries
+        int wcnt = 0;       // vectors in this warp's segment (warp-uniform)
+        bool wovf = false;  // the segment lost vectors (massive ties at the bound)
         float theta = NEG_INF;
         float pub = NEG_INF;  // this warp's last published bound
+
         // rsel-th largest of the lanes' running maxima
         auto lane_bound = [&]() -> float {
             float x = run == run ? run : NEG_INF;
@@ -329,30 +366,57 @@ __global__ void __launch_bounds__(NT + 32, RowsOcc<NT>::value) sv_rows_kernel(co
             for (int w = 1; w < NW; ++w) mn = fminf(mn, *reinterpret_cast<volatile float*>(&S.wbound[w]));
             return mn;
         };
-        // Segment full: sort it, publish its rsel-th largest entry, keep the
-        // entries >= the freshest bound.
+        // Segment full: publish its rsel-th largest key (rank counting), raise
+        // theta to the freshest bound and keep, in order, the vectors >= theta.
         auto compact = [&]() {
-            const int np2 = pow2_ceil(wcnt < 2 ? 2 : wcnt);
-            for (int q = wcnt + lane; q < np2; q += 32) {
-                wkey[q] = NEG_INF;
-                widxs[q] = INT_MAX;
+            float sel = NEG_INF;
+            for (int q0 = 0; q0 < wcnt; q0 += 32) {
+                const int q = q0 + lane;
+                if (q < wcnt) {
+                    const float x = wkey[q];
+                    int gt = 0, ge = 0;
+                    for (int f = 0; f < wcnt; ++f) {
+                        const float y = wkey[f];
+                        gt += y > x;
+                        ge += y >= x;
+                    }
+                    if (gt < rsel && rsel <= ge) sel = x;
+                }
             }
-            __syncwarp();
-            warp_sort_desc(wkey, widxs, np2, lane);
-            if (wcnt >= rsel) publish(wkey[rsel - 1]);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) sel = fmaxf(sel, __shfl_xor_sync(0xffffffffu, sel, o));
+            if (wcnt >= rsel) publish(sel);
             theta = fmaxf(theta, read_bound());
             int keep = 0;
             for (int q0 = 0; q0 < wcnt; q0 += 32) {
-                const bool ge = q0 + lane < wcnt && wkey[q0 + lane] >= theta;
-                keep += __popc(__ballot_sync(0xffffffffu, ge));
+                const int q = q0 + lane;
+                const bool in = q < wcnt;
+                float x = NEG_INF;
+                int ix = 0;
+                if (in) {
+                    x = wkey[q];
+                    ix = widxs[q];
+                }
+                const bool ge = in && x >= theta;
+                const unsigned m = __ballot_sync(0xffffffffu, ge);
+                __syncwarp();
+                if (ge) {
+                    const int d = keep + __popc(m & ((1u << lane) - 1u));
+                    wkey[d] = x;
+                    widxs[d] = ix;
+                }
+                keep += __popc(m);
+                __syncwarp();
             }
-            wcnt = keep;  // sorted descending: the kept entries are the prefix
+            wcnt = keep;
         };
 
         for (int t = 0; t < ntiles; ++t) {
             const int st = t % P.stages;
             const TileGeom g = geom(t);
-            const unsigned char* buf = ring + static_cast<size_t>(st) * STAGE_BYTES;
+            const unsigned char* buf = ring + static_cast<size_t>(st) * SSTRIDE;
+            const uint32_t* const sallow = reinterpret_cast<const uint32_t*>(buf + STAGE_BYTES);
+            const uint32_t* const spen = reinterpret_cast<const uint32_t*>(buf + STAGE_BYTES + MASK_STAGE_BYTES);
             const bool ok = mbar_wait_bounded(&S.full[st], static_cast<uint32_t>((t / P.stages) & 1), P.timeout_ns);
             if (!ok && lane == 0) atomicOr(&S.tmo, 1);
             auto valid = [&](int e) { return e >= g.lo && e < g.hi; };
@@ -378,13 +442,58 @@ __global__ void __launch_bounds__(NT + 32, RowsOcc<NT>::value) sv_rows_kernel(co
                         if (!valid(e + q)) v[q] = NEG_INF;
                 }
             };
+            // PROC: the VEC allow or penalty bits of elements e .. e+VEC-1;
+            // positions before the segment read as `ones` (validity masks them)
+            auto bits_at = [&](const uint32_t* M, int e, bool ones) -> uint32_t {
+                const int rr = e - g.lo;
+                uint32_t x;
+                if (rr >= 0)
+                    x = __funnelshift_r(M[rr >> 5], M[(rr >> 5) + 1], rr & 31);
+                else
+                    x = (M[0] << (-rr)) | (ones ? ((1u << (-rr)) - 1u) : 0u);
+                return x & VMASK;
+            };
+            // PROC: processed values of the vector at `raw` (first element e),
+            // -inf outside the segment
+            auto proc_vals = [&](const uint4& raw, int e, float* v) {
+                unpack<DT>(raw, v);
+                const uint32_t ab = bits_at(sallow, e, true), pb = bits_at(spen, e, false);
+#pragma unroll
+                for (int q = 0; q < VEC; ++q) {
+                    if (!valid(e + q) || !((ab >> q) & 1u))
+                        v[q] = NEG_INF;
+                    else if ((pb >> q) & 1u)
+                        v[q] = penalise(v[q], pen_theta);
+                }
+            };
+            // PROC: processed maximum of vector j (raw errors noted on the way)
+            auto proc_vmax = [&](int j) -> float {
+                const uint4 raw = vec_at(j);
+                const int e = g.e0 + j * VEC;
+                const bool full = e >= g.lo && e + VEC <= g.hi;
+                const float rm = full ? vmax_nan<DT>(raw) : vmax_masked(j);
+                if (!(rm == rm) || rm == POS_INF) rawbad = true;
+                if (full && bits_at(sallow, e, true) == VMASK && bits_at(spen, e, false) == 0u) return rm;
+                float v[VEC];
+                proc_vals(raw, e, v);
+                float m = NEG_INF;
+#pragma unroll
+                for (int q = 0; q < VEC; ++q) m = fmax_nan(m, v[q]);
+                return m;
+            };
             // this thread's vectors: slot i < VPT is vector tid + i*NT; slot VPT
             // is the one vector past TV that a segment starting off a 16-byte
             // boundary spans (vector TV + tid, tid == 0 only)
             auto jof = [&](int i) { return i < VPT ? tid + i * NT : TV + tid; };
             float vm[VPT + 1];
             const bool tile_full = ok && g.e0 == g.lo && g.nvec == TV && g.hi - g.lo == TV * VEC;
-            if (tile_full) {
+            if constexpr (PROC) {
+#pragma unroll
+                for (int i = 0; i <= VPT; ++i) {
+                    const int j = jof(i);
+                    vm[i] = (ok && j < g.nvec) ? proc_vmax(j) : NEG_INF;
+                }
+            } else if (tile_full) {
 #pragma unroll
                 for (int i = 0; i < VPT; ++i) vm[i] = vmax_nan<DT>(vec_at(tid + i * NT));
                 vm[VPT] = NEG_INF;
@@ -398,6 +507,7 @@ __global__ void __launch_bounds__(NT + 32, RowsOcc<NT>::value) sv_rows_kernel(co
             float tm = vm[0];
 #pragma unroll
             for (int i = 1; i <= VPT; ++i) tm = fmax_nan(tm, vm[i]);
+            bool held = true;  // this warp still holds the stage
 
             if constexpr (MODE == MODE_GREEDY) {
                 run = fmax_nan(run, tm);
@@ -436,7 +546,10 @@ __global__ void __launch_bounds__(NT + 32, RowsOcc<NT>::value) sv_rows_kernel(co
                         const int j = jof(i);
                         if (j < g.nvec) {
                             float v[VEC];
-                            load_masked(j, v);
+                            if constexpr (PROC)
+                                proc_vals(vec_at(j), g.e0 + j * VEC, v);
+                            else
+                                load_masked(j, v);
 #pragma unroll
                             for (int q = 0; q < VEC; q += 2) {
                                 sa += ex2(fmaf(v[q], cscale, -m));
@@ -452,6 +565,11 @@ __global__ void __launch_bounds__(NT + 32, RowsOcc<NT>::value) sv_rows_kernel(co
                 }
             } else if constexpr (MODE == MODE_TOPK) {
                 run = fmax_nan(run, tm);
+                // hand the stage back at once: the bookkeeping below reads the
+                // maxima in registers and the warp's list only
+                __syncwarp();
+                if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&S.empty[st])) : "memory");
+                held = false;
                 if (t == 0) {
                     // every warp publishes a bound from the first tile before any append
                     publish(lane_bound());
@@ -460,42 +578,66 @@ __global__ void __launch_bounds__(NT + 32, RowsOcc<NT>::value) sv_rows_kernel(co
                     publish(lane_bound());
                 }
                 theta = fmaxf(theta, read_bound());
-                // Candidate vectors: finite maximum at or above the bound.  A
-                // vector's maximum is one of its elements, so distinct vectors
-                // give distinct elements for the bounds.
-                int mine = 0;
+                // Candidate vectors (finite maximum at or above the bound) go
+                // to the warp's list as (maximum, place in the chunk).
+                unsigned cm = 0u;  // bit i: slot i holds a candidate
+                if (!wovf) {
 #pragma unroll
-                for (int i = 0; i <= VPT; ++i) mine += (ok && vm[i] > NEG_INF && vm[i] >= theta) ? 1 : 0;
-                const int total = __reduce_add_sync(0xffffffffu, mine);
-                if (total) {
-                    if (wcnt + total > wcap && !wovf) compact();  // raises theta
+                    for (int i = 0; i <= VPT; ++i)
+                        if (ok && vm[i] > NEG_INF && vm[i] >= theta) cm |= 1u << i;
+                    // each lane's candidates go to consecutive list entries: an
+                    // exclusive prefix sum of the lanes' counts gives the offsets
+                    int cnt = __popc(cm), incl = cnt;
 #pragma unroll
-                    for (int i = 0; i <= VPT; ++i) {
-                        const bool cnd = ok && vm[i] > NEG_INF && vm[i] >= theta;
-                        const unsigned m = __ballot_sync(0xffffffffu, cnd);
-                        if (m) {
-                            const int p = wcnt + __popc(m & ((1u << lane) - 1u));
-                            if (cnd && p < wcap) {
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                        if (lane >= o) incl += y;
+                    }
+                    int total = __shfl_sync(0xffffffffu, incl, 31);
+                    if (total && wcnt + total > wcap) {
+                        compact();  // raises theta
+#pragma unroll
+                        for (int i = 0; i <= VPT; ++i)
+                            if (!(vm[i] >= theta)) cm &= ~(1u << i);
+                        cnt = __popc(cm);
+                        incl = cnt;
+#pragma unroll
+                        for (int o = 1; o < 32; o <<= 1) {
+                            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                            if (lane >= o) incl += y;
+                        }
+                        total = __shfl_sync(0xffffffffu, incl, 31);
+                        if (wcnt + total > wcap) wovf = true;  // massive ties: exact fallback downstream
+                    }
+                    if (total && !wovf) {
+                        int p = wcnt + incl - cnt;
+#pragma unroll
+                        for (int i = 0; i <= VPT; ++i) {
+                            if ((cm >> i) & 1u) {
                                 wkey[p] = vm[i];
                                 widxs[p] = t * (TV + 1) + jof(i);
+                                ++p;
                             }
-                            const int n = __popc(m);
-                            if (wcnt + n > wcap) wovf = true;
-                            wcnt = min(wcnt + n, wcap);
                         }
+                        wcnt += total;
                     }
                 }
             } else {
                 run = fmax_nan(run, tm);  // MODE_MAXONLY
             }
 
-            // hand the stage back to the producer
-            __syncwarp();
-            if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&S.empty[st])) : "memory");
+            if (held) {
+                // hand the stage back to the producer
+                __syncwarp();
+                if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&S.empty[st])) : "memory");
+            }
             if (!ok) break;
         }
 
         // ---- per-warp results ------------------------------------------------------
+        if constexpr (PROC) {
+            if (__any_sync(0xffffffffu, rawbad) && lane == 0) atomicOr(&S.rawbad, 1);
+        }
         if constexpr (MODE != MODE_SOFTMAX) {
             const float wm = warp_max_nan(run);
             if (lane == 0) {
@@ -516,6 +658,7 @@ __global__ void __launch_bounds__(NT + 32, RowsOcc<NT>::value) sv_rows_kernel(co
 
     const int tmo = S.tmo;
     const int diag = S.diag;
+    const bool rawerr = PROC && S.rawbad;  // the row is an error: its records carry NaN
     const int bad = tmo | diag;
     const int flag = (tmo ? REC_TIMEOUT : 0) | (diag ? REC_DIAG : 0);
 
@@ -531,7 +674,7 @@ __global__ void __launch_bounds__(NT + 32, RowsOcc<NT>::value) sv_rows_kernel(co
             } else {
                 float m = red_m[q * NW], sm = red_s[q * NW];
                 for (int w = 1; w < NW; ++w) ms_combine(m, sm, red_m[q * NW + w], red_s[q * NW + w]);
-                rec.m = m;
+                rec.m = rawerr ? __int_as_float(0x7fc00000) : m;
                 rec.s = sm;
             }
             P.segs[r * P.nseg + s0 + q] = rec;
@@ -552,7 +695,7 @@ __global__ void __launch_bounds__(NT + 32, RowsOcc<NT>::value) sv_rows_kernel(co
             }
             rec.arg = MODE == MODE_GREEDY ? bi : -1;
             rec.flags = flag;
-            if (bad) rec.m = __int_as_float(0x7fc00000);
+            if (bad || rawerr) rec.m = __int_as_float(0x7fc00000);
             P.segs[r * P.nseg + c] = rec;
         }
     }
@@ -571,9 +714,11 @@ __global__ void __launch_bounds__(NT + 32, RowsOcc<NT>::value) sv_rows_kernel(co
                 ch.pad = 0;
                 P.chunks[r * P.nch + c] = ch;
             }
-            // wait (bounded) for the last copy issued into each stage
-            const int issued = S.issued;
+            // wait (bounded) for the last bulk copy issued into each stage, so
+            // that no copy is still writing this CTA's shared memory at exit
+            const int issued = S.issued, copied = S.copied;
             for (int q = 0; q < min(issued, P.stages); ++q) {
+                if (!((copied >> q) & 1)) continue;
                 const int last = q + ((issued - 1 - q) / P.stages) * P.stages;
                 mbar_wait_bounded(&S.full[q], static_cast<uint32_t>((last / P.stages) & 1), P.timeout_ns);
             }
@@ -590,6 +735,7 @@ __global__ void __launch_bounds__(NT + 32, RowsOcc<NT>::value) sv_rows_kernel(co
             thf = fminf(thf, S.wbound[w]);
             ovf |= S.wovf[w];
         }
+        if (rawerr) cmax = __int_as_float(0x7fc00000);
         const int d = (pos < P.k && P.draft_tokens) ? P.draft_tokens[b * P.k + pos] : -1;
         Cand* fl = reinterpret_cast<Cand*>(ring);  // candidate vectors (the ring is free now)
         const int fcap = (P.stages * STAGE_BYTES) / static_cast<int>(sizeof(Cand));
@@ -600,7 +746,7 @@ __global__ void __launch_bounds__(NT + 32, RowsOcc<NT>::value) sv_rows_kernel(co
             S.ne = 0;
             S.nkept = 0;
             S.tau = NEG_INF;
-            S.tauv = NEG_INF;
+            S.thf = NEG_INF;
         }
         __syncthreads();
         // 1. candidate vectors whose maximum reaches the final bound
@@ -633,10 +779,10 @@ __global__ void __launch_bounds__(NT + 32, RowsOcc<NT>::value) sv_rows_kernel(co
                 gt += y > x;
                 ge += y >= x;
             }
-            if (gt < K && K <= ge) S.tauv = x;
+            if (gt < K && K <= ge) S.thf = x;
         }
         __syncthreads();
-        const float tauv = S.tauv;  // -inf: fewer than K candidate vectors (all are expanded)
+        const float tauv = S.thf;  // -inf: fewer than K candidate vectors (all are expanded)
         // 3. the elements >= tau_v of those vectors, read again from the row
         for (int q = tid; q < nv; q += NTH) {
             const Cand cv = fl[q];
@@ -650,6 +796,15 @@ __global__ void __launch_bounds__(NT + 32, RowsOcc<NT>::value) sv_rows_kernel(co
             } else {
 #pragma unroll
                 for (int u = 0; u < VEC; ++u) v[u] = (e + u >= g.lo && e + u < g.hi) ? load_elem<DT>(row, e + u) : NEG_INF;
+            }
+            if constexpr (PROC) {
+                ProcView pv;
+                pv.allow = gallow;
+                pv.pen = gpen;
+                pv.theta = pen_theta;
+#pragma unroll
+                for (int u = 0; u < VEC; ++u)
+                    if (e + u >= g.lo && e + u < g.hi) v[u] = proc_logit(v[u], e + u, pv);
             }
 #pragma unroll
             for (int u = 0; u < VEC; ++u) {

@@ -25,6 +25,7 @@
 #include <climits>
 
 #include "sv_common.cuh"
+#include "sv_procs.cuh"
 
 namespace sv {
 
@@ -46,8 +47,8 @@ struct SeqParams {
     int seg, nseg, spc, nch, kcap;
     int mg;                      // gather capacity per warp (power of two)
     const SegRec* segs;
-    const ChunkRec* chunks;
-    const Cand* cands;
+    const ChunkRec* chunks;      // [R][nch] top-k: per-chunk record
+    const Cand* cands;           // [R][nch][kcap] top-k: per-chunk kept list, index order
     int32_t* out_tokens;         // [B][k+1] (sampler: [B])
     int32_t* out_n;              // [B] or null (sampler)
     float* out_p;                // [B][k] or null
@@ -60,6 +61,12 @@ struct SeqParams {
     const float* top_p;          // [B] nucleus thresholds (top-k path only) or null
     DrawReq* req;                // [B] when defer
     int* counter;                // [B] when defer: zeroed here for the segment kernel
+    // processors (mask, repetition penalty): bitmaps built by K0, or null
+    const uint32_t* allow;       // [S][W4]
+    const uint32_t* pen;         // [S][W4]
+    const float* theta;          // [S] or null
+    int W4;
+    int procs_div;               // sequence of the processors (and top_p) of b: b / procs_div
 };
 
 struct RowStat {
@@ -137,7 +144,10 @@ __global__ void __launch_bounds__(SEQ_NT, 3) sv_seq_kernel(const SeqParams P) {
     // ---- inputs that do not depend on the streaming pass -----------------------
     float T = 1.f;
     if (!greedy && P.temperature) T = P.temperature[b];
-    const float tp = (!greedy && P.top_p) ? P.top_p[b] : 1.f;  // nucleus threshold
+    const long long pseq = b / P.procs_div;  // the processors' sequence (the sampler groups rows)
+    const float tp = (!greedy && P.top_p) ? P.top_p[pseq] : 1.f;  // nucleus threshold
+    const ProcView pv = proc_view(P.allow, P.pen, P.theta, P.W4, pseq);
+    const float th = pv.theta;  // repetition penalty theta
     const float c = (T > 0.f && T != POS_INF) ? LOG2E / T : 1.f;
     for (int i = tid; i < k; i += NT) dtok[i] = P.draft_tokens[b * k + i];
     if (!greedy)
@@ -154,6 +164,7 @@ __global__ void __launch_bounds__(SEQ_NT, 3) sv_seq_kernel(const SeqParams P) {
         if (!greedy) {
             if (!(T > 0.f) || T == POS_INF) bad = 1;
             if (!(tp > 0.f && tp <= 1.f)) bad = 1;
+            if (pv.allow && !(th > 0.f && th != POS_INF)) bad = 1;
             for (int i = 0; i <= k; ++i)
                 if (!(uu[i] >= 0.f && uu[i] < 1.f)) bad = 1;
         }
@@ -161,6 +172,17 @@ __global__ void __launch_bounds__(SEQ_NT, 3) sv_seq_kernel(const SeqParams P) {
     }
     pdl_launch_dependents();  // the segment kernel may be placed early; it waits for this grid
     pdl_wait_primary();       // the streaming pass is complete from here on
+
+    auto row_ptr = [&](int rr) -> const void* {
+        if (rr <= k)
+            return static_cast<const char*>(P.target) + (static_cast<size_t>(b) * (k + 1) + rr) * static_cast<size_t>(V) * ELT;
+        return static_cast<const char*>(P.draft) + (static_cast<size_t>(b) * k + (rr - k - 1)) * static_cast<size_t>(V) * ELT;
+    };
+    auto row_index = [&](int rr) -> long long { return rr <= k ? b * (k + 1) + rr : Rt + b * k + (rr - k - 1); };
+    auto row_dtok = [&](int rr) -> int {
+        const int pos = rr <= k ? rr : rr - k - 1;
+        return pos < k ? dtok[pos] : -1;
+    };
 
     // top-k, one chunk per row: all of the sequence's chunk records and kept
     // lists in one cooperative round of independent loads
@@ -191,17 +213,6 @@ __global__ void __launch_bounds__(SEQ_NT, 3) sv_seq_kernel(const SeqParams P) {
         }
         __syncthreads();
     }
-
-    auto row_ptr = [&](int rr) -> const void* {
-        if (rr <= k)
-            return static_cast<const char*>(P.target) + (static_cast<size_t>(b) * (k + 1) + rr) * static_cast<size_t>(V) * ELT;
-        return static_cast<const char*>(P.draft) + (static_cast<size_t>(b) * k + (rr - k - 1)) * static_cast<size_t>(V) * ELT;
-    };
-    auto row_index = [&](int rr) -> long long { return rr <= k ? b * (k + 1) + rr : Rt + b * k + (rr - k - 1); };
-    auto row_dtok = [&](int rr) -> int {
-        const int pos = rr <= k ? rr : rr - k - 1;
-        return pos < k ? dtok[pos] : -1;
-    };
 
     // gather the entries >= thr of the row's chunk lists into dst (index order)
     auto gather = [&](long long r, float thr, Cand* dst, int cap) -> int {
@@ -374,7 +385,7 @@ __global__ void __launch_bounds__(SEQ_NT, 3) sv_seq_kernel(const SeqParams P) {
             if (mx != mx || mx == POS_INF || bi < 0) st.err = 1;
         } else if (P.mode == MODE_SOFTMAX) {
             // the draft-token logit load is issued before the partials are combined
-            if (d >= 0 && d < V) st.zd = load_elem<DT>(row_ptr(rr), d);
+            if (d >= 0 && d < V) st.zd = proc_logit(load_elem<DT>(row_ptr(rr), d), d, pv);
             float m = NEG_INF, s = 0.f;
             for (int q = lane; q < P.nseg; q += 32) {
                 const SegRec g = P.segs[r * P.nseg + q];
@@ -522,7 +533,8 @@ __global__ void __launch_bounds__(SEQ_NT, 3) sv_seq_kernel(const SeqParams P) {
         for (int rr = 0; rr < nrows; ++rr) {
             if (!rs[rr].slow || rs[rr].err) continue;  // uniform: read after a barrier
             const void* row = row_ptr(rr);
-            constexpr int ROUNDS = (DT == 0) ? 2 : 4;
+            // bf16 logits have 16-bit keys; penalised ones are fp32 values
+            const int ROUNDS = (DT == 0 && !pv.allow) ? 2 : 4;
             if (tid == 0) {
                 S.radix_prefix = 0u;
                 S.radix_k = K;
@@ -533,7 +545,7 @@ __global__ void __launch_bounds__(SEQ_NT, 3) sv_seq_kernel(const SeqParams P) {
                 __syncthreads();
                 const uint32_t pre = S.radix_prefix;
                 for (int e = tid; e < V; e += NT) {
-                    const uint32_t key = okey(load_elem<DT>(row, e));
+                    const uint32_t key = okey(proc_logit(load_elem<DT>(row, e), e, pv));
                     if (round == 0 || (key >> (shift + 8)) == pre) atomicAdd(&S.hist[(key >> shift) & 255u], 1);
                 }
                 __syncthreads();
@@ -554,14 +566,14 @@ __global__ void __launch_bounds__(SEQ_NT, 3) sv_seq_kernel(const SeqParams P) {
                 __syncthreads();
             }
             float tau;
-            if constexpr (DT == 0)
+            if (ROUNDS == 2)
                 tau = okey_inv(S.radix_prefix << 16 | ((S.radix_prefix & 0x8000u) ? 0u : 0xffffu));
             else
                 tau = okey_inv(S.radix_prefix);
             const float msc = rs[rr].msc;
             float acc = 0.f;
             for (int e = tid; e < V; e += NT) {
-                const float z = load_elem<DT>(row, e);
+                const float z = proc_logit(load_elem<DT>(row, e), e, pv);
                 if (z >= tau) acc += ex2(fmaf(z, c, -msc));
             }
             acc = warp_sum(acc);
@@ -573,7 +585,7 @@ __global__ void __launch_bounds__(SEQ_NT, 3) sv_seq_kernel(const SeqParams P) {
                 rs[rr].tau = tau;
                 rs[rr].invS = 1.f / s;
                 const int d = row_dtok(rr);
-                rs[rr].zd = (d >= 0 && d < V) ? load_elem<DT>(row, d) : __int_as_float(0x7fc00000);
+                rs[rr].zd = (d >= 0 && d < V) ? proc_logit(load_elem<DT>(row, d), d, pv) : __int_as_float(0x7fc00000);
             }
             __syncthreads();
         }
@@ -758,6 +770,16 @@ __global__ void __launch_bounds__(SEQ_NT, 3) sv_seq_kernel(const SeqParams P) {
                 float vt[VEC], vd[VEC];
                 load_vec<DT>(rowt, alt, q, V, vt);
                 if (use_q) load_vec<DT>(rowd, ald, q, V, vd);
+                if (pv.allow) {
+#pragma unroll
+                    for (int t = 0; t < VEC; ++t) {
+                        const long long v = static_cast<long long>(q) * VEC + t;
+                        if (v < V) {
+                            vt[t] = proc_logit(vt[t], v, pv);
+                            if (use_q) vd[t] = proc_logit(vd[t], v, pv);
+                        }
+                    }
+                }
 #pragma unroll
                 for (int t = 0; t < VEC; ++t) w[t] = wt(vt[t], use_q ? vd[t] : NEG_INF);
             };

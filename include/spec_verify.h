@@ -99,8 +99,9 @@ typedef struct sv_options {
     void* event_start;         /* cudaEvent_t or NULL, recorded before the streaming kernel */
     void* event_stop;          /* cudaEvent_t or NULL, recorded right after it */
     uint64_t wait_timeout_ns;  /* bound of every device-side wait: 0 = 1e9 ns */
-    uint32_t test_extra_tx;    /* test hook: bytes added to each bulk-copy wait so that
-                                  the bounded wait runs out (0 in normal use) */
+    uint32_t test_extra_tx;    /* test hook (0 in normal use): each ring stage expects this
+                                  many bytes and no bulk copy is issued, so the bounded
+                                  wait runs out with nothing in flight */
     const float* top_p;        /* [B] fp32 or NULL: nucleus threshold per sequence, applied
                                   to p and q alike after top-k and temperature: the most
                                   probable kept tokens whose probabilities first sum to
@@ -110,8 +111,28 @@ typedef struct sv_options {
                                   kept-list path (0 < top_k < V, topk_path 0 or 1), else the
                                   call returns SV_ERR_UNSUPPORTED; a row whose kept list
                                   overflowed (massive ties at tau) becomes a row error.
-                                  Verification only: spec_sample_ex returns
-                                  SV_ERR_UNSUPPORTED when it is set. */
+                                  In spec_sample_ex, top_p[s] applies to the rows of
+                                  sequence s (see rows_per_sequence). */
+    /* Further processors (section "提议与核验的基本步骤", paragraph 4: applied
+     * to the target and draft distributions alike).  They act on the raw
+     * logits, before top-k, temperature, softmax and nucleus, the same way for
+     * every target and draft row of a sequence.  Stochastic mode only: with
+     * SV_MODE_GREEDY a non-NULL vocab_mask or rep_ids returns
+     * SV_ERR_UNSUPPORTED.  S is the number of sequences (B for verification,
+     * ceil(rows / rows_per_sequence) for spec_sample_ex). */
+    const uint32_t* vocab_mask;  /* [S][ceil(V/32)] uint32 or NULL: token v of sequence s is
+                                    allowed iff bit v % 32 of word v / 32 of row s is set; a
+                                    disallowed token gets the logit -inf (probability 0); a
+                                    sequence with no allowed finite logit is a row error */
+    const int32_t* rep_ids;      /* [S][n_rep] int32 or NULL: token ids the repetition penalty
+                                    applies to; ids outside [0, V) are ignored and a repeated
+                                    id is penalised once */
+    int n_rep;                   /* ids per sequence in rep_ids, >= 0 */
+    const float* rep_penalty;    /* [S] fp32 or NULL (all 1): theta > 0; a listed token's logit
+                                    z becomes z / theta if z > 0, else z * theta, rounded to
+                                    fp32; theta not > 0 makes the sequence a row error */
+    int rows_per_sequence;       /* spec_sample_ex only: row r takes the processors and top_p
+                                    of sequence r / rows_per_sequence (0 = 1) */
 } sv_options_t;
 
 /*

@@ -81,12 +81,38 @@ class Report:
         return self.flagged_accept + self.flagged_final
 
 
-def _final_cdf(target, draft, b, j, k, T, top_k):
+def seq_procs(procs, b):
+    """Keyword arguments of ``oracle.process_row_procs`` for sequence b of a
+    processors dict (top_p, rep_penalty, rep_ids, mask: per-sequence arrays or
+    None), or None without processors."""
+    if procs is None:
+        return None
+    out = {}
+    for key in ("top_p", "rep_penalty"):
+        if procs.get(key) is not None:
+            out[key] = float(np.asarray(procs[key]).reshape(-1)[b])
+    if procs.get("rep_ids") is not None:
+        out["rep_ids"] = np.asarray(procs["rep_ids"])[b]
+    if procs.get("mask") is not None:
+        out["mask"] = np.asarray(procs["mask"])[b]
+    return out
+
+
+def process(row, T, top_k, kw=None):
+    """The oracle's processed distribution of one row, with the processors
+    ``kw`` (from ``seq_procs``) when given."""
+    if kw is None:
+        return oracle.process_row(row, T, top_k)
+    return oracle.process_row_procs(row, T, top_k, **kw)
+
+
+def _final_cdf(target, draft, b, j, k, T, top_k, procs=None):
     """The oracle's weights of the final draw of sequence b at position j."""
-    pt = oracle.process_row(target[b, j], T, top_k)
+    kw = seq_procs(procs, b)
+    pt = process(target[b, j], T, top_k, kw)
     w = pt
     if j < k:
-        r = np.maximum(0.0, pt - oracle.process_row(draft[b, j], T, top_k))
+        r = np.maximum(0.0, pt - process(draft[b, j], T, top_k, kw))
         if r.sum() > 0:
             w = r
     return w, np.cumsum(w)
@@ -94,8 +120,9 @@ def _final_cdf(target, draft, b, j, k, T, top_k):
 
 def compare(ref: "oracle.VerifyResult", gpu: GpuResult, uniforms, greedy=False, check_pq=True,
             inputs=None) -> Report:
-    """``inputs`` = (target, draft, drafts, temperature, top_k) enables the
-    window check of final draws flagged as near-threshold."""
+    """``inputs`` = (target, draft, drafts, temperature, top_k[, procs])
+    enables the window check of final draws flagged as near-threshold
+    (``procs``: the per-sequence processors, see ``seq_procs``)."""
     B, k1 = ref.tokens.shape
     k = k1 - 1
     exact = fa = ff = errors = 0
@@ -127,9 +154,10 @@ def compare(ref: "oracle.VerifyResult", gpu: GpuResult, uniforms, greedy=False, 
                 assert np.array_equal(gpu.tokens[b, :j], ref.tokens[b, :j]), b
                 assert np.all(gpu.tokens[b, j + 1:] == -1), b
                 if inputs is not None:
-                    target, draft, drafts, temp, top_k = inputs
+                    target, draft, drafts, temp, top_k = inputs[:5]
+                    procs = inputs[5] if len(inputs) > 5 else None
                     T = 1.0 if temp is None else float(temp[b])
-                    w, C = _final_cdf(target, draft, b, j, k, T, top_k)
+                    w, C = _final_cdf(target, draft, b, j, k, T, top_k, procs)
                     y = int(gpu.tokens[b, j])
                     W = C[-1]
                     lo = (C[y - 1] if y > 0 else 0.0) / W
@@ -207,7 +235,8 @@ class SampleReport:
     errors: int
 
 
-def compare_samples(logits, u, temperature, top_k, got, ref, lo, hi, greedy=False) -> SampleReport:
+def compare_samples(logits, u, temperature, top_k, got, ref, lo, hi, greedy=False, procs=None,
+                    rows_per_seq=1) -> SampleReport:
     """GPU proposer draws vs the oracle's, one token per row of ``logits``.
 
     Greedy: bit-exact.  Stochastic: bit-exact, except rows whose uniform lies
@@ -215,7 +244,8 @@ def compare_samples(logits, u, temperature, top_k, got, ref, lo, hi, greedy=Fals
     token.  Those rows are counted, and the GPU token must have positive
     weight and a CDF interval (under the oracle's fp64 distribution) within
     DECISION_TOL of u.  The flagged count must stay within ``flag_bound`` of
-    the count the rule predicts from the oracle's distributions."""
+    the count the rule predicts from the oracle's distributions.  With
+    ``procs``, row r takes the processors of sequence r // rows_per_seq."""
     rows = got.shape[0]
     exact = flagged = errors = 0
     expected = 0.0
@@ -229,7 +259,7 @@ def compare_samples(logits, u, temperature, top_k, got, ref, lo, hi, greedy=Fals
             exact += 1
             continue
         T = 1.0 if temperature is None else float(temperature[r])
-        w = oracle.process_row(logits[r], T, top_k)
+        w = process(logits[r], T, top_k, seq_procs(procs, r // rows_per_seq))
         expected += flag_probability(w)
         ur = float(u[r])
         if abs(ur - lo[r]) < DECISION_TOL or abs(ur - hi[r]) < DECISION_TOL:

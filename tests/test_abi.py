@@ -57,11 +57,14 @@ def test_options_struct_layout_matches_c(tmp_path):
 #include <stdio.h>
 #include "spec_verify.h"
 int main(void) {
-  printf("%zu %zu %zu %zu %zu %zu %zu %zu %zu\n", sizeof(sv_options_t),
+  printf("%zu %zu %zu %zu %zu %zu %zu %zu %zu %zu %zu %zu %zu %zu\n", sizeof(sv_options_t),
          offsetof(sv_options_t, chunks_per_row), offsetof(sv_options_t, threads),
          offsetof(sv_options_t, topk_path), offsetof(sv_options_t, event_start),
          offsetof(sv_options_t, event_stop), offsetof(sv_options_t, wait_timeout_ns),
-         offsetof(sv_options_t, test_extra_tx), offsetof(sv_options_t, top_p));
+         offsetof(sv_options_t, test_extra_tx), offsetof(sv_options_t, top_p),
+         offsetof(sv_options_t, vocab_mask), offsetof(sv_options_t, rep_ids),
+         offsetof(sv_options_t, n_rep), offsetof(sv_options_t, rep_penalty),
+         offsetof(sv_options_t, rows_per_sequence));
   return 0;
 }
 """)
