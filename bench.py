@@ -44,6 +44,9 @@ KERNEL_SOURCES = [os.path.join(ROOT, "draft_token_verification_verify_b200", "cs
 
 WORKLOAD_ORDER = ("batched", "greedy", "large", "single", "tiny")
 GRAPH_WORKLOADS = ("single", "tiny")  # launch-bound: also timed from a CUDA-graph replay
+# the further processors on top of a workload: (workload, feature), reported as
+# "workload+feature" beside the five workloads
+FEATURES = (("batched", "mask+penalty"), ("batched", "top_p"), ("single", "top_p"))
 DESCR = {
     "tiny": "tiny stochastic verify B=1 k=4 V=32 fp32 T=1",
     "single": "single-sequence stochastic verify B=1 k=8 V=151936 bf16 T=1",
@@ -172,12 +175,32 @@ def pctl(xs, q: float) -> float:
     return s[min(len(s) - 1, max(0, math.ceil(q / 100.0 * len(s)) - 1))]
 
 
-def launches_per_step(case) -> int:
+def launches_per_step(case, feature=None) -> int:
     """Kernels one spec_verify call launches: the streaming pass and the
     per-sequence kernel, plus the residual segment kernel for stochastic
-    verification without top-k."""
+    verification without top-k; the processors add their bitmap kernel, a
+    nucleus without top-k its cut kernel."""
     stochastic_softmax = case.mode != "greedy" and not (0 < case.top_k < case.V)
-    return 3 if stochastic_softmax else 2
+    n = 3 if stochastic_softmax else 2
+    if feature == "mask+penalty":
+        n += 1
+    if feature == "top_p" and stochastic_softmax:
+        n += 1
+    return n
+
+
+def feature_tensors(feature, case, dev, seed):
+    """Device tensors of a feature's options (kept alive by the caller)."""
+    import torch
+
+    if feature is None:
+        return {}
+    pr = workloads.make_processors(seed, case.B, case.V, top_p=(0.7, 0.95))
+    t = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a).view(dt)).to(dev)
+    if feature == "top_p":
+        return {"top_p": t(pr.top_p, np.float32)}
+    return {"vocab_mask": t(pr.mask, np.int32), "rep_ids": t(pr.rep_ids, np.int32),
+            "rep_penalty": t(pr.rep_penalty, np.float32)}
 
 
 def to_dev(a, device):
@@ -369,14 +392,16 @@ def run_reference(args):
     return 0
 
 
-def measure_workload(name, args, sv, dev, world, rank, local, e2e_leg=False):
+def measure_workload(name, args, sv, dev, world, rank, local, e2e_leg=False, feature=None):
     """Time one workload: K steps bracketed by synchronize (and a barrier plus
     the max over ranks under torchrun), the streaming kernel alone from CUDA
     events over its own KSAMPLES launches, clocks sampled while the same steps
-    run, and optionally the end-to-end leg and a CUDA-graph replay."""
+    run, and optionally the end-to-end leg and a CUDA-graph replay.  With a
+    feature the proposer's draw and the verification take its options."""
     import torch
 
     case = workloads.make_case(name, seed=rank_seed(rank))
+    ftens = feature_tensors(feature, case, dev, rank_seed(rank))
     B, k, V = case.B, case.k, case.V
     greedy = case.mode == "greedy"
     mode = (sv.SV_MODE_GREEDY if greedy else sv.SV_MODE_STOCHASTIC) | (
@@ -391,7 +416,8 @@ def measure_workload(name, args, sv, dev, world, rank, local, e2e_leg=False):
     if greedy:
         drafts = sv.sample(to_dev(case.draft_proxy, dev), greedy=True)
     else:
-        drafts = sv.sample(draft0, to_dev(case.draft_uniforms, dev), temp.repeat_interleave(k), case.top_k)
+        drafts = sv.sample(draft0, to_dev(case.draft_uniforms, dev), temp.repeat_interleave(k), case.top_k,
+                           opts=sv.make_options(rows_per_sequence=k, **ftens) if ftens else None)
     torch.cuda.synchronize()
 
     # rotate input sets so that consecutive steps never hit in L2
@@ -403,11 +429,12 @@ def measure_workload(name, args, sv, dev, world, rank, local, e2e_leg=False):
     out_n = torch.empty((B,), dtype=torch.int32, device=dev)
     status = torch.zeros((1,), dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream()
-    wbytes = sv.spec_verify_workspace_size(B, k, V, case.top_k, mode)
+    base_opts = sv.make_options(**ftens) if ftens else None
+    wbytes = sv.spec_verify_workspace_size(B, k, V, case.top_k, mode, base_opts)
     wsp = torch.empty((max(wbytes, 1),), dtype=torch.uint8, device=dev)
 
     def step(i, ev0=None, ev1=None, on=None):
-        opts = sv.make_options(event_start=ev0, event_stop=ev1) if ev0 is not None else None
+        opts = sv.make_options(event_start=ev0, event_stop=ev1, **ftens) if ev0 is not None else base_opts
         st = sv.spec_verify_ex(targets[i % nsets], drafts_l[i % nsets], drafts, unif, B, k, V, temp,
                                case.top_k, mode, out_tok, out_n, None, None, status, wsp, wbytes, opts,
                                stream if on is None else on)
@@ -471,7 +498,7 @@ def measure_workload(name, args, sv, dev, world, rank, local, e2e_leg=False):
     peak, peak_src = measured_peak()
     achieved = logit_bytes / (kmean / 1000.0) / 1e9
     out = {
-        "workload": DESCR[name], "B": B, "k": k, "V": V, "top_k": case.top_k, "mode": case.mode,
+        "workload": DESCR[name] + (f", {feature}" if feature else ""), "B": B, "k": k, "V": V, "top_k": case.top_k, "mode": case.mode,
         "dtype": case.dtype, "value": value, "unit": "positions/s", "steps": args.steps,
         "ms_per_step": elapsed_ms / args.steps, "logit_gbs": gbs, "logit_bytes_per_step": logit_bytes,
         "l2": f"{nsets} rotating input set(s) of {logit_bytes / 1e6:.1f} MB"
@@ -483,7 +510,7 @@ def measure_workload(name, args, sv, dev, world, rank, local, e2e_leg=False):
                      "kernel_ms_p10": pctl(kern_ms, 10), "kernel_ms_p90": pctl(kern_ms, 90),
                      "kernel_samples": len(kern_ms),
                      "frac_of_spec": achieved / SPEC_HBM_GBS, "spec_gbs": SPEC_HBM_GBS},
-        "gpu_launches": launches_per_step(case) * args.steps,
+        "gpu_launches": launches_per_step(case, feature) * args.steps,
         "clocks": clocks,
     }
 
@@ -584,7 +611,8 @@ def run_ours(args):
     sv.lib()
 
     name = args.workload
-    head = measure_workload(name, args, sv, dev, world, rank, local, e2e_leg=not args.no_e2e)
+    head = measure_workload(name, args, sv, dev, world, rank, local, e2e_leg=not (args.no_e2e or args.feature),
+                            feature=args.feature)
     others = {}
     if not args.headline_only:
         for other in WORKLOAD_ORDER:
@@ -594,10 +622,15 @@ def run_ours(args):
             r.pop("_drafts")
             r.pop("_case")
             others[other] = r
+        for base, feature in FEATURES:
+            r = measure_workload(base, args, sv, dev, world, rank, local, feature=feature)
+            r.pop("_drafts")
+            r.pop("_case")
+            others[f"{base}+{feature}"] = r
     case, drafts = head.pop("_case"), head.pop("_drafts")
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.feature:
         try:
             cpu = cpu_baseline(name, args.cpu_budget)
         except Exception as exc:  # the multi-process leg failed: one thread instead
@@ -653,6 +686,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--graph", action="store_true",
                     help="also time the headline's steps replayed from a CUDA graph")
+    ap.add_argument("--feature", choices=sorted({f for _, f in FEATURES}), default=None,
+                    help="profile a feature alone: --workload with these options (no e2e or CPU leg)")
     ap.add_argument("--headline-only", action="store_true",
                     help="measure only --workload (default: every workload, the headline first)")
     args = ap.parse_args()

@@ -37,7 +37,7 @@ __all__ = [
     "SpecVerifyError", "lib", "spec_verify", "spec_verify_ex", "spec_verify_workspace_size",
     "spec_verify_static", "SV_STATIC_WORKSPACE_BYTES",
     "spec_sample", "spec_sample_ex", "spec_sample_workspace_size", "make_options",
-    "spec_verify_status_string", "spec_verify_version", "verify", "sample",
+    "spec_verify_status_string", "spec_verify_version", "spec_verify_pool_allocations", "verify", "sample",
 ]
 
 
@@ -97,6 +97,8 @@ def lib() -> ctypes.CDLL:
         L.spec_verify_status_string.restype = ctypes.c_char_p
         L.spec_verify_version.argtypes = []
         L.spec_verify_version.restype = I
+        L.spec_verify_pool_allocations.argtypes = []
+        L.spec_verify_pool_allocations.restype = ctypes.c_ulonglong
         _lib = L
     return _lib
 
@@ -137,6 +139,11 @@ def spec_verify_status_string(status: int) -> str:
 
 def spec_verify_version() -> int:
     return lib().spec_verify_version()
+
+
+def spec_verify_pool_allocations() -> int:
+    """Workspaces taken from the library's pool so far (calls without one)."""
+    return int(lib().spec_verify_pool_allocations())
 
 
 def spec_verify(target_logits, draft_logits, draft_tokens, uniforms, B, k, V, temperature, top_k,

@@ -9,6 +9,7 @@
 #include <climits>
 #include <cstdint>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "../../include/spec_verify.h"
@@ -114,6 +115,8 @@ struct Plan {
     bool pre = false;    // per-sequence kernel loads every row's kept list at once
     size_t pre_off = 0;
     size_t off_req = 0, off_mass = 0, off_counter = 0;
+    bool nuc = false;  // nucleus without top-k: the nucleus kernel cuts every row
+    size_t off_nuc = 0;
 };
 
 int rows_occupancy(int dev, int dt, int nt, int mode, bool proc, size_t smem);
@@ -214,6 +217,12 @@ sv_status_t make_plan(const DeviceInfo& dev, long long seqs, int k, int V, int d
         p.off_counter = round_up(p.off_mass + static_cast<size_t>(seqs) * p.nseg * sizeof(float2), 256);
         p.ws_bytes = round_up(p.off_counter + static_cast<size_t>(seqs) * sizeof(int), 256);
     }
+    // nucleus without top-k: one cut per row
+    if (opts && opts->top_p && p.mode == sv::MODE_SOFTMAX) {
+        p.nuc = true;
+        p.off_nuc = p.ws_bytes;
+        p.ws_bytes = round_up(p.off_nuc + static_cast<size_t>(p.R) * sizeof(sv::NucRec), 256);
+    }
     // per-sequence kernel: control, row stats, gather buffers, segment masses
     const int nrows = greedy ? k + 1 : 2 * k + 1;
     size_t head = static_cast<size_t>(nrows) * sizeof(sv::RowStat) + static_cast<size_t>(k + 1) * 8 + 8;
@@ -238,6 +247,7 @@ using RowsFn = void (*)(sv::RowsParams);
 using SeqFn = void (*)(sv::SeqParams);
 using ResFn = void (*)(sv::ResidParams);
 using ProcsFn = void (*)(sv::ProcsParams);
+using NucFn = void (*)(sv::NucParams);
 
 template <int DT, int NT, bool PROC>
 RowsFn rows_for_mode(int mode) {
@@ -336,6 +346,9 @@ struct Call {
     int32_t* out_status = nullptr;
 };
 
+// workspaces taken from the library pool by this process (the calls without one)
+std::atomic<unsigned long long> g_pool_allocs{0};
+
 sv_status_t run(const Call& cl, void* workspace, size_t workspace_bytes, const sv_options_t* opts,
                 cudaStream_t st) {
     int dev = 0;
@@ -345,7 +358,7 @@ sv_status_t run(const Call& cl, void* workspace, size_t workspace_bytes, const s
     sv_status_t s = make_plan(*info, cl.seqs, cl.k, cl.V, cl.dt, cl.greedy, cl.top_k, opts, cl.nprocs, &p);
     if (s != SV_OK) return s;
     if (workspace && (workspace_bytes < p.ws_bytes || !aligned(workspace, 16))) return SV_ERR_INVALID_ARG;
-    if (opts && opts->top_p && p.mode != sv::MODE_TOPK) return SV_ERR_UNSUPPORTED;  // nucleus needs the kept lists
+    if (opts && opts->top_p && p.mode == sv::MODE_GREEDY) return SV_ERR_UNSUPPORTED;  // greedy takes no nucleus
     if ((s = set_attrs(dev, cl.dt, p.nt1, p.mode, p.proc)) != SV_OK) return s;
 
     void* ws = workspace;
@@ -356,6 +369,7 @@ sv_status_t run(const Call& cl, void* workspace, size_t workspace_bytes, const s
             cudaGetLastError();
             return SV_ERR_CUDA;
         }
+        g_pool_allocs.fetch_add(1, std::memory_order_relaxed);
         owned = true;
     }
     auto* base = static_cast<unsigned char*>(ws);
@@ -431,6 +445,7 @@ sv_status_t run(const Call& cl, void* workspace, size_t workspace_bytes, const s
     q.out_status = cl.sample ? nullptr : cl.out_status;
     q.defer = p.defer ? 1 : 0;
     q.top_p = opts ? opts->top_p : nullptr;
+    q.nuc = p.nuc ? reinterpret_cast<sv::NucRec*>(base + p.off_nuc) : nullptr;
     q.pre = p.pre ? 1 : 0;
     q.pre_off = static_cast<int>(p.pre_off);
     q.req = p.defer ? reinterpret_cast<sv::DrawReq*>(base + p.off_req) : nullptr;
@@ -490,16 +505,20 @@ sv_status_t run(const Call& cl, void* workspace, size_t workspace_bytes, const s
         c1.stream = st;
         // programmatic dependent launch: the streaming pass may be placed while
         // the preceding kernel finishes (it waits for that grid before any
-        // access).  Not for a single wave that fills more than half the device:
-        // CTAs placed early, as slots free up (the preceding kernels are
-        // themselves placed early), land unevenly, and a few can miss the wave
-        // altogether and run after it (measured: +20 us per step).
+        // access), which hides the launch behind it.  Not for a single wave
+        // that fills more than half the device when an SM can take more than
+        // its even share of the wave: CTAs placed early, as slots free up (the
+        // preceding kernels are themselves placed early), would pile onto the
+        // SMs that free up first, and a few could miss the wave and run after
+        // it (measured: +20 us per step).
         cudaLaunchAttribute a1[1];
         a1[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
         a1[0].val.programmaticStreamSerializationAllowed = 1;
-        const bool tight_wave = p.tasks > p.slots / 2 && p.tasks <= p.slots;
-        c1.attrs = tight_wave ? nullptr : a1;
-        c1.numAttrs = tight_wave ? 0 : 1;
+        const long long per_sm = p.slots / info->sms;  // CTAs an SM can hold
+        const bool uneven = p.tasks > p.slots / 2 && p.tasks <= p.slots &&
+                            per_sm > ceil_div(p.tasks, info->sms);
+        c1.attrs = uneven ? nullptr : a1;
+        c1.numAttrs = uneven ? 0 : 1;
         if (cudaLaunchKernelEx(&c1, f1, r) != cudaSuccess) {
             result = SV_ERR_CUDA;
             break;
@@ -508,6 +527,42 @@ sv_status_t run(const Call& cl, void* workspace, size_t workspace_bytes, const s
             cudaEventRecord(static_cast<cudaEvent_t>(opts->event_stop), st) != cudaSuccess) {
             result = SV_ERR_CUDA;
             break;
+        }
+        if (p.nuc) {
+            // the nucleus cut of every row (programmatic dependent of the
+            // streaming pass; it waits for that grid before reading)
+            sv::NucParams np;
+            std::memset(&np, 0, sizeof np);
+            np.target = cl.target;
+            np.draft = cl.draft;
+            np.B = cl.seqs;
+            np.k = cl.k;
+            np.V = cl.V;
+            np.temperature = cl.temperature;
+            np.segs = r.segs;
+            np.nseg = p.nseg;
+            np.top_p = opts->top_p;
+            np.procs_div = static_cast<int>(cl.rows_per_seq);
+            np.allow = r.allow;
+            np.pen = r.pen;
+            np.theta = r.theta;
+            np.W4 = r.W4;
+            np.out = reinterpret_cast<sv::NucRec*>(base + p.off_nuc);
+            cudaLaunchAttribute an[1];
+            an[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+            an[0].val.programmaticStreamSerializationAllowed = 1;
+            cudaLaunchConfig_t cn;
+            std::memset(&cn, 0, sizeof cn);
+            cn.gridDim = dim3(static_cast<unsigned>(p.R), 1, 1);
+            cn.blockDim = dim3(sv::NUC_NT, 1, 1);
+            cn.stream = st;
+            cn.attrs = an;
+            cn.numAttrs = 1;
+            NucFn fn = cl.dt ? sv::sv_nucleus_kernel<1> : sv::sv_nucleus_kernel<0>;
+            if (cudaLaunchKernelEx(&cn, fn, np) != cudaSuccess) {
+                result = SV_ERR_CUDA;
+                break;
+            }
         }
         cudaLaunchAttribute a2[1];
         a2[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -788,5 +843,7 @@ const char* spec_verify_status_string(sv_status_t status) {
 }
 
 int spec_verify_version(void) { return kVersion; }
+
+unsigned long long spec_verify_pool_allocations(void) { return g_pool_allocs.load(std::memory_order_relaxed); }
 
 }  // extern "C"

@@ -458,13 +458,14 @@ __global__ void __launch_bounds__(NT + 32, RowsOcc<NT, MODE>::value) sv_rows_ker
             auto proc_vals = [&](const uint4& raw, int e, float* v) {
                 unpack<DT>(raw, v);
                 const uint32_t ab = bits_at(sallow, e, true), pb = bits_at(spen, e, false);
+                if (pb) {  // a listed token in this vector (rare): the rounded quotient or product
 #pragma unroll
-                for (int q = 0; q < VEC; ++q) {
-                    if (!valid(e + q) || !((ab >> q) & 1u))
-                        v[q] = NEG_INF;
-                    else if ((pb >> q) & 1u)
-                        v[q] = penalise(v[q], pen_theta);
+                    for (int q = 0; q < VEC; ++q)
+                        if ((pb >> q) & 1u) v[q] = penalise(v[q], pen_theta);
                 }
+#pragma unroll
+                for (int q = 0; q < VEC; ++q)
+                    if (!valid(e + q) || !((ab >> q) & 1u)) v[q] = NEG_INF;
             };
             // PROC: processed maximum of vector j (raw errors noted on the way)
             auto proc_vmax = [&](int j) -> float {

@@ -19,12 +19,16 @@
 // segment of the rejected (target, draft) pair).  Rows whose kept list did
 // not fit (massive ties), or top-k resolved by radix select, get an exact
 // radix select over the row in global memory and a draw that streams the
-// row (pair) in this CTA.
+// row (pair) in this CTA.  A nucleus (top_p < 1) is taken over the kept lists
+// on the top-k path, over the kept set of a radix-selected row here, and, with
+// no top-k, by the nucleus kernel, whose per-row cut and normaliser become
+// the row's threshold; every later read of a probability applies it.
 #pragma once
 
 #include <climits>
 
 #include "sv_common.cuh"
+#include "sv_nucleus.cuh"
 #include "sv_procs.cuh"
 
 namespace sv {
@@ -58,7 +62,8 @@ struct SeqParams {
                                  // list is loaded into shared memory at offset pre_off
     int pre_off;
     int defer;                   // residual draws go to the segment kernel (softmax, verify)
-    const float* top_p;          // [B] nucleus thresholds (top-k path only) or null
+    const float* top_p;          // [S] nucleus thresholds or null
+    const NucRec* nuc;           // [R] nucleus cuts of the rows (softmax mode with top_p) or null
     DrawReq* req;                // [B] when defer
     int* counter;                // [B] when defer: zeroed here for the segment kernel
     // processors (mask, repetition penalty): bitmaps built by K0, or null
@@ -99,23 +104,10 @@ struct __align__(16) SeqCtl {
     float base;
     float W;
     float c;
+    NucCtl nuc;  // nucleus cut of a row resolved here (radix top-k rows)
 };
 
 constexpr int SEQ_CTL_BYTES = (int)((sizeof(SeqCtl) + 127) / 128 * 128);
-
-// vector q of a row: elements [q*VEC, q*VEC + VEC) clipped to [0, V)
-template <int DT>
-__device__ __forceinline__ void load_vec(const void* row, bool aligned, int q, int V, float* v) {
-    constexpr int VEC = VT<DT>::VEC;
-    const long long e = static_cast<long long>(q) * VEC;
-    if (aligned && e + VEC <= V) {
-        const uint4 raw = __ldg(reinterpret_cast<const uint4*>(row) + q);
-        unpack<DT>(raw, v);
-    } else {
-#pragma unroll
-        for (int t = 0; t < VEC; ++t) v[t] = (e + t < V) ? load_elem<DT>(row, e + t) : NEG_INF;
-    }
-}
 
 template <int DT>
 __global__ void __launch_bounds__(SEQ_NT, 3) sv_seq_kernel(const SeqParams P) {
@@ -398,6 +390,13 @@ __global__ void __launch_bounds__(SEQ_NT, 3) sv_seq_kernel(const SeqParams P) {
             st.msc = m;
             st.invS = 1.f / s;
             if (m != m || m == POS_INF || m == NEG_INF || s != s) st.err = 1;
+            if (tp < 1.f && P.nuc && !st.err) {
+                // the nucleus kernel's cut: kept iff z >= cut, renormalised
+                const NucRec nr = P.nuc[r];
+                st.tau = nr.cut;
+                st.invS = nr.invS;
+                if (!(nr.invS > 0.f && nr.invS < POS_INF)) st.err = 1;
+            }
         } else {
             // top-k: raw maximum over the chunks, then the kept set
             float mx = NEG_INF;
@@ -482,10 +481,8 @@ __global__ void __launch_bounds__(SEQ_NT, 3) sv_seq_kernel(const SeqParams P) {
                     st.invS = 1.f / acc;
                     st.zd = zd;  // -inf: the draft token is not kept (probability 0)
                 }
-                if (tp < 1.f && !st.err) {
-                    if (st.slow) {
-                        st.err = 1;  // the nucleus needs the kept list of the row
-                    } else {
+                if (tp < 1.f && !st.err && !st.slow) {  // slow rows: after their radix select
+                    {
                         // Nucleus over the kept set: the cut is the largest kept value
                         // x whose tail mass (probabilities of the values >= x) reaches
                         // top_p; every value >= x is kept and renormalised.
@@ -588,6 +585,17 @@ __global__ void __launch_bounds__(SEQ_NT, 3) sv_seq_kernel(const SeqParams P) {
                 rs[rr].zd = (d >= 0 && d < V) ? proc_logit(load_elem<DT>(row, d), d, pv) : __int_as_float(0x7fc00000);
             }
             __syncthreads();
+            if (tp > 0.f && tp < 1.f) {
+                // the nucleus over the row's kept set {z >= tau}
+                float cut, inv;
+                nucleus_block<DT, NT>(row, V, rs[rr].tau, rs[rr].msc, c, tp, pv, S.nuc, cut, inv);
+                if (tid == 0) {
+                    rs[rr].tau = fmaxf(cut, rs[rr].tau);
+                    rs[rr].invS = inv;
+                    if (!(inv > 0.f && inv < POS_INF)) rs[rr].err = 1;
+                }
+                __syncthreads();
+            }
         }
     }
 
@@ -784,7 +792,7 @@ __global__ void __launch_bounds__(SEQ_NT, 3) sv_seq_kernel(const SeqParams P) {
                 for (int t = 0; t < VEC; ++t) w[t] = wt(vt[t], use_q ? vd[t] : NEG_INF);
             };
             // masses known from the streaming pass: a plain (unmasked) bonus draw
-            const bool known = P.mode == MODE_SOFTMAX && !use_q0;
+            const bool known = P.mode == MODE_SOFTMAX && !use_q0 && !(tp < 1.f);
             for (int attempt = 0; attempt < 2; ++attempt) {
                 if (known) {
                     for (int s = tid; s < P.nseg; s += NT) {

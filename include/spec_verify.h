@@ -107,12 +107,13 @@ typedef struct sv_options {
                                   probable kept tokens whose probabilities first sum to
                                   >= top_p are kept, every token as probable as the last one
                                   included, then renormalised (1 keeps all).  Values outside
-                                  (0, 1] make the sequence a row error.  Needs the top-k
-                                  kept-list path (0 < top_k < V, topk_path 0 or 1), else the
-                                  call returns SV_ERR_UNSUPPORTED; a row whose kept list
-                                  overflowed (massive ties at tau) becomes a row error.
-                                  In spec_sample_ex, top_p[s] applies to the rows of
-                                  sequence s (see rows_per_sequence). */
+                                  (0, 1] make the sequence a row error.  With top-k the cut
+                                  is taken over each row's kept set; without top-k over the
+                                  whole row (one more kernel: an exact cut found by a mass
+                                  histogram and a radix select over the row, two to five
+                                  reads of it).  SV_MODE_GREEDY with top_p returns
+                                  SV_ERR_UNSUPPORTED.  In spec_sample_ex, top_p[s] applies
+                                  to the rows of sequence s (see rows_per_sequence). */
     /* Further processors (section "提议与核验的基本步骤", paragraph 4: applied
      * to the target and draft distributions alike).  They act on the raw
      * logits, before top-k, temperature, softmax and nucleus, the same way for
@@ -257,6 +258,12 @@ SV_API const char* spec_verify_status_string(sv_status_t status);
 
 /* Library version as MAJOR * 10000 + MINOR * 100 + PATCH. */
 SV_API int spec_verify_version(void);
+
+/* Workspaces this process has taken from the library's pool: one per call of
+ * spec_verify, spec_sample, or an _ex entry point given a NULL workspace.
+ * Calls given a workspace (and spec_verify_static, the size queries and
+ * calls refused before launch) allocate nothing and leave it unchanged. */
+SV_API unsigned long long spec_verify_pool_allocations(void);
 
 #ifdef __cplusplus
 }

@@ -29,7 +29,8 @@ def declared_functions():
 def test_header_declares_entry_points():
     assert declared_functions() == sorted([
         "spec_sample", "spec_sample_ex", "spec_sample_workspace_size", "spec_verify", "spec_verify_ex",
-        "spec_verify_static", "spec_verify_status_string", "spec_verify_version", "spec_verify_workspace_size"])
+        "spec_verify_pool_allocations", "spec_verify_static", "spec_verify_status_string", "spec_verify_version",
+        "spec_verify_workspace_size"])
 
 
 def test_library_exports_every_declared_symbol(L):
@@ -41,6 +42,20 @@ def test_library_exports_every_declared_symbol(L):
         assert hasattr(L, name)
     # nothing else leaks out of the C ABI
     assert exported == set(declared_functions())
+
+
+def test_no_pool_allocation_without_a_launch(L):
+    """Size queries, refused calls and calls given a workspace never take a
+    workspace from the library's pool (here, without a GPU, none launches)."""
+    a0 = sv.spec_verify_pool_allocations()
+    sv.spec_verify_workspace_size(64, 4, 151936, 50, 0)
+    sv.spec_sample_workspace_size(8, 1000, 0, 0)
+    st = sv.spec_verify_ex(P, P, P, P, 2, 3, 100, None, 0, 0, P, P, None, None, None, P, 1 << 20, None, 0)
+    assert st != sv.SV_OK
+    st = sv.spec_verify_ex(P, P, P, P, 0, 3, 100, None, 0, 0, P, P, stream=0)  # invalid: B = 0
+    assert st == sv.SV_ERR_INVALID_ARG
+    assert sv.spec_verify(P, P, P, P, 2, 0, 100, None, 0, 0, P, P, stream=0) == sv.SV_ERR_INVALID_ARG  # k = 0
+    assert sv.spec_verify_pool_allocations() == a0
 
 
 def test_version_and_status_strings(L):
@@ -160,13 +175,6 @@ def test_misaligned_top_p_rejected(L):
     o.top_p = 0x1002  # not 4-byte aligned
     st = sv.spec_verify_ex(P, P, P, P, 2, 3, 100, None, 50, 0, P, P, None, None, None, None, 0, o, 0)
     assert st == sv.SV_ERR_INVALID_ARG
-
-
-def test_sampler_refuses_top_p(L):
-    o = sv.make_options()
-    o.top_p = 0x1000
-    st = sv.spec_sample_ex(P, P, 4, 50, None, 5, 0, P, None, 0, o, 0)
-    assert st == sv.SV_ERR_UNSUPPORTED
 
 
 @pytest.mark.parametrize("kw", [dict(B=0), dict(k=0), dict(V=0), dict(top_k=-1), dict(mode=7)])

@@ -104,19 +104,17 @@ def test_top_p_out_of_range_is_a_row_error():
     assert np.all(tok[[0, 1, 3]] == -1)
 
 
-def test_top_p_needs_the_kept_lists():
+def test_greedy_takes_no_nucleus():
     import torch
 
     import draft_token_verification_verify_b200 as sv
 
-    case = workloads.make_case("tiny", seed=58, B=2, k=2, V=64)  # no top-k
-    drafts = np.zeros((2, 2), np.int32)
+    case = workloads.make_case("greedy", seed=58, B=2, V=500)
     dev = torch.device("cuda:0")
     tp = torch.full((2,), 0.9, dtype=torch.float32, device=dev)
-    tok = torch.empty((2, 3), dtype=torch.int32, device=dev)
+    tok = torch.empty((2, case.k + 1), dtype=torch.int32, device=dev)
     n = torch.empty((2,), dtype=torch.int32, device=dev)
-    mode = sv.SV_MODE_STOCHASTIC | sv.SV_DTYPE_F32
-    st = sv.spec_verify_ex(to_dev(case.target), to_dev(case.draft), torch.from_numpy(drafts).to(dev),
-                           to_dev(case.uniforms), 2, 2, 64, None, 0, mode, tok, n,
+    st = sv.spec_verify_ex(to_dev(case.target), None, torch.zeros((2, case.k), dtype=torch.int32, device=dev),
+                           None, 2, case.k, case.V, None, 0, sv.SV_MODE_GREEDY | sv.SV_DTYPE_BF16, tok, n,
                            opts=sv.make_options(top_p=tp))
     assert st == sv.SV_ERR_UNSUPPORTED

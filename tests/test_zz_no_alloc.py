@@ -128,3 +128,32 @@ def test_static_rejects_problems_beyond_its_buffer():
     assert sv.spec_verify_ex(target, draft, drafts, uni, B, k, V, None, K, mode, tok, n) == sv.SV_OK
     torch.cuda.synchronize()
     assert (n >= 0).all()
+
+
+@pytest.mark.parametrize("name,over", CASES[:3], ids=["batched-topk", "batched-softmax", "large-f32"])
+def test_caller_workspace_takes_nothing_from_the_pool(name, over):
+    """spec_verify_ex given a workspace allocates nothing: the pool counter and
+    the device's free memory stay put; without one it takes one workspace
+    from the pool per call."""
+    import torch
+
+    import draft_token_verification_verify_b200 as sv
+
+    case, greedy, t = _inputs(name, **over)
+    need = sv.spec_verify_workspace_size(case.B, case.k, case.V, case.top_k, _mode(case, greedy))
+    ws = torch.empty(need, dtype=torch.uint8, device=torch.device("cuda:0"))
+    outs = [_outputs(case.B, case.k) for _ in range(3)]
+    assert _call(sv.spec_verify_ex, case, greedy, t, outs[0], workspace=ws, workspace_bytes=need) == sv.SV_OK
+    torch.cuda.synchronize()
+    a0 = sv.spec_verify_pool_allocations()
+    free0, _ = torch.cuda.mem_get_info()
+    for o in outs[1:]:
+        assert _call(sv.spec_verify_ex, case, greedy, t, o, workspace=ws, workspace_bytes=need) == sv.SV_OK
+    torch.cuda.synchronize()
+    assert sv.spec_verify_pool_allocations() == a0
+    assert torch.cuda.mem_get_info()[0] == free0
+    for o in outs[1:]:
+        assert torch.equal(o["tok"], outs[0]["tok"]) and torch.equal(o["n"], outs[0]["n"])
+    assert _call(sv.spec_verify_ex, case, greedy, t, _outputs(case.B, case.k)) == sv.SV_OK  # pool
+    torch.cuda.synchronize()
+    assert sv.spec_verify_pool_allocations() == a0 + 1
