@@ -548,16 +548,23 @@ sv_status_t run(const Call& cl, void* workspace, size_t workspace_bytes, const s
             np.theta = r.theta;
             np.W4 = r.W4;
             np.out = reinterpret_cast<sv::NucRec*>(base + p.off_nuc);
-            cudaLaunchAttribute an[1];
+            // few rows: a cluster of up to 8 CTAs shares each row
+            int ncl = 1;
+            while (ncl < 8 && p.R * ncl < info->sms) ncl *= 2;
+            cudaLaunchAttribute an[2];
             an[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
             an[0].val.programmaticStreamSerializationAllowed = 1;
+            an[1].id = cudaLaunchAttributeClusterDimension;
+            an[1].val.clusterDim.x = static_cast<unsigned>(ncl);
+            an[1].val.clusterDim.y = 1;
+            an[1].val.clusterDim.z = 1;
             cudaLaunchConfig_t cn;
             std::memset(&cn, 0, sizeof cn);
-            cn.gridDim = dim3(static_cast<unsigned>(p.R), 1, 1);
+            cn.gridDim = dim3(static_cast<unsigned>(p.R * ncl), 1, 1);
             cn.blockDim = dim3(sv::NUC_NT, 1, 1);
             cn.stream = st;
             cn.attrs = an;
-            cn.numAttrs = 1;
+            cn.numAttrs = 2;
             NucFn fn = cl.dt ? sv::sv_nucleus_kernel<1> : sv::sv_nucleus_kernel<0>;
             if (cudaLaunchKernelEx(&cn, fn, np) != cudaSuccess) {
                 result = SV_ERR_CUDA;

@@ -24,7 +24,13 @@
 //      logits, whose keys have 16 significant bits, four otherwise), each
 //      pass choosing the digit whose tail mass reaches what is left of the
 //      target.
+// With few rows the nucleus kernel splits each row over a thread-block
+// cluster: every CTA histograms its share of the row in its own shared
+// memory, CTA 0 sums the cluster's histograms through distributed shared
+// memory and takes each decision, the others read it back from CTA 0.
 #pragma once
+
+#include <cooperative_groups.h>
 
 #include "sv_common.cuh"
 #include "sv_procs.cuh"
@@ -98,15 +104,53 @@ __device__ __forceinline__ void nuc_pick(const unsigned long long* hist, unsigne
     at = __shfl_sync(0xffffffffu, a, L);
 }
 
-// Block-wide nucleus cut of one row.  Elements below tau0 (a top-k
-// threshold, or -inf) weigh nothing; msc is the row maximum times c (over the
-// elements >= tau0), 0 < tp < 1.  Every thread of the block calls it; the
-// results are returned to all of them.
-template <int DT, int NT>
+// Nucleus cut of one row by one CTA (CL = false) or by the CTAs of a cluster
+// (CL = true, each taking every ncl-th group of vectors).  Elements below
+// tau0 (a top-k threshold, or -inf) weigh nothing; msc is the row maximum
+// times c (over the elements >= tau0), 0 < tp < 1.  Every thread calls it;
+// the results are returned to all of them.
+template <int DT, int NT, bool CL = false>
 __device__ void nucleus_block(const void* row, int V, float tau0, float msc, float c, float tp, const ProcView& pv,
                               NucCtl& N, float& cut, float& invS) {
     constexpr int VEC = VT<DT>::VEC;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    int crank = 0, ncl = 1;
+    if constexpr (CL) {
+        crank = static_cast<int>(cooperative_groups::this_cluster().block_rank());
+        ncl = static_cast<int>(cooperative_groups::this_cluster().num_blocks());
+    }
+    const bool lead = crank == 0;  // takes the decisions
+    // CL: sum the cluster's histograms into CTA 0's
+    auto gather = [&]() {
+        if constexpr (CL) {
+            auto cl = cooperative_groups::this_cluster();
+            cl.sync();
+            if (lead) {
+                for (int h = tid; h < 256; h += NT) {
+                    unsigned long long sum = N.hist[h];
+                    for (int rk = 1; rk < ncl; ++rk) sum += *cl.map_shared_rank(&N.hist[h], rk);
+                    N.hist[h] = sum;
+                }
+            }
+        }
+        __syncthreads();
+    };
+    // CL: every CTA takes CTA 0's decision
+    auto share = [&]() {
+        if constexpr (CL) {
+            auto cl = cooperative_groups::this_cluster();
+            cl.sync();
+            if (!lead && tid == 0) {
+                const NucCtl* D = cl.map_shared_rank(&N, 0);
+                N.bin = D->bin;
+                N.above = D->above;
+                N.trem = D->trem;
+                N.prefix = D->prefix;
+                N.last = D->last;
+            }
+        }
+        __syncthreads();
+    };
     const bool al = (reinterpret_cast<uintptr_t>(row) & 15u) == 0;
     const int nvec = (V + VEC - 1) / VEC;
     const int KROUNDS = (DT == 0 && !pv.allow) ? 2 : 4;
@@ -114,17 +158,18 @@ __device__ void nucleus_block(const void* row, int V, float tau0, float msc, flo
     // h = 255 - weight bin (higher h: heavier)
     auto visit = [&](auto&& f) {
         constexpr int U = 4;  // vector loads in flight per thread
-        for (int q0 = tid; q0 < nvec; q0 += NT * U) {
+        const int step = NT * ncl;
+        for (int q0 = crank * NT + tid; q0 < nvec; q0 += step * U) {
             uint4 raw[U];
 #pragma unroll
             for (int u = 0; u < U; ++u) {
-                const int q = q0 + u * NT;
+                const int q = q0 + u * step;
                 if (al && q < nvec && static_cast<long long>(q + 1) * VEC <= V)
                     raw[u] = __ldg(reinterpret_cast<const uint4*>(row) + q);
             }
 #pragma unroll
             for (int u = 0; u < U; ++u) {
-                const int q = q0 + u * NT;
+                const int q = q0 + u * step;
                 if (q >= nvec) continue;
                 const long long e0 = static_cast<long long>(q) * VEC;
                 float v[VEC];
@@ -162,8 +207,8 @@ __device__ void nucleus_block(const void* row, int V, float tau0, float msc, flo
             atomicAdd(&N.hist[h], W);
     });
     if (tail) atomicAdd(&N.hist[0], tail);
-    __syncthreads();
-    if (warp == 0) {
+    gather();
+    if (lead && warp == 0) {
         unsigned long long tot = 0ull;
 #pragma unroll
         for (int i = 0; i < 8; ++i) tot += N.hist[8 * lane + i];
@@ -183,7 +228,7 @@ __device__ void nucleus_block(const void* row, int V, float tau0, float msc, flo
             N.last = at;
         }
     }
-    __syncthreads();
+    share();
     // 2. exact key digits inside that bin
     const int hb = N.bin;
     for (int round = 0; round < KROUNDS; ++round) {
@@ -198,8 +243,8 @@ __device__ void nucleus_block(const void* row, int V, float tau0, float msc, flo
             const unsigned long long W = weight(x);
             if (W) atomicAdd(&N.hist[(key >> shift) & 255u], W);
         });
-        __syncthreads();
-        if (warp == 0) {
+        gather();
+        if (lead && warp == 0) {
             int dg;
             unsigned long long bf, at;
             nuc_pick(N.hist, N.trem, lane, dg, bf, at);
@@ -210,13 +255,16 @@ __device__ void nucleus_block(const void* row, int V, float tau0, float msc, flo
                 N.last = at;
             }
         }
-        __syncthreads();
+        share();
     }
     const uint32_t p = N.prefix;
     cut = okey_inv(KROUNDS == 2 ? (p << 16 | ((p & 0x8000u) ? 0u : 0xffffu)) : p);
     const unsigned long long kept = N.above + N.last;
     invS = kept ? static_cast<float>(0x1p40 / static_cast<double>(kept)) : __int_as_float(0x7fc00000);
-    __syncthreads();  // N is reused by the caller
+    if constexpr (CL)
+        cooperative_groups::this_cluster().sync();  // no CTA leaves while CTA 0's decision is read
+    else
+        __syncthreads();  // N is reused by the caller
 }
 
 struct NucParams {
@@ -237,14 +285,15 @@ struct NucParams {
     NucRec* out;               // [R]
 };
 
-// One CTA per row: the row's cut and kept normaliser.  Rows whose sequence
-// has no nucleus (top_p = 1), an invalid setting or an invalid row get
-// {-inf, 1/S}: K2 validates the settings and the row itself.
+// One cluster of CTAs per row (launched with cluster size 1 to 8): the row's
+// cut and kept normaliser.  Rows whose sequence has no nucleus (top_p = 1),
+// an invalid setting or an invalid row get {-inf, 1/S}: K2 validates the
+// settings and the row itself.
 template <int DT>
 __global__ void __launch_bounds__(NUC_NT) sv_nucleus_kernel(const NucParams P) {
     constexpr int ELT = VT<DT>::ELT;
     __shared__ NucCtl N;
-    const long long r = blockIdx.x;
+    const long long r = blockIdx.x / cooperative_groups::this_cluster().num_blocks();
     const long long Rt = P.B * (P.k + 1);
     const char* row;
     long long b;
@@ -284,9 +333,9 @@ __global__ void __launch_bounds__(NUC_NT) sv_nucleus_kernel(const NucParams P) {
     if (ok) {  // uniform over the block
         const float c = LOG2E / T;
         const ProcView pv = proc_view(P.allow, P.pen, P.theta, P.W4, s);
-        nucleus_block<DT, NUC_NT>(row, P.V, NEG_INF, m, c, tp, pv, N, rec.cut, rec.invS);
+        nucleus_block<DT, NUC_NT, true>(row, P.V, NEG_INF, m, c, tp, pv, N, rec.cut, rec.invS);
     }
-    if (tid == 0) P.out[r] = rec;
+    if (tid == 0 && cooperative_groups::this_cluster().block_rank() == 0) P.out[r] = rec;
 }
 
 }  // namespace sv

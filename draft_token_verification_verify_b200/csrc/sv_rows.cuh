@@ -111,10 +111,13 @@ constexpr int MASK_STAGE_BYTES = (TILE_BYTES / 2 / 32 * 4 + 32 + 127) / 128 * 12
 constexpr int STAGE_BYTES_PROC = STAGE_BYTES + 2 * MASK_STAGE_BYTES;
 
 // Dynamic shared memory of one streaming CTA.
+__host__ __device__ constexpr int rows_tail_bytes(int mode, int nt, int lcap) {
+    return (mode == MODE_SOFTMAX ? 2 * MAX_TILES_K1 * (nt / 32) * 4 : 0) + (mode == MODE_TOPK ? lcap * (4 + 4) : 0);
+}
 __host__ __device__ constexpr int rows_smem_bytes(int mode, int nt, int stages, int lcap, bool proc) {
-    return ROWS_CTL_BYTES + stages * (proc ? STAGE_BYTES_PROC : STAGE_BYTES) +
-           (mode == MODE_SOFTMAX ? 2 * MAX_TILES_K1 * (nt / 32) * 4 : 0) +
-           (mode == MODE_TOPK ? lcap * (4 + 4) : 0);
+    // processors: each consumer thread parks its vector maxima of a tile
+    return ROWS_CTL_BYTES + stages * (proc ? STAGE_BYTES_PROC : STAGE_BYTES) + rows_tail_bytes(mode, nt, lcap) +
+           (proc ? (TILE_BYTES / 16 / nt + 1) * nt * 4 : 0);
 }
 
 // Geometry of one segment in the ring: the stage mirrors the 16-byte aligned
@@ -155,6 +158,24 @@ __device__ __forceinline__ void consumer_sync() {
     asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory");
 }
 
+// Elements of a packed vector whose bit in `keep` is clear become -inf.
+template <int DT>
+__device__ __forceinline__ uint4 mask_neg_inf(uint4 r, uint32_t keep) {
+    uint32_t* w = reinterpret_cast<uint32_t*>(&r);
+    if constexpr (DT == 0) {  // two bf16 per word
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t k = (((keep >> (2 * i)) & 1u) ? 0x0000ffffu : 0u) |
+                               (((keep >> (2 * i + 1)) & 1u) ? 0xffff0000u : 0u);
+            w[i] = (w[i] & k) | (0xff80ff80u & ~k);
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) w[i] = ((keep >> i) & 1u) ? w[i] : 0xff800000u;
+    }
+    return r;
+}
+
 template <int NT, int MODE>
 struct RowsOcc {  // CTAs per SM the register budget is sized for
     // top-k CTAs hold their candidate lists in shared memory, which caps them
@@ -185,6 +206,7 @@ __global__ void __launch_bounds__(NT + 32, RowsOcc<NT, MODE>::value) sv_rows_ker
     float* const red_s = red_m + MAX_TILES_K1 * NW;
     float* const lkey = reinterpret_cast<float*>(tail);           // top-k: [lcap] candidate-vector maxima
     int* const lidx = reinterpret_cast<int*>(lkey + P.lcap);      //        [lcap] their place: t*(TV+1) + j
+    float* const vmsh = reinterpret_cast<float*>(tail + rows_tail_bytes(MODE, NT, P.lcap));  // PROC: [VPT+1][NT]
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const long long task = blockIdx.x;
@@ -467,14 +489,31 @@ __global__ void __launch_bounds__(NT + 32, RowsOcc<NT, MODE>::value) sv_rows_ker
                 for (int q = 0; q < VEC; ++q)
                     if (!valid(e + q) || !((ab >> q) & 1u)) v[q] = NEG_INF;
             };
-            // PROC: processed maximum of vector j (raw errors noted on the way)
-            auto proc_vmax = [&](int j) -> float {
+            // PROC: processed maximum of vector j (raw errors noted on the way).
+            // Without a penalised element the disallowed (or out-of-segment)
+            // elements are replaced by -inf in the packed vector with bit
+            // operations and the plain maximum is taken; a vector holding a
+            // listed id takes the per-element path.
+            // Top-k with theta >= 1: no processed value exceeds its raw one, so
+            // a vector whose raw maximum is below the running bound cannot be
+            // a candidate and counts as -inf (the bounds stay lower bounds).
+            auto proc_vmax = [&](int j, float skip_below) -> float {
                 const uint4 raw = vec_at(j);
                 const int e = g.e0 + j * VEC;
                 const bool full = e >= g.lo && e + VEC <= g.hi;
                 const float rm = full ? vmax_nan<DT>(raw) : vmax_masked(j);
                 if (!(rm == rm) || rm == POS_INF) rawbad = true;
-                if (full && bits_at(sallow, e, true) == VMASK && bits_at(spen, e, false) == 0u) return rm;
+                if (rm < skip_below) return NEG_INF;
+                uint32_t ab = bits_at(sallow, e, true);
+                const uint32_t pb = bits_at(spen, e, false);
+                if (pb == 0u) {
+                    if (!full) {
+#pragma unroll
+                        for (int q = 0; q < VEC; ++q)
+                            if (!valid(e + q)) ab &= ~(1u << q);
+                    }
+                    return vmax_nan<DT>(mask_neg_inf<DT>(raw, ab));
+                }
                 float v[VEC];
                 proc_vals(raw, e, v);
                 float m = NEG_INF;
@@ -489,11 +528,16 @@ __global__ void __launch_bounds__(NT + 32, RowsOcc<NT, MODE>::value) sv_rows_ker
             float vm[VPT + 1];
             const bool tile_full = ok && g.e0 == g.lo && g.nvec == TV && g.hi - g.lo == TV * VEC;
             if constexpr (PROC) {
-#pragma unroll
+                // one copy of the processing code (a rolled loop); the maxima
+                // come back to registers through this thread's own slots
+                const float skip_below = (MODE == MODE_TOPK && pen_theta >= 1.f) ? theta : NEG_INF;
+#pragma unroll 1
                 for (int i = 0; i <= VPT; ++i) {
                     const int j = jof(i);
-                    vm[i] = (ok && j < g.nvec) ? proc_vmax(j) : NEG_INF;
+                    vmsh[i * NT + tid] = (ok && j < g.nvec) ? proc_vmax(j, skip_below) : NEG_INF;
                 }
+#pragma unroll
+                for (int i = 0; i <= VPT; ++i) vm[i] = vmsh[i * NT + tid];
             } else if (tile_full) {
 #pragma unroll
                 for (int i = 0; i < VPT; ++i) vm[i] = vmax_nan<DT>(vec_at(tid + i * NT));
@@ -542,21 +586,36 @@ __global__ void __launch_bounds__(NT + 32, RowsOcc<NT, MODE>::value) sv_rows_ker
                 const float m = wtm * cscale;
                 float sa = 0.f, sb = 0.f;
                 if (ok && m > NEG_INF && m < POS_INF) {
+                    auto acc_vec = [&](int j) {
+                        float v[VEC];
+                        if constexpr (PROC) {
+                            const int e = g.e0 + j * VEC;
+                            if (bits_at(spen, e, false) == 0u) {
+                                uint32_t ab = bits_at(sallow, e, true);
 #pragma unroll
-                    for (int i = 0; i <= VPT; ++i) {
-                        const int j = jof(i);
-                        if (j < g.nvec) {
-                            float v[VEC];
-                            if constexpr (PROC)
-                                proc_vals(vec_at(j), g.e0 + j * VEC, v);
-                            else
-                                load_masked(j, v);
-#pragma unroll
-                            for (int q = 0; q < VEC; q += 2) {
-                                sa += ex2(fmaf(v[q], cscale, -m));
-                                sb += ex2(fmaf(v[q + 1], cscale, -m));
+                                for (int q = 0; q < VEC; ++q)
+                                    if (!valid(e + q)) ab &= ~(1u << q);
+                                unpack<DT>(mask_neg_inf<DT>(vec_at(j), ab), v);
+                            } else {
+                                proc_vals(vec_at(j), e, v);
                             }
+                        } else {
+                            load_masked(j, v);
                         }
+#pragma unroll
+                        for (int q = 0; q < VEC; q += 2) {
+                            sa += ex2(fmaf(v[q], cscale, -m));
+                            sb += ex2(fmaf(v[q + 1], cscale, -m));
+                        }
+                    };
+                    if constexpr (PROC) {  // one copy of the processing code
+#pragma unroll 1
+                        for (int i = 0; i <= VPT; ++i)
+                            if (jof(i) < g.nvec) acc_vec(jof(i));
+                    } else {
+#pragma unroll
+                        for (int i = 0; i <= VPT; ++i)
+                            if (jof(i) < g.nvec) acc_vec(jof(i));
                     }
                 }
                 const float ws = warp_sum(sa + sb);

@@ -99,6 +99,14 @@ def test_batched_top_k_full_vocabulary(which):
     assert ref.errors == 0 and rep.exact >= case.B - 2
 
 
+def test_penalty_below_one_with_top_k():
+    """theta < 1 raises the listed positive logits: the streaming pass cannot
+    skip a vector on its raw maximum then."""
+    case = workloads.make_case("batched", seed=72, B=8)
+    ref, _, rep = _check(case, _procs(72, case.B, case.V, "mask+penalty", theta=0.6, n_rep=400))
+    assert ref.errors == 0 and rep.exact >= case.B - 2
+
+
 @pytest.mark.parametrize("which", ["mask", "mask+penalty"])
 def test_softmax_full_vocabulary_bf16(which):
     """No top-k: the residual draws rescan the processed row pair."""
