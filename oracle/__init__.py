@@ -43,6 +43,8 @@ def lib():
         _lib.oracle_verify_procs.restype = I
         _lib.oracle_sample_rows_procs.argtypes = [P, I, I, I, I, P, I, P, P, P, I, P, P, P]
         _lib.oracle_sample_rows_procs.restype = I
+        _lib.oracle_verify_tree.argtypes = [P, P, P, P, P, I, I, I, P, I, I, I, P, P, P, P, P, P, P, P]
+        _lib.oracle_verify_tree.restype = I
     return _lib
 
 
@@ -262,3 +264,55 @@ def sample_rows_procs(logits, u, temperature=None, top_k: int = 0, top_p=None, r
     if errs < 0:
         raise MemoryError("oracle_sample_rows_procs could not allocate its work arrays")
     return out.reshape(B, rps)
+
+
+@dataclasses.dataclass
+class TreeResult:
+    tokens: np.ndarray      # [B, N+1] int32: accepted tokens, the final token, then -1
+    n_accepted: np.ndarray  # [B] int32 (-1: error)
+    nodes: np.ndarray       # [B, N+1] int32: the accepted nodes, then -1
+    p: np.ndarray           # [B, N] current-distribution probability of each tested child's token
+    q: np.ndarray           # [B, N] draft probability of it (NaN: not tested)
+    ratio: np.ndarray       # [B, N] acceptance threshold min(1, p/q)
+    cdf_lo: np.ndarray      # [B]
+    cdf_hi: np.ndarray      # [B]
+    errors: int
+
+
+def verify_tree(target, draft, tokens, parents, uniforms=None, temperature=None, top_k: int = 0,
+                greedy: bool = False) -> TreeResult:
+    """Tree verification (reading R18 of the C source): target and draft
+    [B, N+1, V] (one row per node, node 0 the verified context), tokens and
+    parents [B, N] (node n at index n - 1, parent < n), uniforms [B, N+1]."""
+    target = np.ascontiguousarray(target)
+    B, n1, V = target.shape
+    N = n1 - 1
+    dt = _dtype_code(target)
+    if draft is not None:
+        draft = np.ascontiguousarray(draft)
+        assert draft.dtype == target.dtype and draft.shape == (B, N + 1, V)
+    elif not greedy:
+        raise ValueError("stochastic verification needs draft logits")
+    tokens = np.ascontiguousarray(tokens, dtype=np.int32).reshape(B, N)
+    parents = np.ascontiguousarray(parents, dtype=np.int32).reshape(B, N)
+    if uniforms is not None:
+        uniforms = np.ascontiguousarray(uniforms, dtype=np.float32).reshape(B, N + 1)
+    elif not greedy:
+        raise ValueError("stochastic verification needs uniforms")
+    if temperature is not None:
+        temperature = np.ascontiguousarray(temperature, dtype=np.float32).reshape(B)
+    out = np.empty((B, N + 1), dtype=np.int32)
+    n = np.empty(B, dtype=np.int32)
+    nodes = np.empty((B, N + 1), dtype=np.int32)
+    p = np.empty((B, max(N, 1)), dtype=np.float64)
+    q = np.empty_like(p)
+    ratio = np.empty_like(p)
+    lo = np.empty(B, dtype=np.float64)
+    hi = np.empty(B, dtype=np.float64)
+    errs = lib().oracle_verify_tree(_ptr(target), _ptr(draft), _ptr(tokens), _ptr(parents), _ptr(uniforms),
+                                    B, N, V, _ptr(temperature), int(top_k), int(bool(greedy)), dt, _ptr(out),
+                                    _ptr(n), _ptr(nodes), _ptr(p), _ptr(q), _ptr(ratio), _ptr(lo), _ptr(hi))
+    if errs < 0:
+        raise MemoryError("oracle_verify_tree could not allocate its work arrays")
+    return TreeResult(out, n, nodes, p[:, :N], q[:, :N], ratio[:, :N], lo, hi, errs)
+

@@ -557,3 +557,145 @@ int oracle_sample_rows_procs(const void* logits, int dtype, int rows, int rows_p
     free(prob); free(work); free(pv);
     return errors;
 }
+
+/* ==== tree verification =====================================================
+ *
+ * The entry's section "提议方式与实现形态", paragraph 3, names candidate trees
+ * besides chains; the pages give no acceptance rule for them.  The reading
+ * taken here (R18) is the plainest one that reduces to paragraph 2 of
+ * "提议与核验的基本步骤" on a chain:
+ *   - node 0 is the verified context, node n >= 1 carries the draft token
+ *     t_n and a parent par_n < n; target row n and draft row n are the target
+ *     and draft distributions of the token that follows node n's prefix (the
+ *     children of node n were drawn from draft row n);
+ *   - the walk starts at node 0 with the current distribution R = p (the
+ *     processed target row of the node) and tries the node's children in
+ *     index order: child c is accepted iff u_c * q(t_c) < R(t_c) (R1 on the
+ *     current distribution, q the processed draft row of the node, u_c the
+ *     child's own uniform); a rejection replaces R by the normalised residual
+ *     max(0, R - q) (left unchanged when that has no mass, the reading of R8);
+ *   - an accepted child's token is emitted and the walk continues from that
+ *     child; when no child of the current node is accepted (or it has none)
+ *     the final token is drawn from R with the last uniform (R3);
+ *   - greedy: the first child whose token is the lowest-index argmax of the
+ *     node's target row is accepted; if none, that argmax is emitted (R6);
+ *   - the rows a walk reads are those of the nodes it visits; a row error
+ *     (R7) there, a token outside [0, V), a parent outside [0, n) or (in
+ *     stochastic mode) a uniform outside [0, 1) or a bad temperature makes the
+ *     sequence an error.
+ * With children drawn independently from q, each emitted token follows p of
+ * its prefix (rejection with the residual is the one-candidate step applied
+ * again to the residual).
+ *
+ *   target, draft  [B][N+1][V] dtype (draft ignored when greedy)
+ *   tokens, parents [B][N]  (node n at index n - 1)
+ *   uniforms       [B][N+1] (u_c at index c - 1, the final draw at N)
+ * Outputs: out_tokens [B][N+1] (the accepted tokens, the final token, then
+ * -1), out_n [B] (accepted tokens, -1 on an error); optional: out_nodes
+ * [B][N+1] (the accepted nodes, then -1), out_p / out_q / out_ratio [B][N]
+ * (R(t_c), q(t_c) and min(1, R/q) for every child tested, NaN otherwise),
+ * out_lo / out_hi [B] (the CDF points around the final token).
+ * Returns the number of sequences reported as errors (-1: no memory).
+ */
+int oracle_verify_tree(const void* target, const void* draft, const int32_t* tokens,
+                       const int32_t* parents, const float* uniforms, int B, int N, int V,
+                       const float* temperature, int top_k, int greedy, int dtype,
+                       int32_t* out_tokens, int32_t* out_n, int32_t* out_nodes, double* out_p,
+                       double* out_q, double* out_ratio, double* out_lo, double* out_hi) {
+    int b, i, errors = 0;
+    double* R = (double*)malloc(sizeof(double) * (size_t)V);
+    double* Q = (double*)malloc(sizeof(double) * (size_t)V);
+    double* work = (double*)malloc(sizeof(double) * (size_t)V);
+    if (!R || !Q || !work) {
+        free(R); free(Q); free(work);
+        return -1;
+    }
+    for (b = 0; b < B; ++b) {
+        const int32_t* t = tokens + (size_t)b * N;
+        const int32_t* par = parents + (size_t)b * N;
+        const float* u = uniforms ? uniforms + (size_t)b * (N + 1) : NULL;
+        int32_t* tok = out_tokens + (size_t)b * (N + 1);
+        int32_t* nodes = out_nodes ? out_nodes + (size_t)b * (N + 1) : NULL;
+        double T = temperature ? (double)temperature[b] : 1.0;
+        int err = 0, depth = 0, a = 0, y = -1;
+        double lo = NAN, hi = NAN;
+        for (i = 0; i <= N; ++i) {
+            tok[i] = -1;
+            if (nodes) nodes[i] = -1;
+        }
+        for (i = 0; i < N; ++i) {
+            if (out_p) out_p[(size_t)b * N + i] = NAN;
+            if (out_q) out_q[(size_t)b * N + i] = NAN;
+            if (out_ratio) out_ratio[(size_t)b * N + i] = NAN;
+            if (t[i] < 0 || t[i] >= V || par[i] < 0 || par[i] > i) err = 1;
+        }
+        if (!greedy) {
+            if (!(T > 0.0) || isinf(T) || isnan(T)) err = 1;
+            for (i = 0; i <= N && !err; ++i)
+                if (!(u[i] >= 0.0f && u[i] < 1.0f)) err = 1;
+        }
+        while (!err) {
+            const long row = (long)b * (N + 1) + a;
+            int c, next = 0;
+            if (greedy) {
+                int g = oracle_argmax_row(or_row(target, dtype, row, V), dtype, V);
+                if (g < 0) {
+                    err = 1;
+                    break;
+                }
+                for (c = a + 1; c <= N && !next; ++c)
+                    if (par[c - 1] == a && t[c - 1] == g) next = c;
+                if (!next) {
+                    y = g;
+                    break;
+                }
+            } else {
+                long v;
+                err |= oracle_process_row(or_row(target, dtype, row, V), dtype, V, T, top_k, R, work);
+                if (!err) err |= oracle_process_row(or_row(draft, dtype, row, V), dtype, V, T, top_k, Q, work);
+                if (err) break;
+                for (c = a + 1; c <= N && !next; ++c) {
+                    double r, q, W = 0.0;
+                    if (par[c - 1] != a) continue;
+                    r = R[t[c - 1]];
+                    q = Q[t[c - 1]];
+                    if (out_p) out_p[(size_t)b * N + c - 1] = r;
+                    if (out_q) out_q[(size_t)b * N + c - 1] = q;
+                    if (out_ratio)
+                        out_ratio[(size_t)b * N + c - 1] = q > 0.0 ? (r / q < 1.0 ? r / q : 1.0) : (r > 0.0 ? 1.0 : 0.0);
+                    if ((double)u[c - 1] * q < r) {
+                        next = c;
+                        break;
+                    }
+                    /* rejected: the residual becomes the current distribution */
+                    for (v = 0; v < V; ++v) W += (R[v] > Q[v]) ? R[v] - Q[v] : 0.0;
+                    if (W > 0.0)
+                        for (v = 0; v < V; ++v) R[v] = (R[v] > Q[v]) ? (R[v] - Q[v]) / W : 0.0;
+                }
+                if (!next) {
+                    oracle_inverse_cdf(R, V, (double)u[N], &y, &lo, &hi);
+                    break;
+                }
+            }
+            tok[depth] = t[next - 1];
+            if (nodes) nodes[depth] = next;
+            depth++;
+            a = next;
+        }
+        if (err) {
+            for (i = 0; i <= N; ++i) {
+                tok[i] = -1;
+                if (nodes) nodes[i] = -1;
+            }
+            out_n[b] = -1;
+            errors++;
+        } else {
+            tok[depth] = y;
+            out_n[b] = depth;
+        }
+        if (out_lo) out_lo[b] = lo;
+        if (out_hi) out_hi[b] = hi;
+    }
+    free(R); free(Q); free(work);
+    return errors;
+}
