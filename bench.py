@@ -592,6 +592,68 @@ def measure_workload(name, args, sv, dev, world, rank, local, e2e_leg=False, fea
     return out
 
 
+TREE_PARENTS = (0, 0, 1, 1, 2, 2, 3, 3)  # a binary tree of 8 candidate nodes
+
+
+def measure_tree(args, sv, dev, world, rank):
+    """Tree verification on the batched workload's shapes and value model: B
+    sequences of a binary tree of 8 candidates (one target and one draft row
+    per node plus the root), each node's token drawn on the GPU from its
+    parent's processed draft row; K steps bracketed by synchronize."""
+    import torch
+
+    N = len(TREE_PARENTS)
+    case = workloads.make_case("batched", seed=rank_seed(rank), k=N)
+    B, V = case.B, case.V
+    target = to_dev(case.target, dev)                                             # [B, N+1, V]
+    draft = to_dev(np.concatenate([case.draft, case.draft[:, -1:]], axis=1), dev)
+    par = torch.tensor(TREE_PARENTS, dtype=torch.int32, device=dev).repeat(B, 1)
+    par_rows = torch.gather(draft, 1, par.long()[:, :, None].expand(B, N, V))      # [B, N, V]
+    temp = to_dev(case.temperature, dev)
+    toks = sv.sample(par_rows, to_dev(case.draft_uniforms, dev), temp.repeat_interleave(N), case.top_k)
+    toks = toks.view(B, N).contiguous()
+    del par_rows
+    unif = to_dev(case.uniforms, dev)
+    set_bytes = (target.numel() + draft.numel()) * target.element_size()
+    nsets = max(2, -(-4 * L2_BYTES // set_bytes))
+    nsets = min(nsets, 8)
+    targets = [target] + [target.clone() for _ in range(nsets - 1)]
+    drafts = [draft] + [draft.clone() for _ in range(nsets - 1)]
+    out_tok = torch.empty((B, N + 1), dtype=torch.int32, device=dev)
+    out_n = torch.empty((B,), dtype=torch.int32, device=dev)
+    mode = sv.SV_MODE_STOCHASTIC | sv.SV_DTYPE_BF16
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        st = sv.spec_verify_tree(targets[i % nsets], drafts[i % nsets], toks, par, unif, B, N, V, temp,
+                                 case.top_k, mode, out_tok, out_n, None, None, None, stream)
+        if st != sv.SV_OK:
+            raise sv.SpecVerifyError(st, "spec_verify_tree")
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(rank)
+    sampler.start()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    a.record(stream)
+    for i in range(args.steps):
+        step(i)
+    b.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ms = max_over_ranks(a.elapsed_time(b), dev)
+    n_host = out_n.cpu().numpy()
+    return {"workload": f"batched tree verify B={B} N={N} (binary) V={V} bf16 T=0.7 top-k {case.top_k}",
+            "value": job_rate(B * N * args.steps, world, ms), "unit": "verified candidate nodes/s",
+            "ms_per_step": ms / args.steps, "mean_accepted": float(n_host.mean()),
+            "gpu_launches": args.steps, "clocks": clocks,
+            "l2": f"{nsets} rotating input set(s) of {set_bytes / 1e6:.1f} MB"}
+
+
 def run_ours(args):
     import torch
 
@@ -627,6 +689,7 @@ def run_ours(args):
             r.pop("_drafts")
             r.pop("_case")
             others[f"{base}+{feature}"] = r
+        others["tree"] = measure_tree(args, sv, dev, world, local)
     case, drafts = head.pop("_case"), head.pop("_drafts")
 
     cpu = None

@@ -38,6 +38,7 @@ __all__ = [
     "spec_verify_static", "SV_STATIC_WORKSPACE_BYTES",
     "spec_sample", "spec_sample_ex", "spec_sample_workspace_size", "make_options",
     "spec_verify_status_string", "spec_verify_version", "spec_verify_pool_allocations", "verify", "sample",
+    "spec_verify_tree", "verify_tree",
 ]
 
 
@@ -85,6 +86,8 @@ def lib() -> ctypes.CDLL:
         L.spec_verify_ex.restype = I
         L.spec_verify_static.argtypes = [P, P, P, P, I, I, I, P, I, I, P, P, P, P, P, OP, P]
         L.spec_verify_static.restype = I
+        L.spec_verify_tree.argtypes = [P, P, P, P, P, I, I, I, P, I, I, P, P, P, P, P, P]
+        L.spec_verify_tree.restype = I
         L.spec_verify_workspace_size.argtypes = [I, I, I, I, I, OP]
         L.spec_verify_workspace_size.restype = Z
         L.spec_sample.argtypes = [P, P, I, I, P, I, I, P, P]
@@ -244,6 +247,55 @@ def _check(t, name, dtypes, numel, device):
 def _check_cuda(device):
     if device.type != "cuda":
         raise ValueError(f"tensors must be on a CUDA device, got {device}")
+
+
+def spec_verify_tree(target_logits, draft_logits, tokens, parents, uniforms, B, N, V, temperature, top_k, mode,
+                     out_tokens, out_n_accepted, out_nodes=None, out_p=None, out_q=None, stream=None) -> int:
+    return lib().spec_verify_tree(_p(target_logits), _p(draft_logits), _p(tokens), _p(parents), _p(uniforms),
+                                  int(B), int(N), int(V), _p(temperature), int(top_k), int(mode),
+                                  _p(out_tokens), _p(out_n_accepted), _p(out_nodes), _p(out_p), _p(out_q),
+                                  _stream(stream))
+
+
+def verify_tree(target, draft, tokens, parents, uniforms=None, temperature=None, top_k: int = 0,
+                greedy: bool = False, out_nodes=None, out_p=None, out_q=None, stream=None):
+    """Tensor convenience wrapper around ``spec_verify_tree``: target and draft
+    [B, N+1, V] (one row per node, node 0 the verified context), tokens and
+    parents [B, N] int32 (node n at index n - 1), uniforms [B, N+1] fp32,
+    temperature [B] fp32 or None; optional outputs out_nodes [B, N+1] int32,
+    out_p / out_q [B, N] fp32.  Checked like ``verify``.  Returns
+    (out_tokens [B, N+1], out_n_accepted [B])."""
+    import torch
+
+    if target.dim() != 3:
+        raise ValueError(f"target must be [B, N+1, V], got shape {tuple(target.shape)}")
+    B, n1, V = target.shape
+    N = n1 - 1
+    dev = target.device
+    f32, i32 = (torch.float32,), (torch.int32,)
+    mode = (SV_MODE_GREEDY if greedy else SV_MODE_STOCHASTIC) | _dtype_code(target)
+    _check(target, "target", (target.dtype,), B * n1 * V, dev)
+    _check(tokens, "tokens", i32, B * N, dev)
+    _check(parents, "parents", i32, B * N, dev)
+    if not greedy:
+        _check(draft, "draft", (target.dtype,), B * n1 * V, dev)
+        _check(uniforms, "uniforms", f32, B * n1, dev)
+        if temperature is not None:
+            _check(temperature, "temperature", f32, B, dev)
+        for t, name in ((out_p, "out_p"), (out_q, "out_q")):
+            if t is not None:
+                _check(t, name, f32, B * N, dev)
+    if out_nodes is not None:
+        _check(out_nodes, "out_nodes", i32, B * n1, dev)
+    _check_cuda(dev)
+    out_tokens = torch.empty((B, n1), dtype=torch.int32, device=dev)
+    out_n = torch.empty((B,), dtype=torch.int32, device=dev)
+    st = spec_verify_tree(target, None if greedy else draft, tokens, parents, None if greedy else uniforms, B, N, V,
+                          None if greedy else temperature, top_k, mode, out_tokens, out_n, out_nodes,
+                          None if greedy else out_p, None if greedy else out_q, stream)
+    if st != SV_OK:
+        raise SpecVerifyError(st, "spec_verify_tree")
+    return out_tokens, out_n
 
 
 def verify(target, draft, draft_tokens, uniforms=None, temperature=None, top_k: int = 0,

@@ -16,6 +16,7 @@
 #include "sv_rows.cuh"
 #include "sv_resid.cuh"
 #include "sv_seq.cuh"
+#include "sv_tree.cuh"
 
 namespace {
 
@@ -248,6 +249,7 @@ using SeqFn = void (*)(sv::SeqParams);
 using ResFn = void (*)(sv::ResidParams);
 using ProcsFn = void (*)(sv::ProcsParams);
 using NucFn = void (*)(sv::NucParams);
+using TreeFn = void (*)(sv::TreeParams);
 
 template <int DT, int NT, bool PROC>
 RowsFn rows_for_mode(int mode) {
@@ -767,6 +769,59 @@ void* static_scratch(int dev) {
 }  // namespace
 
 extern "C" {
+
+sv_status_t spec_verify_tree(const void* target_logits, const void* draft_logits, const int32_t* tokens,
+                             const int32_t* parents, const float* uniforms, int B, int N, int V,
+                             const float* temperature, int top_k, int mode, int32_t* out_tokens,
+                             int32_t* out_n_accepted, int32_t* out_nodes, float* out_p, float* out_q,
+                             void* stream) {
+    bool greedy = false;
+    int dt = 0;
+    if (B <= 0 || N < 1 || N > sv::TREE_MAX_NODES || V < 1 || top_k < 0) return SV_ERR_INVALID_ARG;
+    if (!decode_mode(mode, &greedy, &dt)) return SV_ERR_INVALID_ARG;
+    const int elt = dt ? 4 : 2;
+    if (static_cast<unsigned long long>(B) * (N + 1) > (1ULL << 62) / (static_cast<unsigned long long>(V) * 4ULL))
+        return SV_ERR_INVALID_ARG;
+    if (!target_logits || !tokens || !parents || !out_tokens || !out_n_accepted) return SV_ERR_INVALID_ARG;
+    if (!greedy && (!draft_logits || !uniforms)) return SV_ERR_INVALID_ARG;
+    if (!aligned(target_logits, elt) || (draft_logits && !aligned(draft_logits, elt)) || !aligned(tokens, 4) ||
+        !aligned(parents, 4) || (uniforms && !aligned(uniforms, 4)) || (temperature && !aligned(temperature, 4)) ||
+        !aligned(out_tokens, 4) || !aligned(out_n_accepted, 4) || (out_nodes && !aligned(out_nodes, 4)) ||
+        (out_p && !aligned(out_p, 4)) || (out_q && !aligned(out_q, 4)))
+        return SV_ERR_INVALID_ARG;
+    if (V > sv::TREE_SEG * sv::TREE_MAX_SEG) return SV_ERR_UNSUPPORTED;
+    int dev = 0;
+    if (!device_info(&dev)) return SV_ERR_UNSUPPORTED;
+    sv::TreeParams t;
+    std::memset(&t, 0, sizeof t);
+    t.target = target_logits;
+    t.draft = greedy ? nullptr : draft_logits;
+    t.tokens = tokens;
+    t.parents = parents;
+    t.uniforms = greedy ? nullptr : uniforms;
+    t.temperature = greedy ? nullptr : temperature;
+    t.B = B;
+    t.N = N;
+    t.V = V;
+    t.top_k = (!greedy && top_k > 0 && top_k < V) ? top_k : 0;
+    t.greedy = greedy ? 1 : 0;
+    t.out_tokens = out_tokens;
+    t.out_n = out_n_accepted;
+    t.out_nodes = out_nodes;
+    t.out_p = greedy ? nullptr : out_p;
+    t.out_q = greedy ? nullptr : out_q;
+    cudaLaunchConfig_t ct;
+    std::memset(&ct, 0, sizeof ct);
+    ct.gridDim = dim3(static_cast<unsigned>(B), 1, 1);
+    ct.blockDim = dim3(sv::TREE_NT, 1, 1);
+    ct.stream = static_cast<cudaStream_t>(stream);
+    TreeFn ft = dt ? sv::sv_tree_kernel<1> : sv::sv_tree_kernel<0>;
+    if (cudaLaunchKernelEx(&ct, ft, t) != cudaSuccess) {
+        cudaGetLastError();
+        return SV_ERR_CUDA;
+    }
+    return SV_OK;
+}
 
 sv_status_t spec_verify_ex(const void* target_logits, const void* draft_logits, const int32_t* draft_tokens,
                            const float* uniforms, int B, int k, int V, const float* temperature, int top_k,

@@ -253,6 +253,44 @@ SV_API sv_status_t spec_sample_ex(const void* logits, const float* uniforms, int
                                   int32_t* out_tokens, void* workspace, size_t workspace_bytes,
                                   const sv_options_t* opts, void* stream);
 
+/*
+ * spec_verify_tree — verify one round of tree-shaped candidates for B
+ * sequences (candidate trees: section "提议方式与实现形态", paragraph 3; the
+ * pages give no acceptance rule for them, the one taken reduces to the chain
+ * rule of "提议与核验的基本步骤", paragraph 2, on a chain).
+ *   Node 0 of each sequence is the verified context; node n in [1, N] carries
+ *   tokens[b][n-1] and has the parent parents[b][n-1] in [0, n).  Row n of
+ *   target_logits / draft_logits [B][N+1][V] (bf16 or fp32, per `mode`) is
+ *   the target / draft distribution of the token after node n's prefix (the
+ *   children of node n were drawn from draft row n).
+ *   Stochastic: the walk starts at node 0 with R = p (the node's processed
+ *   target row, temperature and top-k as in spec_verify) and tries the node's
+ *   children in index order; child c is accepted iff
+ *   uniforms[b][c-1] * q(t_c) < R(t_c) (q the node's processed draft row),
+ *   and the walk continues from it; a rejection replaces R by the normalised
+ *   residual max(0, R - q) (kept as it is when that has no mass); when no
+ *   child is accepted the final token is drawn from R by the inverse CDF
+ *   with uniforms[b][N].  Greedy: the first child whose token is the node's
+ *   lowest-index argmax is accepted, else that argmax is emitted (draft
+ *   logits, uniforms and temperature unused, may be NULL).
+ *   Outputs: out_tokens [B][N+1] (the accepted tokens, the final token, then
+ *   -1), out_n_accepted [B] (-1: the sequence is an error); optional (NULL to
+ *   skip): out_nodes [B][N+1] (the accepted nodes, then -1), out_p / out_q
+ *   [B][N] (R(t_c) and q(t_c) of every tested child, NaN otherwise).
+ *   Only the rows of visited nodes are read.  Row errors: a NaN or +inf
+ *   logit or no finite kept logit in a row read, a token outside [0, V), a
+ *   parent outside [0, n), and (stochastic) a uniform outside [0, 1) or a
+ *   temperature not finite and > 0.  N <= 256, V <= 262,144
+ *   (SV_ERR_UNSUPPORTED above).  Allocates nothing; all work is enqueued on
+ *   `stream`.  Argument errors return SV_ERR_INVALID_ARG before any launch.
+ */
+SV_API sv_status_t spec_verify_tree(const void* target_logits, const void* draft_logits,
+                                    const int32_t* tokens, const int32_t* parents,
+                                    const float* uniforms, int B, int N, int V,
+                                    const float* temperature, int top_k, int mode,
+                                    int32_t* out_tokens, int32_t* out_n_accepted,
+                                    int32_t* out_nodes, float* out_p, float* out_q, void* stream);
+
 /* Static description of a status code. */
 SV_API const char* spec_verify_status_string(sv_status_t status);
 

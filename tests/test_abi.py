@@ -29,8 +29,9 @@ def declared_functions():
 def test_header_declares_entry_points():
     assert declared_functions() == sorted([
         "spec_sample", "spec_sample_ex", "spec_sample_workspace_size", "spec_verify", "spec_verify_ex",
-        "spec_verify_pool_allocations", "spec_verify_static", "spec_verify_status_string", "spec_verify_version",
-        "spec_verify_workspace_size"])
+        "spec_verify_pool_allocations", "spec_verify_static", "spec_verify_status_string", "spec_verify_tree",
+        "spec_verify_version", "spec_verify_workspace_size"])
+
 
 
 def test_library_exports_every_declared_symbol(L):
@@ -303,3 +304,23 @@ def test_sample_wrapper_checks_layout():
         sv.sample(logits, u, torch.ones(12, dtype=torch.float32))   # one temperature per row: valid
     with pytest.raises(ValueError, match="CUDA device"):
         sv.sample(logits, greedy=True)
+
+
+@pytest.mark.parametrize("kw", [dict(B=0), dict(N=0), dict(N=257), dict(V=0), dict(top_k=-1), dict(mode=7),
+                                dict(target=None), dict(tokens=None), dict(parents=None), dict(draft=None),
+                                dict(uniforms=None), dict(target=P + 1), dict(tokens=P + 2), dict(out_p=P + 2)])
+def test_tree_invalid_arguments(L, kw):
+    a = dict(target=P, draft=P, tokens=P, parents=P, uniforms=P, B=2, N=3, V=100, temperature=None, top_k=0,
+             mode=0, out_tokens=P, out_n=P, out_nodes=None, out_p=None, out_q=None)
+    a.update(kw)
+    st = sv.spec_verify_tree(a["target"], a["draft"], a["tokens"], a["parents"], a["uniforms"], a["B"], a["N"],
+                             a["V"], a["temperature"], a["top_k"], a["mode"], a["out_tokens"], a["out_n"],
+                             a["out_nodes"], a["out_p"], a["out_q"], stream=0)
+    assert st == sv.SV_ERR_INVALID_ARG
+
+
+def test_tree_greedy_needs_no_draft(L):
+    # greedy reads neither the draft logits nor the uniforms: NULL passes the checks
+    # (on a machine without a GPU the call then stops at the device: unsupported)
+    st = sv.spec_verify_tree(P, None, P, P, None, 2, 3, 100, None, 0, sv.SV_MODE_GREEDY, P, P, stream=0)
+    assert st in (sv.SV_OK, sv.SV_ERR_UNSUPPORTED)
