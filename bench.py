@@ -623,12 +623,15 @@ def measure_tree(args, sv, dev, world, rank):
     out_n = torch.empty((B,), dtype=torch.int32, device=dev)
     mode = sv.SV_MODE_STOCHASTIC | sv.SV_DTYPE_BF16
     stream = torch.cuda.current_stream()
+    wbytes = sv.spec_verify_tree_workspace_size(B, N, V, case.top_k, mode)  # the list walk's records
+    ws = torch.empty((max(wbytes, 1),), dtype=torch.uint8, device=dev)
 
     def step(i):
-        st = sv.spec_verify_tree(targets[i % nsets], drafts[i % nsets], toks, par, unif, B, N, V, temp,
-                                 case.top_k, mode, out_tok, out_n, None, None, None, stream)
+        st = sv.spec_verify_tree_ex(targets[i % nsets], drafts[i % nsets], toks, par, unif, B, N, V, temp,
+                                    case.top_k, mode, out_tok, out_n, None, None, None,
+                                    ws if wbytes else None, wbytes, stream)
         if st != sv.SV_OK:
-            raise sv.SpecVerifyError(st, "spec_verify_tree")
+            raise sv.SpecVerifyError(st, "spec_verify_tree_ex")
 
     for i in range(args.warmup):
         step(i)
@@ -650,7 +653,8 @@ def measure_tree(args, sv, dev, world, rank):
     return {"workload": f"batched tree verify B={B} N={N} (binary) V={V} bf16 T=0.7 top-k {case.top_k}",
             "value": job_rate(B * N * args.steps, world, ms), "unit": "verified candidate nodes/s",
             "ms_per_step": ms / args.steps, "mean_accepted": float(n_host.mean()),
-            "gpu_launches": args.steps, "clocks": clocks,
+            "gpu_launches": (4 if wbytes else 1) * args.steps, "clocks": clocks,
+            "path": "streaming pass + list walk" if wbytes else "walk over the rows",
             "l2": f"{nsets} rotating input set(s) of {set_bytes / 1e6:.1f} MB"}
 
 

@@ -38,7 +38,7 @@ __all__ = [
     "spec_verify_static", "SV_STATIC_WORKSPACE_BYTES",
     "spec_sample", "spec_sample_ex", "spec_sample_workspace_size", "make_options",
     "spec_verify_status_string", "spec_verify_version", "spec_verify_pool_allocations", "verify", "sample",
-    "spec_verify_tree", "verify_tree",
+    "spec_verify_tree", "spec_verify_tree_ex", "spec_verify_tree_workspace_size", "verify_tree",
 ]
 
 
@@ -88,6 +88,10 @@ def lib() -> ctypes.CDLL:
         L.spec_verify_static.restype = I
         L.spec_verify_tree.argtypes = [P, P, P, P, P, I, I, I, P, I, I, P, P, P, P, P, P]
         L.spec_verify_tree.restype = I
+        L.spec_verify_tree_ex.argtypes = [P, P, P, P, P, I, I, I, P, I, I, P, P, P, P, P, P, Z, P]
+        L.spec_verify_tree_ex.restype = I
+        L.spec_verify_tree_workspace_size.argtypes = [I, I, I, I, I]
+        L.spec_verify_tree_workspace_size.restype = Z
         L.spec_verify_workspace_size.argtypes = [I, I, I, I, I, OP]
         L.spec_verify_workspace_size.restype = Z
         L.spec_sample.argtypes = [P, P, I, I, P, I, I, P, P]
@@ -257,9 +261,24 @@ def spec_verify_tree(target_logits, draft_logits, tokens, parents, uniforms, B, 
                                   _stream(stream))
 
 
+def spec_verify_tree_ex(target_logits, draft_logits, tokens, parents, uniforms, B, N, V, temperature, top_k, mode,
+                        out_tokens, out_n_accepted, out_nodes=None, out_p=None, out_q=None, workspace=None,
+                        workspace_bytes=0, stream=None) -> int:
+    return lib().spec_verify_tree_ex(_p(target_logits), _p(draft_logits), _p(tokens), _p(parents), _p(uniforms),
+                                     int(B), int(N), int(V), _p(temperature), int(top_k), int(mode),
+                                     _p(out_tokens), _p(out_n_accepted), _p(out_nodes), _p(out_p), _p(out_q),
+                                     _p(workspace), int(workspace_bytes), _stream(stream))
+
+
+def spec_verify_tree_workspace_size(B, N, V, top_k, mode) -> int:
+    return int(lib().spec_verify_tree_workspace_size(int(B), int(N), int(V), int(top_k), int(mode)))
+
+
 def verify_tree(target, draft, tokens, parents, uniforms=None, temperature=None, top_k: int = 0,
-                greedy: bool = False, out_nodes=None, out_p=None, out_q=None, stream=None):
-    """Tensor convenience wrapper around ``spec_verify_tree``: target and draft
+                greedy: bool = False, out_nodes=None, out_p=None, out_q=None, workspace=None, stream=None):
+    """Tensor convenience wrapper around ``spec_verify_tree_ex``.  ``workspace``:
+    None allocates (with torch) the bytes the list walk needs, if any; False
+    runs the walk over the rows; a uint8 tensor is used as given.  Target and draft
     [B, N+1, V] (one row per node, node 0 the verified context), tokens and
     parents [B, N] int32 (node n at index n - 1), uniforms [B, N+1] fp32,
     temperature [B] fp32 or None; optional outputs out_nodes [B, N+1] int32,
@@ -290,11 +309,19 @@ def verify_tree(target, draft, tokens, parents, uniforms=None, temperature=None,
     _check_cuda(dev)
     out_tokens = torch.empty((B, n1), dtype=torch.int32, device=dev)
     out_n = torch.empty((B,), dtype=torch.int32, device=dev)
-    st = spec_verify_tree(target, None if greedy else draft, tokens, parents, None if greedy else uniforms, B, N, V,
-                          None if greedy else temperature, top_k, mode, out_tokens, out_n, out_nodes,
-                          None if greedy else out_p, None if greedy else out_q, stream)
+    if workspace is None:
+        need = spec_verify_tree_workspace_size(B, N, V, top_k, mode)
+        workspace = torch.empty((need,), dtype=torch.uint8, device=dev) if need else False
+    if workspace is False:
+        workspace = None
+    elif workspace is not None:
+        _check(workspace, "workspace", (workspace.dtype,), workspace.numel(), dev)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = spec_verify_tree_ex(target, None if greedy else draft, tokens, parents, None if greedy else uniforms, B, N, V,
+                             None if greedy else temperature, top_k, mode, out_tokens, out_n, out_nodes,
+                             None if greedy else out_p, None if greedy else out_q, workspace, wbytes, stream)
     if st != SV_OK:
-        raise SpecVerifyError(st, "spec_verify_tree")
+        raise SpecVerifyError(st, "spec_verify_tree_ex")
     return out_tokens, out_n
 
 

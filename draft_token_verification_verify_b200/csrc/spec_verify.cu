@@ -250,6 +250,7 @@ using ResFn = void (*)(sv::ResidParams);
 using ProcsFn = void (*)(sv::ProcsParams);
 using NucFn = void (*)(sv::NucParams);
 using TreeFn = void (*)(sv::TreeParams);
+using TreeListFn = void (*)(sv::TreeListParams);
 
 template <int DT, int NT, bool PROC>
 RowsFn rows_for_mode(int mode) {
@@ -768,13 +769,53 @@ void* static_scratch(int dev) {
 
 }  // namespace
 
+// The list walk of tree verification: the streaming pass over the trees'
+// rows must produce one chunk per row and (stochastic) kept lists, or
+// (greedy) per-row argmax records.  Workspace: target and draft records and
+// lists, or the greedy records, and one flag per sequence.
+struct TreePlan {
+    bool fast = false;
+    Plan k1;
+    size_t off_ct = 0, off_lt = 0, off_cd = 0, off_ld = 0, off_gt = 0, off_done = 0, ws_bytes = 0;
+};
+
+void tree_plan(const DeviceInfo& dev, int B, int N, int V, int dt, bool greedy, int K, TreePlan* out) {
+    TreePlan t;
+    if (greedy || K > 0) {
+        Plan p;
+        if (make_plan(dev, B, N, V, dt, greedy, K, nullptr, 0, &p) == SV_OK && p.nch == 1 &&
+            p.mode == (greedy ? sv::MODE_GREEDY : sv::MODE_TOPK) && p.kcap <= sv::TREE_LIST_CAP) {
+            const size_t rows = static_cast<size_t>(B) * (N + 1);
+            t.fast = true;
+            t.k1 = p;
+            size_t o = 0;
+            if (greedy) {
+                t.off_gt = o;
+                o = round_up(o + rows * p.nseg * sizeof(sv::SegRec), 256);
+            } else {
+                t.off_ct = o;
+                o = round_up(o + rows * sizeof(sv::ChunkRec), 256);
+                t.off_lt = o;
+                o = round_up(o + rows * p.kcap * sizeof(sv::Cand), 256);
+                t.off_cd = o;
+                o = round_up(o + rows * sizeof(sv::ChunkRec), 256);
+                t.off_ld = o;
+                o = round_up(o + rows * p.kcap * sizeof(sv::Cand), 256);
+            }
+            t.off_done = o;
+            t.ws_bytes = round_up(o + static_cast<size_t>(B) * sizeof(int), 256);
+        }
+    }
+    *out = t;
+}
+
 extern "C" {
 
-sv_status_t spec_verify_tree(const void* target_logits, const void* draft_logits, const int32_t* tokens,
-                             const int32_t* parents, const float* uniforms, int B, int N, int V,
-                             const float* temperature, int top_k, int mode, int32_t* out_tokens,
-                             int32_t* out_n_accepted, int32_t* out_nodes, float* out_p, float* out_q,
-                             void* stream) {
+sv_status_t spec_verify_tree_ex(const void* target_logits, const void* draft_logits, const int32_t* tokens,
+                                const int32_t* parents, const float* uniforms, int B, int N, int V,
+                                const float* temperature, int top_k, int mode, int32_t* out_tokens,
+                                int32_t* out_n_accepted, int32_t* out_nodes, float* out_p, float* out_q,
+                                void* workspace, size_t workspace_bytes, void* stream) {
     bool greedy = false;
     int dt = 0;
     if (B <= 0 || N < 1 || N > sv::TREE_MAX_NODES || V < 1 || top_k < 0) return SV_ERR_INVALID_ARG;
@@ -789,9 +830,93 @@ sv_status_t spec_verify_tree(const void* target_logits, const void* draft_logits
         !aligned(out_tokens, 4) || !aligned(out_n_accepted, 4) || (out_nodes && !aligned(out_nodes, 4)) ||
         (out_p && !aligned(out_p, 4)) || (out_q && !aligned(out_q, 4)))
         return SV_ERR_INVALID_ARG;
+    if (workspace && !aligned(workspace, 16)) return SV_ERR_INVALID_ARG;
     if (V > sv::TREE_SEG * sv::TREE_MAX_SEG) return SV_ERR_UNSUPPORTED;
     int dev = 0;
-    if (!device_info(&dev)) return SV_ERR_UNSUPPORTED;
+    const DeviceInfo* info = device_info(&dev);
+    if (!info) return SV_ERR_UNSUPPORTED;
+    const int K = (!greedy && top_k > 0 && top_k < V) ? top_k : 0;
+    TreePlan tp;
+    tree_plan(*info, B, N, V, dt, greedy, K, &tp);
+    const bool fast = workspace && tp.fast && workspace_bytes >= tp.ws_bytes;
+    if (workspace && tp.fast && workspace_bytes < tp.ws_bytes) return SV_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int* done = nullptr;
+    if (fast) {
+        const Plan& p = tp.k1;
+        sv_status_t s = set_attrs(dev, dt, p.nt1, p.mode, false);
+        if (s != SV_OK) return s;
+        auto* base = static_cast<unsigned char*>(workspace);
+        done = reinterpret_cast<int*>(base + tp.off_done);
+        sv::RowsParams r;
+        std::memset(&r, 0, sizeof r);
+        r.B = B;
+        r.k = N;  // rows b*(N+1) + n: the sequence of a row is row / (N+1)
+        r.V = V;
+        r.top_k = K;
+        r.temperature = greedy ? nullptr : temperature;
+        r.nseg = p.nseg;
+        r.spc = p.spc;
+        r.nch = p.nch;
+        r.stages = p.stages;
+        r.lcap = p.lcap;
+        r.kcap = p.kcap;
+        r.timeout_ns = kDefaultTimeoutNs;
+        r.procs_div = 1;
+        int slot = 0;
+        RowsFn f1 = pick_rows(dt, p.nt1, p.mode, false, &slot);
+        cudaLaunchConfig_t c1;
+        std::memset(&c1, 0, sizeof c1);
+        c1.gridDim = dim3(static_cast<unsigned>(static_cast<long long>(B) * (N + 1)), 1, 1);
+        c1.blockDim = dim3(p.nt1 + 32, 1, 1);
+        c1.dynamicSmemBytes = p.smem1;
+        c1.stream = st;
+        // the streaming pass over the target rows, then over the draft rows
+        for (int side = 0; side < (greedy ? 1 : 2); ++side) {
+            r.target = side ? draft_logits : target_logits;
+            r.segs = reinterpret_cast<sv::SegRec*>(base + tp.off_gt);
+            r.chunks = reinterpret_cast<sv::ChunkRec*>(base + (side ? tp.off_cd : tp.off_ct));
+            r.cands = reinterpret_cast<sv::Cand*>(base + (side ? tp.off_ld : tp.off_lt));
+            if (cudaLaunchKernelEx(&c1, f1, r) != cudaSuccess) {
+                cudaGetLastError();
+                return SV_ERR_CUDA;
+            }
+        }
+        sv::TreeListParams lp;
+        std::memset(&lp, 0, sizeof lp);
+        lp.ct = reinterpret_cast<sv::ChunkRec*>(base + tp.off_ct);
+        lp.lt = reinterpret_cast<sv::Cand*>(base + tp.off_lt);
+        lp.cd = reinterpret_cast<sv::ChunkRec*>(base + tp.off_cd);
+        lp.ld = reinterpret_cast<sv::Cand*>(base + tp.off_ld);
+        lp.gt = reinterpret_cast<sv::SegRec*>(base + tp.off_gt);
+        lp.nseg = p.nseg;
+        lp.kcap = p.kcap;
+        lp.tokens = tokens;
+        lp.parents = parents;
+        lp.uniforms = greedy ? nullptr : uniforms;
+        lp.temperature = greedy ? nullptr : temperature;
+        lp.B = B;
+        lp.N = N;
+        lp.V = V;
+        lp.greedy = greedy ? 1 : 0;
+        lp.out_tokens = out_tokens;
+        lp.out_n = out_n_accepted;
+        lp.out_nodes = out_nodes;
+        lp.out_p = greedy ? nullptr : out_p;
+        lp.out_q = greedy ? nullptr : out_q;
+        lp.done = done;
+        cudaLaunchConfig_t cl2;
+        std::memset(&cl2, 0, sizeof cl2);
+        cl2.gridDim = dim3(static_cast<unsigned>(B), 1, 1);
+        cl2.blockDim = dim3(sv::TREE_LIST_NT, 1, 1);
+        cl2.stream = st;
+        TreeListFn fl = sv::sv_tree_list_kernel;
+        if (cudaLaunchKernelEx(&cl2, fl, lp) != cudaSuccess) {
+            cudaGetLastError();
+            return SV_ERR_CUDA;
+        }
+    }
+    // the row walk: every sequence, or those the list walk left
     sv::TreeParams t;
     std::memset(&t, 0, sizeof t);
     t.target = target_logits;
@@ -803,24 +928,48 @@ sv_status_t spec_verify_tree(const void* target_logits, const void* draft_logits
     t.B = B;
     t.N = N;
     t.V = V;
-    t.top_k = (!greedy && top_k > 0 && top_k < V) ? top_k : 0;
+    t.top_k = K;
     t.greedy = greedy ? 1 : 0;
     t.out_tokens = out_tokens;
     t.out_n = out_n_accepted;
     t.out_nodes = out_nodes;
     t.out_p = greedy ? nullptr : out_p;
     t.out_q = greedy ? nullptr : out_q;
+    t.done = done;
     cudaLaunchConfig_t ct;
     std::memset(&ct, 0, sizeof ct);
     ct.gridDim = dim3(static_cast<unsigned>(B), 1, 1);
     ct.blockDim = dim3(sv::TREE_NT, 1, 1);
-    ct.stream = static_cast<cudaStream_t>(stream);
+    ct.stream = st;
     TreeFn ft = dt ? sv::sv_tree_kernel<1> : sv::sv_tree_kernel<0>;
     if (cudaLaunchKernelEx(&ct, ft, t) != cudaSuccess) {
         cudaGetLastError();
         return SV_ERR_CUDA;
     }
     return SV_OK;
+}
+
+sv_status_t spec_verify_tree(const void* target_logits, const void* draft_logits, const int32_t* tokens,
+                             const int32_t* parents, const float* uniforms, int B, int N, int V,
+                             const float* temperature, int top_k, int mode, int32_t* out_tokens,
+                             int32_t* out_n_accepted, int32_t* out_nodes, float* out_p, float* out_q,
+                             void* stream) {
+    return spec_verify_tree_ex(target_logits, draft_logits, tokens, parents, uniforms, B, N, V, temperature, top_k,
+                               mode, out_tokens, out_n_accepted, out_nodes, out_p, out_q, nullptr, 0, stream);
+}
+
+size_t spec_verify_tree_workspace_size(int B, int N, int V, int top_k, int mode) {
+    bool greedy = false;
+    int dt = 0;
+    if (B <= 0 || N < 1 || N > sv::TREE_MAX_NODES || V < 1 || top_k < 0) return 0;
+    if (!decode_mode(mode, &greedy, &dt)) return 0;
+    int dev = 0;
+    const DeviceInfo* info = device_info(&dev);
+    if (!info) return 0;
+    const int K = (!greedy && top_k > 0 && top_k < V) ? top_k : 0;
+    TreePlan tp;
+    tree_plan(*info, B, N, V, dt, greedy, K, &tp);
+    return tp.fast ? tp.ws_bytes : 0;
 }
 
 sv_status_t spec_verify_ex(const void* target_logits, const void* draft_logits, const int32_t* draft_tokens,

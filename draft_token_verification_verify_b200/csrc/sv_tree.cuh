@@ -12,7 +12,15 @@
 // is drawn from R by the inverse CDF with the last uniform.  Greedy: the first
 // child whose token is the node's lowest-index argmax, else that argmax.
 //
-// Only the rows of visited nodes are read.  Per visited node the CTA streams
+// Two paths.  With top-k (or greedy) and a workspace, the streaming pass (K1)
+// first runs over every target and draft row of the trees, and the list walk
+// (sv_tree_list_kernel) takes each visited node's statistics and kept list
+// from its records: the probabilities, every residual and the final draw live
+// on the kept lists, so the walk reads no logits.  A sequence whose records
+// are incomplete (a list that overflowed, a wait that ran out) and every
+// sequence of the other cases go through the row walk (sv_tree_kernel).
+//
+// Row walk: only the rows of visited nodes are read.  Per visited node the CTA streams
 // the target and draft rows: their maxima (and raw NaN / +inf), the exact
 // top-k threshold by a radix select over order-preserving keys when top-k is
 // on, and the normalisers; one more pass over the pair per rejection (the
@@ -24,6 +32,7 @@
 
 #include "sv_common.cuh"
 #include "sv_nucleus.cuh"  // load_vec
+#include "sv_rows.cuh"     // record flags
 
 namespace sv {
 
@@ -50,6 +59,7 @@ struct TreeParams {
     int32_t* out_nodes;        // [B][N+1] or null
     float* out_p;              // [B][N] or null: R(t_c) of each tested child, NaN if untested
     float* out_q;              // [B][N] or null: q(t_c), NaN if untested
+    const int* done;           // [B] or null: sequences the list walk has finished (skipped here)
 };
 
 struct TreeRow {
@@ -85,6 +95,7 @@ __global__ void __launch_bounds__(TREE_NT, 1) sv_tree_kernel(const TreeParams P)
     __shared__ TreeCtl S;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const long long b = blockIdx.x;
+    if (P.done && P.done[b]) return;  // uniform over the CTA
     const int N = P.N, V = P.V, K = P.top_k;
     const int nvec = (V + VEC - 1) / VEC;
     const bool greedy = P.greedy != 0;
@@ -482,6 +493,232 @@ __global__ void __launch_bounds__(TREE_NT, 1) sv_tree_kernel(const TreeParams P)
         }
     }
     if (tid == 0) P.out_n[b] = err ? -1 : depth;
+}
+
+constexpr int TREE_LIST_NT = 128;
+constexpr int TREE_LIST_CAP = 1024;  // kept entries per row (the planner's largest kcap)
+
+struct TreeListParams {
+    const ChunkRec* ct;        // [B*(N+1)] target rows' records (one chunk per row)
+    const Cand* lt;            // [B*(N+1)][kcap] their kept lists, by index
+    const ChunkRec* cd;        // draft rows
+    const Cand* ld;
+    const SegRec* gt;          // greedy: [B*(N+1)][nseg], chunk 0 of each row
+    int nseg;
+    int kcap;
+    const int32_t* tokens;
+    const int32_t* parents;
+    const float* uniforms;
+    const float* temperature;
+    long long B;
+    int N;
+    int V;
+    int greedy;
+    int32_t* out_tokens;
+    int32_t* out_n;
+    int32_t* out_nodes;
+    float* out_p;
+    float* out_q;
+    int* done;                 // [B]: 1 = finished here, 0 = left to the row walk
+};
+
+struct __align__(16) TreeListCtl {
+    Cand lt[TREE_LIST_CAP];
+    Cand ld[TREE_LIST_CAP];
+    float pw[TREE_LIST_CAP];   // p of the target list's entries
+    float qw[TREE_LIST_CAP];   // q of the same tokens
+    int tok[TREE_MAX_NODES];
+    int par[TREE_MAX_NODES];
+    float W[TREE_MAX_NODES];
+    float red[TREE_LIST_NT / 32];
+    int err;
+    int slow;
+    int token;
+};
+
+// One CTA per sequence: the tree walk on the kept lists of the streaming
+// pass (top-k) or on its per-row argmax (greedy).  Same rule and outputs as
+// sv_tree_kernel.
+__global__ void __launch_bounds__(TREE_LIST_NT) sv_tree_list_kernel(const TreeListParams P) {
+    constexpr int NT = TREE_LIST_NT, NW = NT / 32;
+    __shared__ TreeListCtl S;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const long long b = blockIdx.x;
+    const int N = P.N, V = P.V;
+    const bool greedy = P.greedy != 0;
+    const float* u = greedy ? nullptr : P.uniforms + b * (N + 1);
+    float T = 1.f;
+    if (!greedy && P.temperature) T = P.temperature[b];
+    const float c = (T > 0.f && T != POS_INF) ? LOG2E / T : 1.f;
+    if (tid == 0) {
+        S.err = 0;
+        S.slow = 0;
+    }
+    __syncthreads();
+    for (int i = tid; i < N; i += NT) {
+        const int t = P.tokens[b * N + i], p = P.parents[b * N + i];
+        S.tok[i] = t;
+        S.par[i] = p;
+        if (t < 0 || t >= V || p < 0 || p > i) S.err = 1;
+        if (P.out_p) P.out_p[b * N + i] = __int_as_float(0x7fc00000);
+        if (P.out_q) P.out_q[b * N + i] = __int_as_float(0x7fc00000);
+    }
+    if (!greedy) {
+        if (tid == 0 && !(T > 0.f && T != POS_INF)) S.err = 1;
+        for (int i = tid; i <= N; i += NT)
+            if (!(u[i] >= 0.f && u[i] < 1.f)) S.err = 1;
+    }
+    __syncthreads();
+    auto block_sum = [&](float v) -> float {
+        v = warp_sum(v);
+        if (lane == 0) S.red[warp] = v;
+        __syncthreads();
+        float s = 0.f;
+        for (int w = 0; w < NW; ++w) s += S.red[w];
+        __syncthreads();
+        return s;
+    };
+    // entry of token x in a list sorted by index, or -1
+    auto find = [](const Cand* L, int n, int x) {
+        int lo = 0, hi = n - 1;
+        while (lo <= hi) {
+            const int mid = (lo + hi) >> 1;
+            const int y = L[mid].i;
+            if (y == x) return mid;
+            if (y < x) lo = mid + 1; else hi = mid - 1;
+        }
+        return -1;
+    };
+
+    int a = 0, depth = 0, y = -1;
+    int err = S.err, slow = 0;
+    while (!err) {
+        const long long r = b * (N + 1) + a;
+        int next = 0;
+        if (greedy) {
+            const SegRec g = P.gt[r * P.nseg];
+            if (g.flags & (REC_TIMEOUT | REC_DIAG)) {
+                slow = 1;
+                break;
+            }
+            if (!(g.m == g.m) || g.m == POS_INF || !(g.m > NEG_INF) || g.arg < 0) {
+                err = 1;
+                break;
+            }
+            for (int ch = a + 1; ch <= N && !next; ++ch)
+                if (S.par[ch - 1] == a && S.tok[ch - 1] == g.arg) next = ch;
+            if (!next) {
+                y = g.arg;
+                break;
+            }
+        } else {
+            const ChunkRec ct = P.ct[r], cd = P.cd[r];
+            if ((ct.flags | cd.flags) & (REC_TIMEOUT | REC_OVERFLOW | REC_DIAG)) {
+                slow = 1;
+                break;
+            }
+            if (!(ct.m == ct.m) || ct.m == POS_INF || !(ct.m > NEG_INF) || !(cd.m == cd.m) || cd.m == POS_INF ||
+                !(cd.m > NEG_INF) || !(ct.s > 0.f) || !(cd.s > 0.f)) {
+                err = 1;
+                break;
+            }
+            const int nt = min(ct.n, TREE_LIST_CAP), nd = min(cd.n, TREE_LIST_CAP);
+            const float mt = ct.m * c, md = cd.m * c, it = 1.f / ct.s, id = 1.f / cd.s;
+            for (int i = tid; i < nt; i += NT) S.lt[i] = P.lt[r * P.kcap + i];
+            for (int i = tid; i < nd; i += NT) S.ld[i] = P.ld[r * P.kcap + i];
+            __syncthreads();
+            for (int i = tid; i < nt; i += NT) {
+                S.pw[i] = ex2(fmaf(S.lt[i].v, c, -mt)) * it;
+                const int j = find(S.ld, nd, S.lt[i].i);
+                S.qw[i] = j >= 0 ? ex2(fmaf(S.ld[j].v, c, -md)) * id : 0.f;
+            }
+            __syncthreads();
+            int levels = 0;
+            auto cur = [&](int i) {  // current distribution at target-list entry i
+                float rr = S.pw[i];
+                for (int l = 0; l < levels; ++l) rr = fmaxf(rr - S.qw[i], 0.f) / S.W[l];
+                return rr;
+            };
+            for (int ch = a + 1; ch <= N; ++ch) {
+                if (S.par[ch - 1] != a) continue;
+                const int x = S.tok[ch - 1];
+                const int ip = find(S.lt, nt, x), iq = find(S.ld, nd, x);
+                const float rr = ip >= 0 ? cur(ip) : 0.f;
+                const float qv = iq >= 0 ? ex2(fmaf(S.ld[iq].v, c, -md)) * id : 0.f;
+                if (tid == 0) {
+                    if (P.out_p) P.out_p[b * N + ch - 1] = rr;
+                    if (P.out_q) P.out_q[b * N + ch - 1] = qv;
+                }
+                if (u[ch - 1] * qv < rr) {
+                    next = ch;
+                    break;
+                }
+                float acc = 0.f;
+                for (int i = tid; i < nt; i += NT) acc += fmaxf(cur(i) - S.qw[i], 0.f);
+                const float W = block_sum(acc);
+                if (W > 0.f) {
+                    if (tid == 0) S.W[levels] = W;
+                    __syncthreads();
+                    ++levels;
+                }
+            }
+            if (!next) {
+                // inverse CDF over the target list in index order (warp 0)
+                if (warp == 0) {
+                    float Wt = 0.f;
+                    for (int i0 = 0; i0 < nt; i0 += 32) {
+                        const float w = i0 + lane < nt ? cur(i0 + lane) : 0.f;
+                        Wt += __shfl_sync(0xffffffffu, warp_incl_scan(w, lane), 31);
+                    }
+                    const float xx = u[N] * Wt;
+                    float carry = 0.f;
+                    int token = -1, lastp = -1;
+                    for (int i0 = 0; i0 < nt; i0 += 32) {
+                        const float w = i0 + lane < nt ? cur(i0 + lane) : 0.f;
+                        const float incl = warp_incl_scan(w, lane);
+                        const unsigned hit = __ballot_sync(0xffffffffu, i0 + lane < nt && carry + incl > xx);
+                        const unsigned pos = __ballot_sync(0xffffffffu, w > 0.f);
+                        if (pos) lastp = i0 + 31 - __clz(pos);
+                        if (hit) {
+                            token = S.lt[i0 + __ffs(hit) - 1].i;
+                            break;
+                        }
+                        carry += __shfl_sync(0xffffffffu, incl, 31);
+                    }
+                    if (lane == 0) S.token = token >= 0 ? token : (lastp >= 0 ? S.lt[lastp].i : -1);
+                }
+                __syncthreads();
+                y = S.token;
+                if (y < 0) err = 1;
+                break;
+            }
+            __syncthreads();  // the lists are reloaded for the next node
+        }
+        if (tid == 0) {
+            if (P.out_nodes) P.out_nodes[b * (N + 1) + depth] = next;
+            P.out_tokens[b * (N + 1) + depth] = S.tok[next - 1];
+        }
+        ++depth;
+        a = next;
+    }
+    __syncthreads();
+    if (slow) {  // the row walk takes the whole sequence
+        if (tid == 0) P.done[b] = 0;
+        return;
+    }
+    for (int i = tid; i <= N; i += NT) {
+        if (err || i > depth) {
+            P.out_tokens[b * (N + 1) + i] = -1;
+            if (P.out_nodes) P.out_nodes[b * (N + 1) + i] = -1;
+        } else if (i == depth) {
+            P.out_tokens[b * (N + 1) + i] = y;
+            if (P.out_nodes) P.out_nodes[b * (N + 1) + i] = -1;
+        }
+    }
+    if (tid == 0) {
+        P.out_n[b] = err ? -1 : depth;
+        P.done[b] = 1;
+    }
 }
 
 }  // namespace sv

@@ -291,6 +291,27 @@ SV_API sv_status_t spec_verify_tree(const void* target_logits, const void* draft
                                     int32_t* out_tokens, int32_t* out_n_accepted,
                                     int32_t* out_nodes, float* out_p, float* out_q, void* stream);
 
+/*
+ * spec_verify_tree with a caller workspace (device memory, 16-byte aligned,
+ * at least spec_verify_tree_workspace_size bytes; NULL: as spec_verify_tree).
+ * With top-k (0 < top_k < V, up to 256) or greedy, and a workspace, the
+ * streaming pass first reads every target and draft row of the trees once and
+ * the walk then works on the kept lists (or the per-row argmax) alone; rows
+ * whose kept list overflowed fall back to the walk over the rows.  Same
+ * results.  The workspace is not read before it is written.
+ */
+SV_API sv_status_t spec_verify_tree_ex(const void* target_logits, const void* draft_logits,
+                                       const int32_t* tokens, const int32_t* parents,
+                                       const float* uniforms, int B, int N, int V,
+                                       const float* temperature, int top_k, int mode,
+                                       int32_t* out_tokens, int32_t* out_n_accepted,
+                                       int32_t* out_nodes, float* out_p, float* out_q,
+                                       void* workspace, size_t workspace_bytes, void* stream);
+
+/* Workspace bytes for spec_verify_tree_ex's list walk; 0 when the call has no
+ * list walk (no top-k) or on invalid arguments / no usable device. */
+SV_API size_t spec_verify_tree_workspace_size(int B, int N, int V, int top_k, int mode);
+
 /* Static description of a status code. */
 SV_API const char* spec_verify_status_string(sv_status_t status);
 

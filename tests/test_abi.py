@@ -30,7 +30,7 @@ def test_header_declares_entry_points():
     assert declared_functions() == sorted([
         "spec_sample", "spec_sample_ex", "spec_sample_workspace_size", "spec_verify", "spec_verify_ex",
         "spec_verify_pool_allocations", "spec_verify_static", "spec_verify_status_string", "spec_verify_tree",
-        "spec_verify_version", "spec_verify_workspace_size"])
+        "spec_verify_tree_ex", "spec_verify_tree_workspace_size", "spec_verify_version", "spec_verify_workspace_size"])
 
 
 
@@ -45,9 +45,19 @@ def test_library_exports_every_declared_symbol(L):
     assert exported == set(declared_functions())
 
 
+def _no_gpu():
+    """Calls below pass placeholder device pointers that get past the argument
+    checks: they may only run where no GPU can launch anything."""
+    import torch
+
+    if torch.cuda.is_available():
+        pytest.skip("placeholder device pointers: runs only without a GPU")
+
+
 def test_no_pool_allocation_without_a_launch(L):
     """Size queries, refused calls and calls given a workspace never take a
     workspace from the library's pool (here, without a GPU, none launches)."""
+    _no_gpu()
     a0 = sv.spec_verify_pool_allocations()
     sv.spec_verify_workspace_size(64, 4, 151936, 50, 0)
     sv.spec_sample_workspace_size(8, 1000, 0, 0)
@@ -320,7 +330,16 @@ def test_tree_invalid_arguments(L, kw):
 
 
 def test_tree_greedy_needs_no_draft(L):
+    _no_gpu()
     # greedy reads neither the draft logits nor the uniforms: NULL passes the checks
     # (on a machine without a GPU the call then stops at the device: unsupported)
     st = sv.spec_verify_tree(P, None, P, P, None, 2, 3, 100, None, 0, sv.SV_MODE_GREEDY, P, P, stream=0)
     assert st in (sv.SV_OK, sv.SV_ERR_UNSUPPORTED)
+
+
+def test_tree_ex_checks_the_workspace(L):
+    st = sv.spec_verify_tree_ex(P, P, P, P, P, 2, 3, 100, None, 5, 0, P, P, workspace=P + 8, workspace_bytes=1 << 20,
+                                stream=0)
+    assert st == sv.SV_ERR_INVALID_ARG  # not 16-byte aligned
+    assert sv.spec_verify_tree_workspace_size(0, 3, 100, 5, 0) == 0
+    assert sv.spec_verify_tree_workspace_size(2, 0, 100, 5, 0) == 0

@@ -53,7 +53,7 @@ def _tree_case(name, seed, B, N, shape, **over):
     return case, target, draft, np.asarray(toks, np.int32).reshape(B, N), parents.astype(np.int32), u
 
 
-def _run(case, target, draft, toks, parents, u, greedy):
+def _run(case, target, draft, toks, parents, u, greedy, path="list"):
     import torch
 
     import draft_token_verification_verify_b200 as sv
@@ -66,16 +66,17 @@ def _run(case, target, draft, toks, parents, u, greedy):
     tok, n = sv.verify_tree(to_dev(target), None if greedy else to_dev(draft), torch.from_numpy(toks).to(dev),
                             torch.from_numpy(parents).to(dev), None if greedy else to_dev(u),
                             None if greedy else to_dev(case.temperature), case.top_k, greedy=greedy,
-                            out_nodes=nodes, out_p=None if greedy else p, out_q=None if greedy else q)
+                            out_nodes=nodes, out_p=None if greedy else p, out_q=None if greedy else q,
+                            workspace=None if path == "list" else False)
     torch.cuda.synchronize()
     return tok.cpu().numpy(), n.cpu().numpy(), nodes.cpu().numpy(), p.cpu().numpy(), q.cpu().numpy()
 
 
-def _check(case, target, draft, toks, parents, u, max_flag_frac=0.05):
+def _check(case, target, draft, toks, parents, u, max_flag_frac=0.05, path="list"):
     greedy = case.mode == "greedy"
     ref = oracle.verify_tree(target, draft, toks, parents, u, None if greedy else case.temperature, case.top_k,
                              greedy=greedy)
-    tok, n, nodes, p, q = _run(case, target, draft, toks, parents, u, greedy)
+    tok, n, nodes, p, q = _run(case, target, draft, toks, parents, u, greedy, path)
     B, N = toks.shape
     flagged = exact = 0
     for b in range(B):
@@ -101,11 +102,15 @@ def _check(case, target, draft, toks, parents, u, max_flag_frac=0.05):
     return ref, (tok, n, nodes, p, q)
 
 
+PATHS = ["list", "rows"]  # the walk on the streaming pass's kept lists, or over the rows
+
+
+@pytest.mark.parametrize("path", PATHS)
 @pytest.mark.parametrize("shape", ["binary", "star", "mixed"])
-def test_batched_top_k_full_vocabulary(shape):
+def test_batched_top_k_full_vocabulary(shape, path):
     """bf16, V = 151,936, T = 0.7, top-k 50 (the batched workload's value model)."""
     case, t, d, toks, par, u = _tree_case("batched", 91, 16, 9, shape)
-    ref, _ = _check(case, t, d, toks, par, u)
+    ref, _ = _check(case, t, d, toks, par, u, path=path)
     assert ref.errors == 0
 
 
@@ -119,10 +124,11 @@ def test_single_full_vocabulary_no_top_k():
     _check(case, t, d, toks, par, u)
 
 
+@pytest.mark.parametrize("path", PATHS)
 @pytest.mark.parametrize("V", [3, 257, 30011])
-def test_ragged_and_tiny_vocabularies(V):
+def test_ragged_and_tiny_vocabularies(V, path):
     case, t, d, toks, par, u = _tree_case("batched", 94, 24, 6, "binary", V=V, top_k=min(5, V - 1))
-    _check(case, t, d, toks, par, u)
+    _check(case, t, d, toks, par, u, path=path)
 
 
 def test_chain_trees_match_chain_verification():
@@ -154,14 +160,28 @@ def test_chain_trees_match_chain_verification():
         assert int(n_t[b]) == int(n_c[b]) == j
 
 
+@pytest.mark.parametrize("path", PATHS)
 @pytest.mark.parametrize("shape", ["binary", "star"])
-def test_greedy_trees(shape):
+def test_greedy_trees(shape, path):
     case, t, d, toks, par, u = _tree_case("greedy", 96, 32, 7, shape, V=30011)
-    ref, _ = _check(case, t, d, toks, par, u)
+    ref, _ = _check(case, t, d, toks, par, u, path=path)
     assert ref.errors == 0
 
 
-def test_row_errors():
+def test_overflowing_kept_list_falls_back_to_the_rows():
+    """3,000 tied maxima in one target row: its kept list cannot hold them,
+    the list walk leaves the sequence to the walk over the rows."""
+    case, t, d, toks, par, u = _tree_case("batched", 99, 6, 4, "binary", V=30011)
+    t = t.copy()
+    row = t[2, 0]
+    top = row[np.argmax((row.astype(np.uint32) << 16).view(np.float32))]  # bf16 bits of the row maximum
+    t[2, 0, :3000] = top
+    ref, _ = _check(case, t, d, toks, par, u, path="list")
+    assert ref.n_accepted[2] >= 0
+
+
+@pytest.mark.parametrize("path", PATHS)
+def test_row_errors(path):
     case, t, d, toks, par, u = _tree_case("batched", 97, 6, 4, "binary", V=4099)
     t = t.copy()
     toks = toks.copy()
@@ -172,7 +192,7 @@ def test_row_errors():
     par[2, 0] = -1               # parent outside [0, n)
     u[3, 1] = 1.0                # uniform outside [0, 1)
     t[4, 0, 7] = 0x7fc0          # bf16 NaN in the root's target row (always read)
-    ref, (tok, n, *_rest) = _check(case, t, d, toks, par, u)
+    ref, (tok, n, *_rest) = _check(case, t, d, toks, par, u, path=path)
     assert list(ref.n_accepted[:5]) == [-1] * 5 and list(n[:5]) == [-1] * 5
     assert ref.n_accepted[5] >= 0 and n[5] >= 0
 
