@@ -638,6 +638,13 @@ def measure_tree(args, sv, dev, world, rank):
     torch.cuda.synchronize()
     sampler = ClockSampler(rank)
     sampler.start()
+    t_end = time.perf_counter() + getattr(args, "clock_window", 0.0)  # the same calls while clocks are sampled
+    i = 0
+    while time.perf_counter() < t_end:
+        for _ in range(16):
+            step(i)
+            i += 1
+        torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         torch.distributed.barrier()
