@@ -105,6 +105,8 @@ struct __align__(16) SeqCtl {
     float W;
     float c;
     NucCtl nuc;  // nucleus cut of a row resolved here (radix top-k rows)
+    float ftau[32];  // one-warp path with a nucleus: each row's cut and 1 / kept mass
+    float finv[32];
 };
 
 constexpr int SEQ_CTL_BYTES = (int)((sizeof(SeqCtl) + 127) / 128 * 128);
@@ -230,13 +232,48 @@ __global__ void __launch_bounds__(SEQ_NT, 3) sv_seq_kernel(const SeqParams P) {
     // Warp 0 alone finishes the sequence: lane r holds row r's statistics, the
     // decisions come from shuffles and a ballot, and the draw reads the kept
     // lists already in shared memory.  Same arithmetic as the block path below.
-    if (P.pre && nrows <= 32 && tp >= 1.f) {
+    if (P.pre && nrows <= 32) {
         const bool clean = tid >= nrows || (prec[tid].flags == 0 && prec[tid].m == prec[tid].m &&
                                             prec[tid].m != POS_INF && prec[tid].m != NEG_INF);
         if (__syncthreads_and(clean) && !S.err) {
+            const bool nucleus = tp < 1.f;
+            if (nucleus) {
+                // every warp: the nucleus over its rows' kept lists (the cut is the
+                // largest kept value whose tail mass reaches top_p), as the block path
+                for (int rr = warp; rr < nrows; rr += NW) {
+                    const Cand* L = plist + static_cast<size_t>(rr) * P.kcap;
+                    const int n = prec[rr].n;
+                    const float rm = prec[rr].m * c, ri = 1.f / prec[rr].s, rt = prec[rr].tau;
+                    float cand = NEG_INF;
+                    for (int e = lane; e < n; e += 32) {
+                        const float x = L[e].v;
+                        if (!(x >= rt)) continue;
+                        float mass = 0.f;
+                        for (int f = 0; f < n; ++f) {
+                            const float y = L[f].v;
+                            if (y >= x && y >= rt) mass += ex2(fmaf(y, c, -rm)) * ri;
+                        }
+                        if (mass >= tp) cand = fmaxf(cand, x);
+                    }
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) cand = fmaxf(cand, __shfl_xor_sync(0xffffffffu, cand, o));
+                    const float cut = fmaxf(cand, rt);
+                    float acc = 0.f;
+                    for (int e = lane; e < n; e += 32)
+                        if (L[e].v >= cut) acc += ex2(fmaf(L[e].v, c, -rm));
+                    acc = warp_sum(acc);
+                    if (lane == 0) {
+                        S.ftau[rr] = cut;
+                        S.finv[rr] = 1.f / acc;
+                    }
+                }
+                __syncthreads();
+            }
             if (warp != 0) return;
             const ChunkRec rec = prec[lane < nrows ? lane : 0];
-            const float msc = rec.m * c, invS = 1.f / rec.s, tau = rec.tau, zd = rec.zd;
+            const float msc = rec.m * c, zd = rec.zd;
+            const float invS = nucleus ? S.finv[lane < nrows ? lane : 0] : 1.f / rec.s;
+            const float tau = nucleus ? S.ftau[lane < nrows ? lane : 0] : rec.tau;
             // decisions: lane i < k holds target row i; draft row i is lane k+1+i
             int j = k;
             for (int i0 = 0; i0 < k; i0 += 32) {
@@ -260,9 +297,11 @@ __global__ void __launch_bounds__(SEQ_NT, 3) sv_seq_kernel(const SeqParams P) {
             // draw from the kept lists of position j
             const bool use_q0 = j < k;
             const float t_msc = __shfl_sync(0xffffffffu, msc, j), t_inv = __shfl_sync(0xffffffffu, invS, j);
+            const float t_cut = __shfl_sync(0xffffffffu, tau, j);
             const int nt = __shfl_sync(0xffffffffu, rec.n, j);
             const int jd = use_q0 ? k + 1 + j : 0;
             const float d_msc = __shfl_sync(0xffffffffu, msc, jd), d_inv = __shfl_sync(0xffffffffu, invS, jd);
+            const float d_cut = __shfl_sync(0xffffffffu, tau, jd);
             const int nd = use_q0 ? __shfl_sync(0xffffffffu, rec.n, jd) : 0;
             const Cand* lt = plist + static_cast<size_t>(j) * P.kcap;
             const Cand* ld = plist + static_cast<size_t>(jd) * P.kcap;
@@ -282,11 +321,12 @@ __global__ void __launch_bounds__(SEQ_NT, 3) sv_seq_kernel(const SeqParams P) {
             float W = 0.f;
             for (int attempt = 0; attempt < 2; ++attempt) {
                 for (int e = lane; e < nt; e += 32) {
-                    const float pt = ex2(fmaf(lt[e].v, c, -t_msc)) * t_inv;
+                    // entries below a row's threshold (a nucleus cut) weigh nothing
+                    const float pt = lt[e].v >= t_cut ? ex2(fmaf(lt[e].v, c, -t_msc)) * t_inv : 0.f;
                     float w = pt;
                     if (use_q) {
                         const int pd = find(lt[e].i);
-                        const float q = pd >= 0 ? ex2(fmaf(ld[pd].v, c, -d_msc)) * d_inv : 0.f;
+                        const float q = (pd >= 0 && ld[pd].v >= d_cut) ? ex2(fmaf(ld[pd].v, c, -d_msc)) * d_inv : 0.f;
                         w = fmaxf(pt - q, 0.f);
                     }
                     wv[e] = w;
