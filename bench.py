@@ -683,6 +683,14 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     sv.lib()
 
+    if args.tree_only:
+        r = measure_tree(args, sv, dev, world, local)
+        if world > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+        if rank == 0:
+            print(json.dumps(r), flush=True)
+        return 0
     name = args.workload
     head = measure_workload(name, args, sv, dev, world, rank, local, e2e_leg=not (args.no_e2e or args.feature),
                             feature=args.feature)
@@ -762,6 +770,8 @@ def main():
                     help="also time the headline's steps replayed from a CUDA graph")
     ap.add_argument("--feature", choices=sorted({f for _, f in FEATURES}), default=None,
                     help="profile a feature alone: --workload with these options (no e2e or CPU leg)")
+    ap.add_argument("--tree-only", action="store_true",
+                    help="measure only the tree-verification line (one JSON line; for profiling)")
     ap.add_argument("--headline-only", action="store_true",
                     help="measure only --workload (default: every workload, the headline first)")
     args = ap.parse_args()
