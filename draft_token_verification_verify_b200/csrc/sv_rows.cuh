@@ -527,7 +527,47 @@ __global__ void __launch_bounds__(NT + 32, RowsOcc<NT, MODE>::value) sv_rows_ker
             auto jof = [&](int i) { return i < VPT ? tid + i * NT : TV + tid; };
             float vm[VPT + 1];
             const bool tile_full = ok && g.e0 == g.lo && g.nvec == TV && g.hi - g.lo == TV * VEC;
-            if constexpr (PROC) {
+            // softmax with processors: this thread's running maximum of z*c and
+            // sum of 2^(z*c - maximum) over its processed elements, one pass
+            float pm = NEG_INF, ps = 0.f;
+            (void)pm;
+            (void)ps;
+            if constexpr (PROC && MODE == MODE_SOFTMAX) {
+#pragma unroll 1
+                for (int i = 0; i <= VPT; ++i) {
+                    const int j = jof(i);
+                    if (!(ok && j < g.nvec)) continue;
+                    const uint4 raw = vec_at(j);
+                    const int e = g.e0 + j * VEC;
+                    const bool full = e >= g.lo && e + VEC <= g.hi;
+                    const float rm = full ? vmax_nan<DT>(raw) : vmax_masked(j);
+                    if (!(rm == rm) || rm == POS_INF) rawbad = true;
+                    float v[VEC];
+                    if (bits_at(spen, e, false) == 0u) {
+                        uint32_t ab = bits_at(sallow, e, true);
+#pragma unroll
+                        for (int q = 0; q < VEC; ++q)
+                            if (!valid(e + q)) ab &= ~(1u << q);
+                        unpack<DT>(mask_neg_inf<DT>(raw, ab), v);
+                    } else {
+                        proc_vals(raw, e, v);
+                    }
+                    float vmx = NEG_INF;
+#pragma unroll
+                    for (int q = 0; q < VEC; ++q) vmx = fmaxf(vmx, v[q]);
+                    const float mc = vmx * cscale;
+                    if (mc > pm) {
+                        ps = pm > NEG_INF ? ps * ex2(pm - mc) : 0.f;
+                        pm = mc;
+                    }
+                    if (pm > NEG_INF) {
+#pragma unroll
+                        for (int q = 0; q < VEC; ++q) ps += ex2(fmaf(v[q], cscale, -pm));
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i <= VPT; ++i) vm[i] = NEG_INF;
+            } else if constexpr (PROC) {
                 // one copy of the processing code (a rolled loop); the maxima
                 // come back to registers through this thread's own slots
                 const float skip_below = (MODE == MODE_TOPK && pen_theta >= 1.f) ? theta : NEG_INF;
@@ -577,6 +617,16 @@ __global__ void __launch_bounds__(NT + 32, RowsOcc<NT, MODE>::value) sv_rows_ker
                     for (int o = 16; o > 0; o >>= 1) my = min(my, __shfl_xor_sync(0xffffffffu, my, o));
                     wbest = wtm;
                     widx = my;
+                }
+            } else if constexpr (MODE == MODE_SOFTMAX && PROC) {
+                // the lanes' running (maximum, sum) pairs, combined
+                float m = pm, sm = ps;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1)
+                    ms_combine(m, sm, __shfl_xor_sync(0xffffffffu, m, o), __shfl_xor_sync(0xffffffffu, sm, o));
+                if (lane == 0) {
+                    red_m[t * NW + warp] = m;
+                    red_s[t * NW + warp] = sm;
                 }
             } else if constexpr (MODE == MODE_SOFTMAX) {
                 // one maximum per warp; pass B sums 2^(z*c - m) with two accumulators
