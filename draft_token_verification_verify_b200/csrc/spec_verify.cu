@@ -551,9 +551,17 @@ sv_status_t run(const Call& cl, void* workspace, size_t workspace_bytes, const s
             np.theta = r.theta;
             np.W4 = r.W4;
             np.out = reinterpret_cast<sv::NucRec*>(base + p.off_nuc);
-            // few rows: a cluster of up to 8 CTAs shares each row
+            // few rows: a cluster of up to 16 CTAs shares each row (16 is a
+            // non-portable size: the kernel opts in, and 8 is used if refused)
+            NucFn fn = cl.dt ? sv::sv_nucleus_kernel<1> : sv::sv_nucleus_kernel<0>;
+            static std::once_flag nuc_once[2];
+            static bool nuc16[2] = {false, false};
+            std::call_once(nuc_once[cl.dt], [&] {
+                nuc16[cl.dt] = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
+                cudaGetLastError();
+            });
             int ncl = 1;
-            while (ncl < 8 && p.R * ncl < info->sms) ncl *= 2;
+            while (ncl < (nuc16[cl.dt] ? 16 : 8) && p.R * ncl < 2 * info->sms) ncl *= 2;
             cudaLaunchAttribute an[2];
             an[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
             an[0].val.programmaticStreamSerializationAllowed = 1;
@@ -568,8 +576,14 @@ sv_status_t run(const Call& cl, void* workspace, size_t workspace_bytes, const s
             cn.stream = st;
             cn.attrs = an;
             cn.numAttrs = 2;
-            NucFn fn = cl.dt ? sv::sv_nucleus_kernel<1> : sv::sv_nucleus_kernel<0>;
-            if (cudaLaunchKernelEx(&cn, fn, np) != cudaSuccess) {
+            cudaError_t le = cudaLaunchKernelEx(&cn, fn, np);
+            if (le != cudaSuccess && ncl > 8) {  // the larger cluster cannot be placed: 8
+                cudaGetLastError();
+                an[1].val.clusterDim.x = 8;
+                cn.gridDim = dim3(static_cast<unsigned>(p.R * 8), 1, 1);
+                le = cudaLaunchKernelEx(&cn, fn, np);
+            }
+            if (le != cudaSuccess) {
                 result = SV_ERR_CUDA;
                 break;
             }

@@ -285,7 +285,7 @@ struct NucParams {
     NucRec* out;               // [R]
 };
 
-// One cluster of CTAs per row (launched with cluster size 1 to 8): the row's
+// One cluster of CTAs per row (launched with cluster size 1 to 16): the row's
 // cut and kept normaliser.  Rows whose sequence has no nucleus (top_p = 1),
 // an invalid setting or an invalid row get {-inf, 1/S}: K2 validates the
 // settings and the row itself.
