@@ -14,7 +14,9 @@ input can reach:
     p = q and the two draws agree;
   * the nucleus reaching top_p with ">" instead of ">=": the two differ only
     when an fp64 running sum of exponentials equals a float32 top_p exactly,
-    which no float32 logit row gives dependably.
+    which no float32 logit row gives dependably;
+  * the tree residual's mass taken as the sum of max(0, q - R) instead of
+    max(0, R - q): R and q both sum to 1, so the two sums are equal.
 """
 import os
 import shutil
@@ -26,7 +28,7 @@ import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "spec_verify_oracle.c")
-PIN_FILES = ["tests/test_oracle.py", "tests/test_oracle_processors.py"]
+PIN_FILES = ["tests/test_oracle.py", "tests/test_oracle_processors.py", "tests/test_oracle_tree.py"]
 
 # (name, text, replacement, which occurrence of text)
 MUTANTS = [
@@ -95,6 +97,22 @@ MUTANTS = [
     ("nucleus_one_past", "cut = pv[i].p;", "cut = pv[i + 1 < n ? i + 1 : i].p;", 0),
     ("top_p_of_first_sequence", "pr.top_p = top_p ? (double)top_p[b] : 1.0;", "pr.top_p = top_p ? (double)top_p[0] : 1.0;", 0),
     ("proposer_processors_of_first_sequence", "const int s = r / rows_per_seq;", "const int s = 0 * rows_per_seq;", 0),
+    # R18 tree verification
+    ("tree_accept_transposed", "if ((double)u[c - 1] * q < r) {", "if ((double)u[c - 1] * r < q) {", 0),
+    ("tree_accept_non_strict", "if ((double)u[c - 1] * q < r) {", "if ((double)u[c - 1] * q <= r) {", 0),
+    ("tree_child_uniform_index", "if ((double)u[c - 1] * q < r) {", "if ((double)u[c] * q < r) {", 0),
+    ("tree_residual_not_renormalised", "R[v] = (R[v] > Q[v]) ? (R[v] - Q[v]) / W : 0.0;",
+     "R[v] = (R[v] > Q[v]) ? (R[v] - Q[v]) : 0.0;", 0),
+    ("tree_residual_never_taken", "if (W > 0.0)\n", "if (W < 0.0)\n", 0),
+    ("tree_children_last_first", "for (c = a + 1; c <= N && !next; ++c) {\n                    double r, q, W = 0.0;",
+     "for (c = N; c > a && !next; --c) {\n                    double r, q, W = 0.0;", 0),
+    ("tree_final_uniform_index", "oracle_inverse_cdf(R, V, (double)u[N], &y, &lo, &hi);",
+     "oracle_inverse_cdf(R, V, (double)u[0], &y, &lo, &hi);", 0),
+    ("tree_rows_of_the_parent", "const long row = (long)b * (N + 1) + a;",
+     "const long row = (long)b * (N + 1) + (a > 0 ? par[a - 1] : 0);", 0),
+    ("tree_greedy_any_child", "if (par[c - 1] == a && t[c - 1] == g) next = c;", "if (par[c - 1] == a) next = c;", 0),
+    ("tree_parent_not_checked", "|| par[i] < 0 || par[i] > i) err = 1;", "|| par[i] < 0 || par[i] > i + 1) err = 1;", 0),
+    ("tree_out_p_is_q", "if (out_p) out_p[(size_t)b * N + c - 1] = r;", "if (out_p) out_p[(size_t)b * N + c - 1] = q;", 0),
 ]
 
 
