@@ -568,16 +568,27 @@ __global__ void __launch_bounds__(NT + 32, RowsOcc<NT, MODE>::value) sv_rows_ker
 #pragma unroll
                 for (int i = 0; i <= VPT; ++i) vm[i] = NEG_INF;
             } else if constexpr (PROC) {
-                // one copy of the processing code (a rolled loop); the maxima
-                // come back to registers through this thread's own slots
+                // raw maxima first (the plain path's cost); then one copy of the
+                // processing code (a rolled loop) over the vectors that need it,
+                // whose maxima come back through this thread's own slots
                 const float skip_below = (MODE == MODE_TOPK && pen_theta >= 1.f) ? theta : NEG_INF;
-#pragma unroll 1
+                unsigned need = 0u;
+#pragma unroll
                 for (int i = 0; i <= VPT; ++i) {
                     const int j = jof(i);
-                    vmsh[i * NT + tid] = (ok && j < g.nvec) ? proc_vmax(j, skip_below) : NEG_INF;
+                    float rm = NEG_INF;
+                    if (ok && j < g.nvec) {
+                        rm = tile_full ? vmax_nan<DT>(vec_at(j)) : vmax_masked(j);
+                        if (!(rm < skip_below)) need |= 1u << i;
+                    }
+                    if (!(rm == rm) || rm == POS_INF) rawbad = true;
+                }
+                for (unsigned mm = need; mm; mm &= mm - 1u) {
+                    const int i = __ffs(mm) - 1;
+                    vmsh[i * NT + tid] = proc_vmax(jof(i), NEG_INF);
                 }
 #pragma unroll
-                for (int i = 0; i <= VPT; ++i) vm[i] = vmsh[i * NT + tid];
+                for (int i = 0; i <= VPT; ++i) vm[i] = ((need >> i) & 1u) ? vmsh[i * NT + tid] : NEG_INF;
             } else if (tile_full) {
 #pragma unroll
                 for (int i = 0; i < VPT; ++i) vm[i] = vmax_nan<DT>(vec_at(tid + i * NT));
