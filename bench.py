@@ -665,6 +665,99 @@ def measure_tree(args, sv, dev, world, rank):
             "l2": f"{nsets} rotating input set(s) of {set_bytes / 1e6:.1f} MB"}
 
 
+HEAD_SHAPE = (64, 4, 151936, 4096)  # B, k, V, H: the batched shape with a 4,096-wide hidden state
+FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0  # a seconds-long cuBLAS bf16 loop under the 1 kW cap
+
+
+def measured_bf16_peak():
+    """The dense bf16 peak for a kernel timed inside a long loop: the
+    sustained figure (the clocks settle under the power cap)."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops_sustained"]), "measured (sustained)"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS_SUSTAINED, "fallback (sustained)"
+
+
+def measure_head(args, sv, dev, world, rank):
+    """Greedy verification fused into the output projection: B x (k+1)
+    hidden states [4,096] bf16 times a [V, 4,096] bf16 weight (1.24 GB, ten
+    times L2: every step streams it from HBM), the logits reduced on chip.
+    Draft tokens are random (the step's time does not depend on them).  The
+    projection kernel is also timed alone between an event pair on KSAMPLES
+    steps."""
+    import torch
+
+    B, k, V, H = HEAD_SHAPE
+    case = workloads.make_head_case(rank_seed(rank), B, k, V, H)
+    hidden = to_dev(case.hidden, dev)
+    weight = to_dev(case.weight, dev)
+    del case
+    drafts = torch.from_numpy(np.random.default_rng(rank_seed(rank)).integers(0, V, (B, k)).astype(np.int32)).to(dev)
+    out_tok = torch.empty((B, k + 1), dtype=torch.int32, device=dev)
+    out_n = torch.empty((B,), dtype=torch.int32, device=dev)
+    status = torch.zeros((1,), dtype=torch.int32, device=dev)
+    wbytes = sv.spec_verify_head_workspace_size(B, k, V, H)
+    ws = torch.empty((wbytes,), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev0=None, ev1=None):
+        opts = sv.make_options(event_start=ev0, event_stop=ev1) if ev0 is not None else None
+        st = sv.spec_verify_head_greedy(hidden, weight, drafts, B, k, V, H, out_tok, out_n, None, ws, wbytes, opts,
+                                        status, stream)
+        if st != sv.SV_OK:
+            raise sv.SpecVerifyError(st, "spec_verify_head_greedy")
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(rank)
+    sampler.start()
+    t_end = time.perf_counter() + getattr(args, "clock_window", 0.0)
+    while time.perf_counter() < t_end:
+        for _ in range(8):
+            step()
+        torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    a.record(stream)
+    for _ in range(args.steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(a.elapsed_time(b), dev)
+    evk = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(KSAMPLES)]
+    for e0, e1 in evk:
+        e0.record(stream)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    for e0, e1 in evk:
+        step(e0, e1)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if int(status.item()) != 0:
+        raise SystemExit(f"head: device status {int(status.item())}")
+    kern_ms = [e0.elapsed_time(e1) for e0, e1 in evk]
+    kmean = sum(kern_ms) / len(kern_ms)
+    rows = B * (k + 1)
+    flops = 2.0 * rows * V * H  # the logits of every position, no padding counted
+    peak, src = measured_bf16_peak()
+    achieved = flops / (kmean / 1000.0) / 1e12
+    w_bytes = V * H * 2
+    return {"workload": f"greedy verify fused into the output projection B={B} k={k} V={V} H={H} bf16",
+            "value": job_rate(B * k * args.steps, world, ms), "unit": "positions/s",
+            "ms_per_step": ms / args.steps, "gpu_launches": 2 * args.steps, "clocks": clocks,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "peak_source": src, "kernel": "sv_head_kernel",
+                         "kernel_ms_mean": kmean, "kernel_ms_median": statistics.median(kern_ms),
+                         "kernel_samples": len(kern_ms), "flops_per_launch": flops,
+                         "weight_gbs": w_bytes / (kmean / 1000.0) / 1e9, "weight_bytes": w_bytes},
+            "logits_written_bytes": 0,
+            "l2": f"weight {w_bytes / 1e9:.2f} GB per step (> 126 MB L2)"}
+
+
 def run_ours(args):
     import torch
 
@@ -683,8 +776,8 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     sv.lib()
 
-    if args.tree_only:
-        r = measure_tree(args, sv, dev, world, local)
+    if args.tree_only or args.head_only:
+        r = (measure_tree if args.tree_only else measure_head)(args, sv, dev, world, local)
         if world > 1:
             torch.distributed.barrier()
             torch.distributed.destroy_process_group()
@@ -709,6 +802,7 @@ def run_ours(args):
             r.pop("_case")
             others[f"{base}+{feature}"] = r
         others["tree"] = measure_tree(args, sv, dev, world, local)
+        others["head_greedy"] = measure_head(args, sv, dev, world, local)
     case, drafts = head.pop("_case"), head.pop("_drafts")
 
     cpu = None
@@ -772,6 +866,8 @@ def main():
                     help="profile a feature alone: --workload with these options (no e2e or CPU leg)")
     ap.add_argument("--tree-only", action="store_true",
                     help="measure only the tree-verification line (one JSON line; for profiling)")
+    ap.add_argument("--head-only", action="store_true",
+                    help="measure only the output-projection greedy line (one JSON line; for profiling)")
     ap.add_argument("--headline-only", action="store_true",
                     help="measure only --workload (default: every workload, the headline first)")
     args = ap.parse_args()

@@ -39,6 +39,7 @@ __all__ = [
     "spec_sample", "spec_sample_ex", "spec_sample_workspace_size", "make_options",
     "spec_verify_status_string", "spec_verify_version", "spec_verify_pool_allocations", "verify", "sample",
     "spec_verify_tree", "spec_verify_tree_ex", "spec_verify_tree_workspace_size", "verify_tree",
+    "spec_verify_head_greedy", "spec_verify_head_workspace_size", "verify_head_greedy",
 ]
 
 
@@ -92,6 +93,10 @@ def lib() -> ctypes.CDLL:
         L.spec_verify_tree_ex.restype = I
         L.spec_verify_tree_workspace_size.argtypes = [I, I, I, I, I]
         L.spec_verify_tree_workspace_size.restype = Z
+        L.spec_verify_head_greedy.argtypes = [P, P, P, I, I, I, I, P, P, P, P, Z, OP, P, P]
+        L.spec_verify_head_greedy.restype = I
+        L.spec_verify_head_workspace_size.argtypes = [I, I, I, I]
+        L.spec_verify_head_workspace_size.restype = Z
         L.spec_verify_workspace_size.argtypes = [I, I, I, I, I, OP]
         L.spec_verify_workspace_size.restype = Z
         L.spec_sample.argtypes = [P, P, I, I, P, I, I, P, P]
@@ -322,6 +327,59 @@ def verify_tree(target, draft, tokens, parents, uniforms=None, temperature=None,
                              None if greedy else out_p, None if greedy else out_q, workspace, wbytes, stream)
     if st != SV_OK:
         raise SpecVerifyError(st, "spec_verify_tree_ex")
+    return out_tokens, out_n
+
+
+def spec_verify_head_greedy(hidden, weight, draft_tokens, B, k, V, H, out_tokens, out_n_accepted,
+                            out_argmax=None, workspace=None, workspace_bytes=0,
+                            opts: Optional[SvOptions] = None, out_status=None, stream=None) -> int:
+    return lib().spec_verify_head_greedy(_p(hidden), _p(weight), _p(draft_tokens), int(B), int(k), int(V), int(H),
+                                         _p(out_tokens), _p(out_n_accepted), _p(out_argmax), _p(workspace),
+                                         int(workspace_bytes), _opts(opts), _p(out_status), _stream(stream))
+
+
+def spec_verify_head_workspace_size(B, k, V, H) -> int:
+    return int(lib().spec_verify_head_workspace_size(int(B), int(k), int(V), int(H)))
+
+
+def verify_head_greedy(hidden, weight, draft_tokens, out_argmax=None, out_status=None, workspace=None,
+                       opts: Optional[SvOptions] = None, stream=None):
+    """Tensor convenience wrapper around ``spec_verify_head_greedy``: hidden
+    [B, k+1, H] and weight [V, H] bf16 (contiguous, on the GPU), draft_tokens
+    [B, k] int32; optional out_argmax [B, k+1] and out_status [1] int32; the
+    workspace (uint8) is allocated with torch when None.  Returns
+    (out_tokens [B, k+1], out_n_accepted [B])."""
+    import torch
+
+    if hidden.dim() != 3 or weight.dim() != 2:
+        raise ValueError(f"hidden must be [B, k+1, H] and weight [V, H], got {tuple(hidden.shape)}, "
+                         f"{tuple(weight.shape)}")
+    B, n1, H = hidden.shape
+    V = weight.shape[0]
+    k = n1 - 1
+    dev = hidden.device
+    bf, i32 = (torch.bfloat16,), (torch.int32,)
+    _check(hidden, "hidden", bf, B * n1 * H, dev)
+    _check(weight, "weight", bf, V * H, dev)
+    _check(draft_tokens, "draft_tokens", i32, B * k, dev)
+    if out_argmax is not None:
+        _check(out_argmax, "out_argmax", i32, B * n1, dev)
+    if out_status is not None:
+        _check(out_status, "out_status", i32, 1, dev)
+    _check_cuda(dev)
+    out_tokens = torch.empty((B, n1), dtype=torch.int32, device=dev)
+    out_n = torch.empty((B,), dtype=torch.int32, device=dev)
+    if workspace is None:
+        need = spec_verify_head_workspace_size(B, k, V, H)
+        if need == 0:
+            raise SpecVerifyError(SV_ERR_INVALID_ARG, "spec_verify_head_workspace_size")
+        workspace = torch.empty((need,), dtype=torch.uint8, device=dev)
+    _check(workspace, "workspace", (workspace.dtype,), workspace.numel(), dev)
+    wbytes = workspace.numel() * workspace.element_size()
+    st = spec_verify_head_greedy(hidden, weight, draft_tokens, B, k, V, H, out_tokens, out_n, out_argmax, workspace,
+                                 wbytes, opts, out_status, stream)
+    if st != SV_OK:
+        raise SpecVerifyError(st, "spec_verify_head_greedy")
     return out_tokens, out_n
 
 

@@ -9,7 +9,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libspec_verify.so")
 SOURCES = [os.path.join(CSRC, "spec_verify.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("sv_common.cuh", "sv_rows.cuh", "sv_seq.cuh", "sv_resid.cuh", "sv_ptx.cuh", "sv_procs.cuh", "sv_nucleus.cuh", "sv_tree.cuh")] + [
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("sv_common.cuh", "sv_rows.cuh", "sv_seq.cuh", "sv_resid.cuh", "sv_ptx.cuh", "sv_procs.cuh", "sv_nucleus.cuh", "sv_tree.cuh", "sv_head.cuh")] + [
     os.path.join(ROOT, "include", "spec_verify.h")]
 
 NVCC_FLAGS = [

@@ -5,6 +5,7 @@
 // verification the segment kernel of the residual draws.  Nothing here
 // synchronises the caller's stream.
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include <climits>
 #include <cstdint>
@@ -17,6 +18,7 @@
 #include "sv_resid.cuh"
 #include "sv_seq.cuh"
 #include "sv_tree.cuh"
+#include "sv_head.cuh"
 
 namespace {
 
@@ -823,6 +825,60 @@ void tree_plan(const DeviceInfo& dev, int B, int N, int V, int dt, bool greedy, 
     *out = t;
 }
 
+namespace {
+
+// ---- the output projection with greedy verification ------------------------
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+std::once_flag g_head_attr_once[kMaxDevices];
+cudaError_t g_head_attr_err[kMaxDevices];
+
+// The driver's tensor-map encoder, looked up through the runtime (no link
+// against the driver library).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    std::call_once(g_encode_once, [] {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+        else
+            cudaGetLastError();
+    });
+    return g_encode;
+}
+
+// Row-major bf16 matrix [outer][inner] as 2D tiles of box_outer rows x 64
+// elements, 128-byte swizzled (the K-major operand layout of the MMA), zeros
+// outside the matrix.
+bool encode_bf16_rows(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint32_t box_outer) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {inner * 2};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(sv::HEAD_BK), box_outer};
+    cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+constexpr int kHeadMaxVTiles = 65535;  // grid y
+
+// Workspace of the fused path: each row's running best (8 bytes) and the
+// timeout flag, zeroed by one memset per call.  0 on invalid sizes.
+size_t head_ws_bytes(int B, int k, int V) {
+    if (B <= 0 || k < 1 || V < 1) return 0;
+    const long long rows = static_cast<long long>(B) * (k + 1);
+    const long long vt = ceil_div(V, sv::HEAD_BN);
+    if (rows > INT_MAX / 2 || vt > kHeadMaxVTiles) return 0;
+    return static_cast<size_t>(round_up(rows * 8, 16) + 16);
+}
+
+}  // namespace
+
 extern "C" {
 
 sv_status_t spec_verify_tree_ex(const void* target_logits, const void* draft_logits, const int32_t* tokens,
@@ -1054,6 +1110,122 @@ size_t spec_sample_workspace_size(int rows, int V, int top_k, int mode, const sv
     Call cl;
     if (sample_args(nullptr, nullptr, rows, V, nullptr, top_k, mode, nullptr, opts, false, &cl) != SV_OK) return 0;
     return workspace_for(cl, opts);
+}
+
+sv_status_t spec_verify_head_greedy(const void* hidden, const void* weight, const int32_t* draft_tokens, int B,
+                                    int k, int V, int H, int32_t* out_tokens, int32_t* out_n_accepted,
+                                    int32_t* out_argmax, void* workspace, size_t workspace_bytes,
+                                    const sv_options_t* opts, int32_t* out_status, void* stream) {
+    if (B <= 0 || k < 1 || V < 1 || H < 1 || H % 8 != 0) return SV_ERR_INVALID_ARG;
+    if (!hidden || !weight || !draft_tokens || !out_tokens || !out_n_accepted) return SV_ERR_INVALID_ARG;
+    if (!aligned(hidden, 16) || !aligned(weight, 16) || !aligned(draft_tokens, 4) || !aligned(out_tokens, 4) ||
+        !aligned(out_n_accepted, 4) || (out_argmax && !aligned(out_argmax, 4)) ||
+        (out_status && !aligned(out_status, 4)))
+        return SV_ERR_INVALID_ARG;
+    const size_t need = head_ws_bytes(B, k, V);
+    if (need == 0) return ceil_div(V, sv::HEAD_BN) > kHeadMaxVTiles ? SV_ERR_UNSUPPORTED : SV_ERR_INVALID_ARG;
+    if (workspace && (!aligned(workspace, 16) || workspace_bytes < need)) return SV_ERR_INVALID_ARG;
+    if (opts && check_options(opts) != SV_OK) return SV_ERR_INVALID_ARG;
+    if (opts && (opts->top_p || opts->vocab_mask || opts->rep_ids)) return SV_ERR_UNSUPPORTED;  // greedy only
+    int dev = 0;
+    const DeviceInfo* info = device_info(&dev);
+    if (!info) return SV_ERR_UNSUPPORTED;
+    const int rows = B * (k + 1);
+    const int vtiles = static_cast<int>(ceil_div(V, sv::HEAD_BN));
+    CUtensorMap tm_h, tm_w;
+    if (!tensor_map_encoder()) return SV_ERR_UNSUPPORTED;
+    if (!encode_bf16_rows(&tm_h, hidden, static_cast<uint64_t>(H), static_cast<uint64_t>(rows), sv::HEAD_BM) ||
+        !encode_bf16_rows(&tm_w, weight, static_cast<uint64_t>(H), static_cast<uint64_t>(V), sv::HEAD_BN))
+        return SV_ERR_INVALID_ARG;
+    std::call_once(g_head_attr_once[dev], [dev] {
+        g_head_attr_err[dev] =
+            cudaFuncSetAttribute(sv::sv_head_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, sv::HEAD_SMEM);
+        if (g_head_attr_err[dev] != cudaSuccess) cudaGetLastError();
+    });
+    if (g_head_attr_err[dev] != cudaSuccess) return SV_ERR_CUDA;
+
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    void* ws = workspace;
+    bool owned = false;
+    if (!ws) {
+        cudaMemPool_t pool = device_pool(dev);
+        if (!pool || cudaMallocFromPoolAsync(&ws, need, pool, st) != cudaSuccess) {
+            cudaGetLastError();
+            return SV_ERR_CUDA;
+        }
+        g_pool_allocs.fetch_add(1, std::memory_order_relaxed);
+        owned = true;
+    }
+    auto* base = static_cast<unsigned char*>(ws);
+    int* err = reinterpret_cast<int*>(base + need - 16);
+    sv::HeadParams P;
+    P.rows = rows;
+    P.V = V;
+    P.H = H;
+    P.best = reinterpret_cast<unsigned long long*>(base);
+    P.err = err;
+    P.timeout_ns = (opts && opts->wait_timeout_ns) ? opts->wait_timeout_ns : kDefaultTimeoutNs;
+    P.test_hook = (opts && opts->test_extra_tx) ? 1 : 0;
+    sv::HeadDecideParams D;
+    D.best = P.best;
+    D.err = err;
+    D.draft_tokens = draft_tokens;
+    D.B = B;
+    D.k = k;
+    D.V = V;
+    D.out_tokens = out_tokens;
+    D.out_n_accepted = out_n_accepted;
+    D.out_argmax = out_argmax;
+    D.out_status = out_status;
+
+    sv_status_t result = SV_OK;
+    do {
+        if (cudaMemsetAsync(base, 0, need, st) != cudaSuccess) {  // the running bests and the flag
+            result = SV_ERR_CUDA;
+            break;
+        }
+        if (opts && opts->event_start &&
+            cudaEventRecord(static_cast<cudaEvent_t>(opts->event_start), st) != cudaSuccess) {
+            result = SV_ERR_CUDA;
+            break;
+        }
+        sv::sv_head_kernel<<<dim3(static_cast<unsigned>(ceil_div(rows, sv::HEAD_BM)), static_cast<unsigned>(vtiles), 1),
+                             sv::HEAD_NT, sv::HEAD_SMEM, st>>>(tm_h, tm_w, P);
+        if (cudaGetLastError() != cudaSuccess) {
+            result = SV_ERR_CUDA;
+            break;
+        }
+        if (opts && opts->event_stop &&
+            cudaEventRecord(static_cast<cudaEvent_t>(opts->event_stop), st) != cudaSuccess) {
+            result = SV_ERR_CUDA;
+            break;
+        }
+        cudaLaunchAttribute a[1];
+        a[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        a[0].val.programmaticStreamSerializationAllowed = 1;
+        cudaLaunchConfig_t c;
+        std::memset(&c, 0, sizeof c);
+        c.gridDim = dim3(static_cast<unsigned>(ceil_div(B, sv::HEAD_DECIDE_NT / 32)), 1, 1);
+        c.blockDim = dim3(sv::HEAD_DECIDE_NT, 1, 1);
+        c.stream = st;
+        c.attrs = a;
+        c.numAttrs = 1;
+        if (cudaLaunchKernelEx(&c, sv::sv_head_decide_kernel, D) != cudaSuccess) {
+            result = SV_ERR_CUDA;
+            break;
+        }
+    } while (false);
+    if (result != SV_OK) cudaGetLastError();
+    if (owned && cudaFreeAsync(ws, st) != cudaSuccess) {
+        cudaGetLastError();
+        if (result == SV_OK) result = SV_ERR_CUDA;
+    }
+    return result;
+}
+
+size_t spec_verify_head_workspace_size(int B, int k, int V, int H) {
+    if (H < 1 || H % 8 != 0) return 0;
+    return head_ws_bytes(B, k, V);
 }
 
 const char* spec_verify_status_string(sv_status_t status) {

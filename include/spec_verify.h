@@ -312,6 +312,49 @@ SV_API sv_status_t spec_verify_tree_ex(const void* target_logits, const void* dr
  * list walk (no top-k) or on invalid arguments / no usable device. */
 SV_API size_t spec_verify_tree_workspace_size(int B, int N, int V, int top_k, int mode);
 
+/*
+ * spec_verify_head_greedy — greedy verification fused into the target's
+ * output projection.  The target scores the k+1 positions of a sequence in
+ * one forward pass (section "提议与核验的基本步骤", paragraph 1); here its
+ * last step, the logits z_v = h . W[v], is computed on the tensor cores and
+ * reduced on chip to each position's lowest-index argmax, so the logits are
+ * never written to memory; the greedy rule of paragraph 4 then runs as in
+ * spec_verify with SV_MODE_GREEDY.
+ *   hidden        [B][k+1][H] bf16, 16-byte aligned: the target's final
+ *                 hidden state at each position
+ *   weight        [V][H] bf16, 16-byte aligned: the output projection
+ *   draft_tokens  [B][k] int32
+ *   H             > 0 and a multiple of 8 (16-byte rows)
+ *   out_tokens, out_n_accepted   as spec_verify (greedy)
+ *   out_argmax    [B][k+1] int32 or NULL: each position's argmax, -1 for a
+ *                 row with a NaN or +inf logit or none finite
+ *   workspace     spec_verify_head_workspace_size(B, k, V, H) bytes of device
+ *                 memory, 16-byte aligned, or NULL (taken from the library's
+ *                 pool on `stream` and released there); written before read
+ *   opts          NULL or options: wait_timeout_ns, event_start / event_stop
+ *                 (around the projection kernel) and test_extra_tx (non-zero:
+ *                 the projection kernel also waits for an accumulator phase
+ *                 that never completes, so its bounded wait runs out with no
+ *                 copy or MMA in flight); top_p, vocab_mask and rep_ids give
+ *                 SV_ERR_UNSUPPORTED
+ *   out_status    1 int32 or NULL: SV_OK, or SV_ERR_DEVICE_TIMEOUT when a
+ *                 device-side wait ran out (then every sequence is an error)
+ * The products of bf16 values are exact and are summed in fp32 on the tensor
+ * cores, so a logit differs from its exact value by rounding of that sum
+ * only.  Row errors as spec_verify: a draft token outside [0, V), a NaN or
+ * +inf logit, or a row with no finite logit, anywhere in the sequence.
+ * V up to 16,776,960 (SV_ERR_UNSUPPORTED above).
+ */
+SV_API sv_status_t spec_verify_head_greedy(const void* hidden, const void* weight,
+                                           const int32_t* draft_tokens, int B, int k, int V, int H,
+                                           int32_t* out_tokens, int32_t* out_n_accepted,
+                                           int32_t* out_argmax, void* workspace,
+                                           size_t workspace_bytes, const sv_options_t* opts,
+                                           int32_t* out_status, void* stream);
+
+/* Workspace bytes for spec_verify_head_greedy; 0 on invalid sizes. */
+SV_API size_t spec_verify_head_workspace_size(int B, int k, int V, int H);
+
 /* Static description of a status code. */
 SV_API const char* spec_verify_status_string(sv_status_t status);
 

@@ -17,6 +17,7 @@ from . import build as _build
 
 DTYPE_BF16 = 0
 DTYPE_F32 = 1
+DTYPE_F64 = 2  # logits the oracle formed itself (the output projection)
 
 _lib = None
 
@@ -45,6 +46,9 @@ def lib():
         _lib.oracle_sample_rows_procs.restype = I
         _lib.oracle_verify_tree.argtypes = [P, P, P, P, P, I, I, I, P, I, I, I, P, P, P, P, P, P, P, P]
         _lib.oracle_verify_tree.restype = I
+        L = ctypes.c_long
+        _lib.oracle_head_logits.argtypes = [P, P, L, L, I, I, P, P]
+        _lib.oracle_head_logits.restype = None
     return _lib
 
 
@@ -57,7 +61,9 @@ def _dtype_code(a: np.ndarray) -> int:
         return DTYPE_BF16
     if a.dtype == np.float32:
         return DTYPE_F32
-    raise TypeError(f"logits must be uint16 (bf16 bits) or float32, got {a.dtype}")
+    if a.dtype == np.float64:
+        return DTYPE_F64
+    raise TypeError(f"logits must be uint16 (bf16 bits), float32 or float64, got {a.dtype}")
 
 
 def process_row(row: np.ndarray, temperature: float = 1.0, top_k: int = 0):
@@ -316,3 +322,55 @@ def verify_tree(target, draft, tokens, parents, uniforms=None, temperature=None,
         raise MemoryError("oracle_verify_tree could not allocate its work arrays")
     return TreeResult(out, n, nodes, p[:, :N], q[:, :N], ratio[:, :N], lo, hi, errs)
 
+
+def head_logits(hidden: np.ndarray, weight: np.ndarray, row0: int = 0, n: Optional[int] = None):
+    """The output projection in fp64 (``oracle_head_logits``): hidden [rows, H]
+    (any leading shape) and weight [V, H] as bf16 bit patterns (uint16).
+    Returns (z, abs) for rows row0 .. row0+n, each [n, V]: z the logits summed
+    in index order, abs the sums of the products' magnitudes."""
+    H = hidden.shape[-1]
+    h = np.ascontiguousarray(hidden, dtype=np.uint16).reshape(-1, H)
+    w = np.ascontiguousarray(weight, dtype=np.uint16)
+    V = w.shape[0]
+    assert w.shape == (V, H)
+    n = h.shape[0] - row0 if n is None else n
+    z = np.empty((n, V), dtype=np.float64)
+    a = np.empty((n, V), dtype=np.float64)
+    lib().oracle_head_logits(_ptr(h), _ptr(w), int(row0), int(n), int(V), int(H), _ptr(z), _ptr(a))
+    return z, a
+
+
+@dataclasses.dataclass
+class HeadResult:
+    seqs: np.ndarray        # [S] the sequences verified
+    result: VerifyResult    # greedy verification of those sequences
+    z: np.ndarray           # [S, k+1, V] fp64 logits
+    abs: np.ndarray         # [S, k+1, V] fp64 sums of |h_j * W[v][j]|
+
+
+def verify_head_greedy(hidden: np.ndarray, weight: np.ndarray, draft_tokens: np.ndarray, seqs=None,
+                       threads: int = 1) -> HeadResult:
+    """Greedy verification on the logits of the output projection: hidden
+    [B, k+1, H] and weight [V, H] (bf16 bits), draft_tokens [B, k].  ``seqs``
+    picks the sequences to verify (all when None); ``threads`` > 1 forms the
+    logits of several sequences at once (the C routine runs without the GIL)."""
+    B, k1, H = hidden.shape
+    seqs = np.arange(B) if seqs is None else np.asarray(seqs, dtype=np.int64)
+    draft_tokens = np.asarray(draft_tokens, dtype=np.int32).reshape(B, k1 - 1)
+    V = weight.shape[0]
+    z = np.empty((len(seqs), k1, V), dtype=np.float64)
+    a = np.empty_like(z)
+
+    def one(i):
+        z[i], a[i] = head_logits(hidden, weight, int(seqs[i]) * k1, k1)
+
+    if threads > 1:
+        from concurrent.futures import ThreadPoolExecutor
+
+        with ThreadPoolExecutor(threads) as ex:
+            list(ex.map(one, range(len(seqs))))
+    else:
+        for i in range(len(seqs)):
+            one(i)
+    res = verify(z, None, draft_tokens[seqs], None, greedy=True)
+    return HeadResult(seqs, res, z, a)

@@ -48,6 +48,7 @@
 
 #define OR_DTYPE_BF16 0
 #define OR_DTYPE_F32 1
+#define OR_DTYPE_F64 2 /* logits formed here (the output projection below) */
 
 /* ---- reading logits (bf16 widening is exact) ---------------------------- */
 
@@ -58,11 +59,12 @@ static double or_logit(const void* row, int dtype, long v) {
         memcpy(&f, &bits, sizeof f);
         return (double)f;
     }
+    if (dtype == OR_DTYPE_F64) return ((const double*)row)[v];
     return (double)((const float*)row)[v];
 }
 
 static const void* or_row(const void* base, int dtype, long row, long V) {
-    size_t elt = dtype == OR_DTYPE_BF16 ? 2 : 4;
+    size_t elt = dtype == OR_DTYPE_BF16 ? 2 : (dtype == OR_DTYPE_F64 ? 8 : 4);
     return (const char*)base + (size_t)row * (size_t)V * elt;
 }
 
@@ -698,4 +700,34 @@ int oracle_verify_tree(const void* target, const void* draft, const int32_t* tok
     }
     free(R); free(Q); free(work);
     return errors;
+}
+
+/*
+ * The target's output projection (section "提议与核验的基本步骤", paragraph 1:
+ * one forward pass scores every position; its last step maps the hidden
+ * state h of a position to the logits z_v = sum_j h_j * W[v][j]).
+ *   hidden  [rows][H] bf16 bits, weight [V][H] bf16 bits
+ *   out_z   [rows][V] fp64: z_v summed in index order j = 0 .. H-1
+ *   out_abs [rows][V] fp64 or NULL: sum_j |h_j * W[v][j]|, the scale of the
+ *           rounding of any other summation of the same products
+ * The products of two bf16 values are exact in double (8-bit significands);
+ * only the running sum rounds.  Writes the given rows only (row0 .. row0+n).
+ */
+void oracle_head_logits(const uint16_t* hidden, const uint16_t* weight, long row0, long n, int V, int H,
+                        double* out_z, double* out_abs) {
+    long r, v, j;
+    for (r = row0; r < row0 + n; ++r) {
+        const void* h = hidden + (size_t)r * (size_t)H;
+        for (v = 0; v < V; ++v) {
+            const void* w = weight + (size_t)v * (size_t)H;
+            double z = 0.0, a = 0.0;
+            for (j = 0; j < H; ++j) {
+                double t = or_logit(h, OR_DTYPE_BF16, j) * or_logit(w, OR_DTYPE_BF16, j);
+                z += t;
+                a += fabs(t);
+            }
+            out_z[(size_t)(r - row0) * (size_t)V + v] = z;
+            if (out_abs) out_abs[(size_t)(r - row0) * (size_t)V + v] = a;
+        }
+    }
 }

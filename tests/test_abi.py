@@ -30,7 +30,8 @@ def test_header_declares_entry_points():
     assert declared_functions() == sorted([
         "spec_sample", "spec_sample_ex", "spec_sample_workspace_size", "spec_verify", "spec_verify_ex",
         "spec_verify_pool_allocations", "spec_verify_static", "spec_verify_status_string", "spec_verify_tree",
-        "spec_verify_tree_ex", "spec_verify_tree_workspace_size", "spec_verify_version", "spec_verify_workspace_size"])
+        "spec_verify_tree_ex", "spec_verify_tree_workspace_size", "spec_verify_version", "spec_verify_workspace_size",
+        "spec_verify_head_greedy", "spec_verify_head_workspace_size"])
 
 
 
@@ -214,13 +215,12 @@ def test_no_device_is_reported_as_unsupported(L):
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
-    import importlib
-
+    # monkeypatch puts the loaded library back afterwards; a module reload here
+    # would leave the options class out of step with the loaded signatures
     monkeypatch.setattr(sv, "_lib", None)
     monkeypatch.setattr(sv, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(ImportError):
         sv.lib()
-    importlib.reload(sv)
 
 
 # --------------------------------------------------------------------------
@@ -343,3 +343,43 @@ def test_tree_ex_checks_the_workspace(L):
     assert st == sv.SV_ERR_INVALID_ARG  # not 16-byte aligned
     assert sv.spec_verify_tree_workspace_size(0, 3, 100, 5, 0) == 0
     assert sv.spec_verify_tree_workspace_size(2, 0, 100, 5, 0) == 0
+
+
+@pytest.mark.parametrize("kw", [dict(B=0), dict(k=0), dict(V=0), dict(H=0), dict(H=100), dict(hidden=None),
+                                dict(weight=None), dict(drafts=None), dict(out_tokens=None), dict(out_n=None),
+                                dict(hidden=P + 8), dict(weight=P + 2), dict(drafts=P + 2), dict(out_argmax=P + 1),
+                                dict(out_status=P + 2), dict(workspace=P + 8), dict(workspace_bytes=16),
+                                dict(V=1 << 30)])
+def test_head_invalid_arguments(L, kw):
+    a = dict(hidden=P, weight=P, drafts=P, B=4, k=3, V=1000, H=256, out_tokens=P, out_n=P, out_argmax=None,
+             workspace=P, workspace_bytes=1 << 20, out_status=None)
+    a.update(kw)
+    st = sv.spec_verify_head_greedy(a["hidden"], a["weight"], a["drafts"], a["B"], a["k"], a["V"], a["H"],
+                                    a["out_tokens"], a["out_n"], a["out_argmax"], a["workspace"],
+                                    a["workspace_bytes"], None, a["out_status"], stream=0)
+    expect = sv.SV_ERR_UNSUPPORTED if kw.get("V") == 1 << 30 else sv.SV_ERR_INVALID_ARG
+    assert st == expect, kw
+
+
+def test_head_processors_unsupported(L):
+    import torch
+
+    tp = torch.ones(4, dtype=torch.float32)
+    st = sv.spec_verify_head_greedy(P, P, P, 4, 3, 1000, 256, P, P, None, P, 1 << 20,
+                                    sv.make_options(top_p=tp), None, stream=0)
+    assert st == sv.SV_ERR_UNSUPPORTED
+
+
+def test_head_workspace_size(L):
+    # one 8-byte running best per row, and a flag
+    assert sv.spec_verify_head_workspace_size(64, 4, 151936, 4096) == 320 * 8 + 16
+    assert sv.spec_verify_head_workspace_size(3, 2, 1000, 200) == ((9 * 8 + 15) // 16) * 16 + 16
+    assert sv.spec_verify_head_workspace_size(0, 4, 100, 64) == 0
+    assert sv.spec_verify_head_workspace_size(2, 4, 100, 60) == 0   # H not a multiple of 8
+    assert sv.spec_verify_head_workspace_size(2, 4, 1 << 30, 64) == 0
+
+
+def test_head_no_device_is_unsupported(L):
+    _no_gpu()
+    st = sv.spec_verify_head_greedy(P, P, P, 4, 3, 1000, 256, P, P, None, P, 1 << 20, None, None, stream=0)
+    assert st == sv.SV_ERR_UNSUPPORTED

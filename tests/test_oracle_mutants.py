@@ -28,7 +28,8 @@ import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "spec_verify_oracle.c")
-PIN_FILES = ["tests/test_oracle.py", "tests/test_oracle_processors.py", "tests/test_oracle_tree.py"]
+PIN_FILES = ["tests/test_oracle.py", "tests/test_oracle_processors.py", "tests/test_oracle_tree.py",
+             "tests/test_oracle_head.py"]
 
 # (name, text, replacement, which occurrence of text)
 MUTANTS = [
@@ -76,7 +77,10 @@ MUTANTS = [
      "if (!(u[i] >= 0.0f && u[i] <= 1.0f)) err = 1;", 1),
     # outputs and layout
     ("out_p_is_q", "if (out_p) out_p[(size_t)b * k + i] = p;", "if (out_p) out_p[(size_t)b * k + i] = q;", 0),
-    ("f32_row_stride", "size_t elt = dtype == OR_DTYPE_BF16 ? 2 : 4;", "size_t elt = 2;", 0),
+    ("f32_row_stride", "size_t elt = dtype == OR_DTYPE_BF16 ? 2 : (dtype == OR_DTYPE_F64 ? 8 : 4);",
+     "size_t elt = dtype == OR_DTYPE_BF16 ? 2 : (dtype == OR_DTYPE_F64 ? 8 : 2);", 0),
+    ("f64_row_stride", "size_t elt = dtype == OR_DTYPE_BF16 ? 2 : (dtype == OR_DTYPE_F64 ? 8 : 4);",
+     "size_t elt = dtype == OR_DTYPE_BF16 ? 2 : 4;", 0),
     # R13 repetition penalty
     ("penalty_ignores_sign", "z = z > 0.0 ? (double)(float)(z / pr->rep_penalty) : (double)(float)(z * pr->rep_penalty);",
      "z = (double)(float)(z / pr->rep_penalty);", 0),
@@ -113,6 +117,18 @@ MUTANTS = [
     ("tree_greedy_any_child", "if (par[c - 1] == a && t[c - 1] == g) next = c;", "if (par[c - 1] == a) next = c;", 0),
     ("tree_parent_not_checked", "|| par[i] < 0 || par[i] > i) err = 1;", "|| par[i] < 0 || par[i] > i + 1) err = 1;", 0),
     ("tree_out_p_is_q", "if (out_p) out_p[(size_t)b * N + c - 1] = r;", "if (out_p) out_p[(size_t)b * N + c - 1] = q;", 0),
+    # the output projection and the fp64 rows it feeds to greedy verification
+    ("head_skips_last_term", "for (j = 0; j < H; ++j) {\n                double t",
+     "for (j = 0; j + 1 < H; ++j) {\n                double t", 0),
+    ("head_weight_row_stride", "const void* w = weight + (size_t)v * (size_t)H;",
+     "const void* w = weight + (size_t)v * (size_t)(H - 1);", 0),
+    ("head_hidden_row_stride", "const void* h = hidden + (size_t)r * (size_t)H;",
+     "const void* h = hidden + (size_t)r * (size_t)(H - 1);", 0),
+    ("head_abs_signed", "a += fabs(t);", "a += t;", 0),
+    ("head_columns_reversed", "out_z[(size_t)(r - row0) * (size_t)V + v] = z;",
+     "out_z[(size_t)(r - row0) * (size_t)V + (V - 1 - v)] = z;", 0),
+    ("f64_rows_read_as_float", "if (dtype == OR_DTYPE_F64) return ((const double*)row)[v];",
+     "if (dtype == OR_DTYPE_F64) return (double)((const float*)row)[2 * v];", 0),
 ]
 
 

@@ -52,6 +52,7 @@ large       512   3   128256   f32    target N(0,4^2), draft = target +
 from __future__ import annotations
 
 import dataclasses
+import os
 from typing import Optional
 
 import numpy as np
@@ -60,6 +61,7 @@ __all__ = [
     "GAMMA", "mix64", "splitmix64_stream", "stream_state", "uniform_f32",
     "normals_f64", "f64_to_bf16_bits", "bf16_bits_to_f32", "f64_to_f32",
     "WORKLOADS", "Case", "make_case", "workload_bytes", "Processors", "make_processors",
+    "HeadCase", "make_head_case",
 ]
 
 M64 = (1 << 64) - 1
@@ -80,6 +82,8 @@ TAG_PROXY_NOISE = 8
 TAG_TOP_P = 9
 TAG_REP_IDS = 10
 TAG_MASK = 11
+TAG_HEAD_HIDDEN = 12
+TAG_HEAD_WEIGHT = 13
 
 _U = np.uint64
 
@@ -349,3 +353,42 @@ def make_processors(seed: int, B: int, V: int, top_p=(0.7, 0.95), rep_penalty: f
     weights = (np.uint64(1) << np.arange(32, dtype=np.uint64))
     mask = (bits.reshape(B, words, 32) * weights).sum(axis=2).astype(np.uint32)
     return Processors(tp, rp, ids, mask)
+
+
+@dataclasses.dataclass
+class HeadCase:
+    """Inputs of the target's output projection: the final hidden state at
+    each of the k+1 positions and the projection weight, as bf16 bits."""
+    hidden: np.ndarray  # [B, k+1, H] uint16
+    weight: np.ndarray  # [V, H] uint16
+    B: int
+    k: int
+    V: int
+    H: int
+
+
+def make_head_case(seed: int, B: int, k: int, V: int, H: int, chunk_rows: int = 2048) -> HeadCase:
+    """Hidden states N(0, 1) per element; weight entries uniform on
+    [-sqrt(3/H), sqrt(3/H)) (variance 1/H, so each logit has variance about
+    the squared norm of the hidden state over H, about 1); both rounded to
+    bf16.  The weight is generated in blocks of ``chunk_rows`` rows."""
+    hidden = f64_to_bf16_bits(normals_f64(seed, TAG_HEAD_HIDDEN, np.arange(B * (k + 1)), H)).reshape(B, k + 1, H)
+    a = np.sqrt(3.0 / H)
+    weight = np.empty((V, H), dtype=np.uint16)
+
+    def block(r0):
+        rows = np.arange(r0, min(V, r0 + chunk_rows))
+        x = _outputs(stream_state(seed, TAG_HEAD_WEIGHT, rows), H)
+        u = (x >> _U(40)).astype(np.float64) * 2.0 ** -24
+        weight[r0:r0 + rows.size] = f64_to_bf16_bits((2.0 * u - 1.0) * a)
+
+    starts = range(0, V, chunk_rows)
+    if len(starts) > 1:
+        from concurrent.futures import ThreadPoolExecutor
+
+        with ThreadPoolExecutor(min(16, os.cpu_count() or 1)) as ex:  # the blocks are independent
+            list(ex.map(block, starts))
+    else:
+        for r0 in starts:
+            block(r0)
+    return HeadCase(hidden, weight, B, k, V, H)
