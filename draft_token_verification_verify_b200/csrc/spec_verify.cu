@@ -1162,6 +1162,8 @@ sv_status_t spec_verify_head_greedy(const void* hidden, const void* weight, cons
     P.rows = rows;
     P.V = V;
     P.H = H;
+    P.mtiles = static_cast<int>(ceil_div(rows, sv::HEAD_BM));
+    P.tiles = P.mtiles * vtiles;
     P.best = reinterpret_cast<unsigned long long*>(base);
     P.err = err;
     P.timeout_ns = (opts && opts->wait_timeout_ns) ? opts->wait_timeout_ns : kDefaultTimeoutNs;
@@ -1189,8 +1191,9 @@ sv_status_t spec_verify_head_greedy(const void* hidden, const void* weight, cons
             result = SV_ERR_CUDA;
             break;
         }
-        sv::sv_head_kernel<<<dim3(static_cast<unsigned>(ceil_div(rows, sv::HEAD_BM)), static_cast<unsigned>(vtiles), 1),
-                             sv::HEAD_NT, sv::HEAD_SMEM, st>>>(tm_h, tm_w, P);
+        // persistent: one CTA per SM (its shared memory admits no second)
+        const int grid = P.tiles < info->sms ? P.tiles : info->sms;
+        sv::sv_head_kernel<<<grid, sv::HEAD_NT, sv::HEAD_SMEM, st>>>(tm_h, tm_w, P);
         if (cudaGetLastError() != cudaSuccess) {
             result = SV_ERR_CUDA;
             break;

@@ -23,13 +23,17 @@ namespace sv {
 constexpr int HEAD_BM = 128;  // hidden-state rows per tile: the tensor-memory lanes
 constexpr int HEAD_BN = 256;  // vocabulary entries per tile: fp32 tensor-memory columns
 constexpr int HEAD_BK = 64;   // K per stage: one 128-byte swizzle row of bf16
-constexpr int HEAD_STAGES = 2;
-constexpr int HEAD_NT = 128;  // four warps: one per 32-lane quarter of tensor memory
+constexpr int HEAD_STAGES = 4;
+// six warps: 0 issues the copies, 1 the MMAs, 2-5 read tensor memory (warp w
+// reaches the 32-lane quarter w % 4, so the four cover all 128 lanes)
+constexpr int HEAD_NT = 192;
+constexpr int HEAD_ACCS = 2;  // accumulators in tensor memory: the epilogue of one tile overlaps the next's MMAs
+constexpr int HEAD_TMEM_COLS = HEAD_ACCS * HEAD_BN;
 constexpr int HEAD_A_BYTES = HEAD_BM * HEAD_BK * 2;
 constexpr int HEAD_B_BYTES = HEAD_BN * HEAD_BK * 2;
 constexpr int HEAD_STAGE_BYTES = HEAD_A_BYTES + HEAD_B_BYTES;
 // stages, 1 KB of slack to align them to the 1,024-byte swizzle period, barriers
-constexpr int HEAD_SMEM = HEAD_STAGES * HEAD_STAGE_BYTES + 1024 + 128;
+constexpr int HEAD_SMEM = HEAD_STAGES * HEAD_STAGE_BYTES + 1024 + 256;
 constexpr int HEAD_DECIDE_NT = 128;  // one warp per sequence
 
 // Instruction descriptor of tcgen05.mma kind::f16: fp32 accumulator (bits 4-5),
@@ -55,6 +59,8 @@ struct HeadParams {
     int rows;  // B * (k + 1)
     int V;
     int H;
+    int mtiles;  // ceil(rows / HEAD_BM)
+    int tiles;   // mtiles * ceil(V / HEAD_BN)
     unsigned long long* best;  // [rows], zeroed before the launch
     int* err;                  // set to non-zero by a wait that ran out
     unsigned long long timeout_ns;
@@ -111,6 +117,9 @@ __device__ __forceinline__ void tmem_relinquish() {
 __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
 }
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
 __device__ __forceinline__ void tc_fence_before() {
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -150,14 +159,18 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-// ---- K_head: logits tile on the tensor cores, (max, argmax) per row ------------
+// ---- K_head: logits tiles on the tensor cores, (max, argmax) per row -----------
 //
-// Grid (ceil(rows / 128), ceil(V / 256)): the row tiles of one vocabulary tile
-// are neighbours in launch order, so their weight tile is read from HBM once
-// and from L2 by the others.  Warp 0's lane 0 issues the copies, warp 1's lane
-// 0 the MMAs (a two-stage ring per CTA, two CTAs per SM), then all four warps
-// read tensor memory.  Every wait is bounded; a wait that runs out sets *err.
-__global__ void __launch_bounds__(HEAD_NT, 2)
+// Persistent: one CTA per SM takes the tiles blockIdx.x, blockIdx.x + grid, ...
+// of the order (row tile fastest, then vocabulary tile), so the CTAs running
+// at one time cover whole groups of row tiles of the same vocabulary tile and
+// a weight tile comes from HBM once and from L2 for the others.  Warp 0's lane
+// 0 streams the copies of every tile through one ring of HEAD_STAGES stages;
+// warp 1's lane 0 issues each tile's MMAs into one of two accumulators; warps
+// 2-5 reduce a finished accumulator while the next tile's MMAs run in the
+// other.  Every wait is bounded; a wait that runs out sets *err, the roles
+// stop, and the CTA drains its copies and MMAs before it frees tensor memory.
+__global__ void __launch_bounds__(HEAD_NT, 1)
     sv_head_kernel(const __grid_constant__ CUtensorMap tm_h, const __grid_constant__ CUtensorMap tm_w,
                    HeadParams P) {
     extern __shared__ __align__(1024) unsigned char head_raw[];
@@ -165,12 +178,12 @@ __global__ void __launch_bounds__(HEAD_NT, 2)
     unsigned char* base = head_raw + ((1024u - (raw_s & 1023u)) & 1023u);
     uint64_t* full = reinterpret_cast<uint64_t*>(base + HEAD_STAGES * HEAD_STAGE_BYTES);
     uint64_t* empty = full + HEAD_STAGES;
-    uint64_t* accum = empty + HEAD_STAGES;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
+    uint64_t* tfull = empty + HEAD_STAGES;  // an accumulator holds a finished tile
+    uint64_t* tempty = tfull + HEAD_ACCS;   // the epilogue has read it
+    uint64_t* done = tempty + HEAD_ACCS;    // every MMA of this CTA is complete
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int m0 = blockIdx.x * HEAD_BM;
-    const int n0 = blockIdx.y * HEAD_BN;
     const int nk = (P.H + HEAD_BK - 1) / HEAD_BK;
 
     if (tid == 0) {
@@ -178,13 +191,17 @@ __global__ void __launch_bounds__(HEAD_NT, 2)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(accum, 1);
+        for (int a = 0; a < HEAD_ACCS; ++a) {
+            mbar_init(&tfull[a], 1);
+            mbar_init(&tempty[a], 4);  // one arrival per epilogue warp
+        }
+        mbar_init(done, 1);
         fence_mbar_init();
         tmap_prefetch(&tm_h);
         tmap_prefetch(&tm_w);
     }
     if (warp == 0) {
-        tmem_alloc(tmem_slot, HEAD_BN);
+        tmem_alloc(tmem_slot, HEAD_TMEM_COLS);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -194,76 +211,104 @@ __global__ void __launch_bounds__(HEAD_NT, 2)
     int failed = 0;
 
     if (warp == 0 && lane == 0) {
-        int kb = 0;
-        for (; kb < nk; ++kb) {
-            const int s = kb % HEAD_STAGES;
-            if (kb >= HEAD_STAGES &&
-                !mbar_wait_bounded(&empty[s], ((kb / HEAD_STAGES) - 1) & 1, P.timeout_ns)) {
-                failed = 1;
-                break;
+        int it = 0;  // stage uses so far, across tiles
+        for (int t = blockIdx.x; t < P.tiles && !failed; t += gridDim.x) {
+            const int m0 = (t % P.mtiles) * HEAD_BM, n0 = (t / P.mtiles) * HEAD_BN;
+            for (int kb = 0; kb < nk; ++kb, ++it) {
+                const int s = it % HEAD_STAGES;
+                if (it >= HEAD_STAGES &&
+                    !mbar_wait_bounded(&empty[s], ((it / HEAD_STAGES) - 1) & 1, P.timeout_ns)) {
+                    failed = 1;
+                    break;
+                }
+                unsigned char* st = base + s * HEAD_STAGE_BYTES;
+                mbar_arrive_expect_tx(&full[s], HEAD_STAGE_BYTES);
+                tma_load_2d(st, &tm_h, kb * HEAD_BK, m0, &full[s]);
+                tma_load_2d(st + HEAD_A_BYTES, &tm_w, kb * HEAD_BK, n0, &full[s]);
             }
-            unsigned char* st = base + s * HEAD_STAGE_BYTES;
-            mbar_arrive_expect_tx(&full[s], HEAD_STAGE_BYTES);
-            tma_load_2d(st, &tm_h, kb * HEAD_BK, m0, &full[s]);
-            tma_load_2d(st + HEAD_A_BYTES, &tm_w, kb * HEAD_BK, n0, &full[s]);
         }
         // no copy may land after the CTA is gone: wait for the last ones issued
-        for (int j = kb > HEAD_STAGES ? kb - HEAD_STAGES : 0; j < kb; ++j)
+        for (int j = it > HEAD_STAGES ? it - HEAD_STAGES : 0; j < it; ++j)
             if (!mbar_wait_bounded(&full[j % HEAD_STAGES], (j / HEAD_STAGES) & 1, P.timeout_ns)) failed = 1;
     } else if (warp == 1 && lane == 0) {
-        for (int kb = 0; kb < nk; ++kb) {
-            const int s = kb % HEAD_STAGES;
-            if (!mbar_wait_bounded(&full[s], (kb / HEAD_STAGES) & 1, P.timeout_ns)) {
+        int it = 0, lt = 0;
+        for (int t = blockIdx.x; t < P.tiles && !failed; t += gridDim.x, ++lt) {
+            const int acc = lt & 1;
+            if (lt >= HEAD_ACCS && !mbar_wait_bounded(&tempty[acc], ((lt >> 1) - 1) & 1, P.timeout_ns)) {
                 failed = 1;
                 break;
             }
             tc_fence_after();
-            const uint32_t a = smem_u32(base + s * HEAD_STAGE_BYTES);
-            const uint32_t b = a + HEAD_A_BYTES;
+            const uint32_t d = tmem + static_cast<uint32_t>(acc * HEAD_BN);
+            for (int kb = 0; kb < nk; ++kb, ++it) {
+                const int s = it % HEAD_STAGES;
+                if (!mbar_wait_bounded(&full[s], (it / HEAD_STAGES) & 1, P.timeout_ns)) {
+                    failed = 1;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t a = smem_u32(base + s * HEAD_STAGE_BYTES);
+                const uint32_t b = a + HEAD_A_BYTES;
 #pragma unroll
-            for (int kk = 0; kk < HEAD_BK / 16; ++kk)
-                umma_bf16(tmem, head_desc(a + kk * 32), head_desc(b + kk * 32), (kb | kk) != 0 ? 1u : 0u);
-            umma_commit(&empty[s]);  // frees the stage once these MMAs have read it
+                for (int kk = 0; kk < HEAD_BK / 16; ++kk)
+                    umma_bf16(d, head_desc(a + kk * 32), head_desc(b + kk * 32), (kb | kk) != 0 ? 1u : 0u);
+                umma_commit(&empty[s]);  // frees the stage once these MMAs have read it
+            }
+            if (!failed) umma_commit(&tfull[acc]);
         }
-        umma_commit(accum);  // every MMA issued above is complete when this phase completes
-    }
-    __syncwarp();
-
-    bool got = mbar_wait_bounded(accum, 0, P.timeout_ns);
-    if (got && P.test_hook) got = mbar_wait_bounded(accum, 1, P.timeout_ns);  // never completes
-    if (!got) failed = 1;
-    tc_fence_after();
-    if (__any_sync(0xffffffffu, failed) && lane == 0) atomicOr(P.err, 1);
-
-    if (__all_sync(0xffffffffu, got)) {
-        const int m = m0 + warp * 32 + lane;
-        float best = -__int_as_float(0x7f800000);
-        int arg = -1;
-        bool bad = false;
-        for (int c = 0; c < HEAD_BN / 32; ++c) {
-            const int col0 = n0 + c * 32;
-            if (col0 >= P.V) break;  // the same for the whole warp
-            uint32_t r[32];
-            tmem_ld32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + static_cast<uint32_t>(c * 32), r);
+        umma_commit(done);  // completes when every MMA issued above is complete
+    } else if (warp >= 2) {
+        const int q = warp & 3;  // the tensor-memory quarter this warp may read
+        int lt = 0;
+        for (int t = blockIdx.x; t < P.tiles; t += gridDim.x, ++lt) {
+            const int acc = lt & 1;
+            bool got = mbar_wait_bounded(&tfull[acc], (lt >> 1) & 1, P.timeout_ns);
+            if (got && P.test_hook) got = mbar_wait_bounded(&tfull[acc], ((lt >> 1) & 1) ^ 1, P.timeout_ns);
+            if (!__all_sync(0xffffffffu, got)) {
+                failed = 1;
+                break;
+            }
+            tc_fence_after();
+            const int m = (t % P.mtiles) * HEAD_BM + q * 32 + lane;
+            const int n0 = (t / P.mtiles) * HEAD_BN;
+            float best = -__int_as_float(0x7f800000);
+            int arg = -1;
+            bool bad = false;
+            for (int c = 0; c < HEAD_BN / 32; ++c) {
+                const int col0 = n0 + c * 32;
+                if (col0 >= P.V) break;  // the same for the whole warp
+                uint32_t r[32];
+                tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) +
+                              static_cast<uint32_t>(acc * HEAD_BN + c * 32),
+                          r);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const float z = __uint_as_float(r[j]);
-                if (col0 + j < P.V) {
-                    bad |= !(z == z) || z == __int_as_float(0x7f800000);
-                    if (z > best) {  // ascending index: the first of equal maxima stays
-                        best = z;
-                        arg = col0 + j;
+                for (int j = 0; j < 32; ++j) {
+                    const float z = __uint_as_float(r[j]);
+                    if (col0 + j < P.V) {
+                        bad |= !(z == z) || z == __int_as_float(0x7f800000);
+                        if (z > best) {  // ascending index: the first of equal maxima stays
+                            best = z;
+                            arg = col0 + j;
+                        }
                     }
                 }
             }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[acc]);  // the accumulator may take the tile after next
+            if (m < P.rows && (bad || arg >= 0)) atomicMax(P.best + m, bad ? HEAD_BAD : head_key(best, arg));
         }
-        if (m < P.rows && (bad || arg >= 0)) atomicMax(P.best + m, bad ? HEAD_BAD : head_key(best, arg));
     }
+    __syncwarp();
+    if (__any_sync(0xffffffffu, failed) && lane == 0) atomicOr(P.err, 1);
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
+        // the MMAs of a CTA that stopped early may still be running: free tensor memory after them
+        if (lane == 0 && !mbar_wait_bounded(done, 0, P.timeout_ns)) atomicOr(P.err, 1);
+        __syncwarp();
         tc_fence_after();
-        tmem_dealloc(tmem, HEAD_BN);
+        tmem_dealloc(tmem, HEAD_TMEM_COLS);
     }
 }
 
