@@ -865,7 +865,25 @@ bool encode_bf16_rows(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t 
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-constexpr int kHeadMaxVTiles = 65535;  // grid y
+constexpr int kHeadMaxVTiles = 65535;  // grid y of the first design; kept as the size bound
+
+// Vocabulary entries per tile of the persistent projection kernel: the
+// multiple of 16 in [64, 256] that minimises (rounds of tiles over the SMs) x
+// (entries per tile + a fixed per-tile cost), so the last round is as full as
+// the shape allows (151,936 entries, 3 row tiles, 148 SMs: 240, 12.9 rounds).
+int head_plan_bn(int mtiles, int V, int sms) {
+    int best = sv::HEAD_BN;
+    long long best_cost = LLONG_MAX;
+    for (int bn = sv::HEAD_BN; bn >= 64; bn -= 16) {
+        const long long tiles = static_cast<long long>(mtiles) * ceil_div(V, bn);
+        const long long cost = ceil_div(tiles, sms) * (bn + 16);
+        if (cost < best_cost) {
+            best_cost = cost;
+            best = bn;
+        }
+    }
+    return best;
+}
 
 // Workspace of the fused path: each row's running best (8 bytes) and the
 // timeout flag, zeroed by one memset per call.  0 on invalid sizes.
@@ -1131,11 +1149,13 @@ sv_status_t spec_verify_head_greedy(const void* hidden, const void* weight, cons
     const DeviceInfo* info = device_info(&dev);
     if (!info) return SV_ERR_UNSUPPORTED;
     const int rows = B * (k + 1);
-    const int vtiles = static_cast<int>(ceil_div(V, sv::HEAD_BN));
+    const int mtiles = static_cast<int>(ceil_div(rows, sv::HEAD_BM));
+    const int bn = head_plan_bn(mtiles, V, info->sms);
+    const int vtiles = static_cast<int>(ceil_div(V, bn));
     CUtensorMap tm_h, tm_w;
     if (!tensor_map_encoder()) return SV_ERR_UNSUPPORTED;
     if (!encode_bf16_rows(&tm_h, hidden, static_cast<uint64_t>(H), static_cast<uint64_t>(rows), sv::HEAD_BM) ||
-        !encode_bf16_rows(&tm_w, weight, static_cast<uint64_t>(H), static_cast<uint64_t>(V), sv::HEAD_BN))
+        !encode_bf16_rows(&tm_w, weight, static_cast<uint64_t>(H), static_cast<uint64_t>(V), static_cast<uint32_t>(bn)))
         return SV_ERR_INVALID_ARG;
     std::call_once(g_head_attr_once[dev], [dev] {
         g_head_attr_err[dev] =
@@ -1162,8 +1182,9 @@ sv_status_t spec_verify_head_greedy(const void* hidden, const void* weight, cons
     P.rows = rows;
     P.V = V;
     P.H = H;
-    P.mtiles = static_cast<int>(ceil_div(rows, sv::HEAD_BM));
-    P.tiles = P.mtiles * vtiles;
+    P.bn = bn;
+    P.mtiles = mtiles;
+    P.tiles = mtiles * vtiles;
     P.best = reinterpret_cast<unsigned long long*>(base);
     P.err = err;
     P.timeout_ns = (opts && opts->wait_timeout_ns) ? opts->wait_timeout_ns : kDefaultTimeoutNs;

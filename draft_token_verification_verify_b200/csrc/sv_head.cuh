@@ -21,7 +21,7 @@
 namespace sv {
 
 constexpr int HEAD_BM = 128;  // hidden-state rows per tile: the tensor-memory lanes
-constexpr int HEAD_BN = 256;  // vocabulary entries per tile: fp32 tensor-memory columns
+constexpr int HEAD_BN = 256;  // vocabulary entries per tile at most: fp32 tensor-memory columns
 constexpr int HEAD_BK = 64;   // K per stage: one 128-byte swizzle row of bf16
 constexpr int HEAD_STAGES = 4;
 // six warps: 0 issues the copies, 1 the MMAs, 2-5 read tensor memory (warp w
@@ -38,10 +38,11 @@ constexpr int HEAD_DECIDE_NT = 128;  // one warp per sequence
 
 // Instruction descriptor of tcgen05.mma kind::f16: fp32 accumulator (bits 4-5),
 // bf16 A and B (bits 7-9, 10-12), both K-major (bits 15, 16 clear), N / 8 at
-// bit 17, M / 16 at bit 24.
-constexpr uint32_t HEAD_IDESC = (1u << 4) | (1u << 7) | (1u << 10) |
-                                (static_cast<uint32_t>(HEAD_BN >> 3) << 17) |
-                                (static_cast<uint32_t>(HEAD_BM >> 4) << 24);
+// bit 17, M / 16 at bit 24; N = bn, the tile's vocabulary entries.
+__host__ __device__ constexpr uint32_t head_idesc(int bn) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(bn >> 3) << 17) |
+           (static_cast<uint32_t>(HEAD_BM >> 4) << 24);
+}
 
 // A row's running best as one orderable 64-bit word: the order-preserving
 // bits of the largest logit (-0.0 taken as +0.0) above the complement of its
@@ -59,8 +60,9 @@ struct HeadParams {
     int rows;  // B * (k + 1)
     int V;
     int H;
+    int bn;      // vocabulary entries per tile: a multiple of 16 in [64, HEAD_BN]
     int mtiles;  // ceil(rows / HEAD_BM)
-    int tiles;   // mtiles * ceil(V / HEAD_BN)
+    int tiles;   // mtiles * ceil(V / bn)
     unsigned long long* best;  // [rows], zeroed before the launch
     int* err;                  // set to non-zero by a wait that ran out
     unsigned long long timeout_ns;
@@ -127,13 +129,14 @@ __device__ __forceinline__ void tc_fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// D (tensor memory) = A . B^T (+ D when `acc`), M = 128, N = 256, K = 16, bf16.
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t acc) {
+// D (tensor memory) = A . B^T (+ D when `acc`), K = 16, bf16; M and N from `idesc`.
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t acc) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(HEAD_IDESC), "r"(acc)
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
         : "memory");
 }
 
@@ -185,6 +188,8 @@ __global__ void __launch_bounds__(HEAD_NT, 1)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nk = (P.H + HEAD_BK - 1) / HEAD_BK;
+    const int bn = P.bn;
+    const uint32_t stage_tx = static_cast<uint32_t>(HEAD_A_BYTES + bn * HEAD_BK * 2);  // the two boxes
 
     if (tid == 0) {
         for (int s = 0; s < HEAD_STAGES; ++s) {
@@ -213,7 +218,7 @@ __global__ void __launch_bounds__(HEAD_NT, 1)
     if (warp == 0 && lane == 0) {
         int it = 0;  // stage uses so far, across tiles
         for (int t = blockIdx.x; t < P.tiles && !failed; t += gridDim.x) {
-            const int m0 = (t % P.mtiles) * HEAD_BM, n0 = (t / P.mtiles) * HEAD_BN;
+            const int m0 = (t % P.mtiles) * HEAD_BM, n0 = (t / P.mtiles) * bn;
             for (int kb = 0; kb < nk; ++kb, ++it) {
                 const int s = it % HEAD_STAGES;
                 if (it >= HEAD_STAGES &&
@@ -222,7 +227,7 @@ __global__ void __launch_bounds__(HEAD_NT, 1)
                     break;
                 }
                 unsigned char* st = base + s * HEAD_STAGE_BYTES;
-                mbar_arrive_expect_tx(&full[s], HEAD_STAGE_BYTES);
+                mbar_arrive_expect_tx(&full[s], stage_tx);
                 tma_load_2d(st, &tm_h, kb * HEAD_BK, m0, &full[s]);
                 tma_load_2d(st + HEAD_A_BYTES, &tm_w, kb * HEAD_BK, n0, &full[s]);
             }
@@ -232,6 +237,7 @@ __global__ void __launch_bounds__(HEAD_NT, 1)
             if (!mbar_wait_bounded(&full[j % HEAD_STAGES], (j / HEAD_STAGES) & 1, P.timeout_ns)) failed = 1;
     } else if (warp == 1 && lane == 0) {
         int it = 0, lt = 0;
+        const uint32_t idesc = head_idesc(bn);
         for (int t = blockIdx.x; t < P.tiles && !failed; t += gridDim.x, ++lt) {
             const int acc = lt & 1;
             if (lt >= HEAD_ACCS && !mbar_wait_bounded(&tempty[acc], ((lt >> 1) - 1) & 1, P.timeout_ns)) {
@@ -251,7 +257,7 @@ __global__ void __launch_bounds__(HEAD_NT, 1)
                 const uint32_t b = a + HEAD_A_BYTES;
 #pragma unroll
                 for (int kk = 0; kk < HEAD_BK / 16; ++kk)
-                    umma_bf16(d, head_desc(a + kk * 32), head_desc(b + kk * 32), (kb | kk) != 0 ? 1u : 0u);
+                    umma_bf16(d, head_desc(a + kk * 32), head_desc(b + kk * 32), idesc, (kb | kk) != 0 ? 1u : 0u);
                 umma_commit(&empty[s]);  // frees the stage once these MMAs have read it
             }
             if (!failed) umma_commit(&tfull[acc]);
@@ -270,13 +276,14 @@ __global__ void __launch_bounds__(HEAD_NT, 1)
             }
             tc_fence_after();
             const int m = (t % P.mtiles) * HEAD_BM + q * 32 + lane;
-            const int n0 = (t / P.mtiles) * HEAD_BN;
+            const int n0 = (t / P.mtiles) * bn;
+            const int n1 = n0 + bn < P.V ? n0 + bn : P.V;  // the tile's columns: n0 .. n1
             float best = -__int_as_float(0x7f800000);
             int arg = -1;
             bool bad = false;
-            for (int c = 0; c < HEAD_BN / 32; ++c) {
+            for (int c = 0; c < HEAD_BN / 32; ++c) {  // 32-column loads within the 256 allocated
                 const int col0 = n0 + c * 32;
-                if (col0 >= P.V) break;  // the same for the whole warp
+                if (col0 >= n1) break;  // the same for the whole warp
                 uint32_t r[32];
                 tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) +
                               static_cast<uint32_t>(acc * HEAD_BN + c * 32),
@@ -284,7 +291,7 @@ __global__ void __launch_bounds__(HEAD_NT, 1)
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
                     const float z = __uint_as_float(r[j]);
-                    if (col0 + j < P.V) {
+                    if (col0 + j < n1) {
                         bad |= !(z == z) || z == __int_as_float(0x7f800000);
                         if (z > best) {  // ascending index: the first of equal maxima stays
                             best = z;
