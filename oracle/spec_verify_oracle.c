@@ -21,6 +21,10 @@
  *     the target's most probable token and replaces it at the first
  *     mismatch; temperature / top-k must be applied identically to p and q
  *     and kept consistent in the correction step.
+ *   - same section, paragraph 1: the target scores the k+1 positions in one
+ *     forward pass; its last step, the output projection of the hidden
+ *     states, is written out in oracle_head_logits (end of this file) for
+ *     greedy verification on the logits it forms.
  *
  * Readings of what the pages leave open (each stated where it is used):
  *   R1 accept iff u*q < p  (i.e. u < min(1, p/q) for u in [0,1));
