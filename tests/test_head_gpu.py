@@ -130,6 +130,7 @@ def _case_and_ref(seed, B, k, V, H, seqs=None, threads=4):
     (50, 4, 4099, 512),   # 250 rows: a full and a ragged row tile
     (4, 40, 300, 8),      # long drafts, H below one K block
     (5, 2, 1, 64),        # a vocabulary of one
+    (100, 7, 5003, 320),  # 800 rows: seven row tiles, the last one of 32 rows
 ])
 def test_parity_small(B, k, V, H):
     case, drafts, ref = _case_and_ref(10 + B + k, B, k, V, H)
@@ -215,3 +216,48 @@ def test_caller_workspace_is_written_before_read():
     for x, y in zip(a, b):
         assert np.array_equal(x, y)
     _check(case, drafts, ref, *a[:3])
+
+
+def test_single_sequence_full_vocabulary():
+    """B = 1, k = 1 at V = 151,936, H = 4,096: one row tile, many narrow vocabulary tiles."""
+    case, drafts, ref = _case_and_ref(27, 1, 1, 151936, 4096)
+    tok, n, arg, status = _run(case, drafts)
+    assert status == 0
+    _check(case, drafts, ref, tok, n, arg)
+
+
+def test_graph_capture_and_replay():
+    """The call (a memset and two launches on the caller's stream) captures
+    into a CUDA graph; replays give the eager result."""
+    import torch
+
+    import draft_token_verification_verify_b200 as sv
+
+    case, drafts, ref = _case_and_ref(28, 12, 4, 20011, 512)
+    dev = torch.device("cuda:0")
+    h, w, d = to_dev(case.hidden), to_dev(case.weight), torch.from_numpy(drafts).to(dev)
+    ws = torch.empty((sv.spec_verify_head_workspace_size(12, 4, 20011, 512),), dtype=torch.uint8, device=dev)
+    tok = torch.empty((12, 5), dtype=torch.int32, device=dev)
+    n = torch.empty((12,), dtype=torch.int32, device=dev)
+    arg = torch.empty((12, 5), dtype=torch.int32, device=dev)
+    s = torch.cuda.Stream()
+
+    def call():
+        st = sv.spec_verify_head_greedy(h, w, d, 12, 4, 20011, 512, tok, n, arg, ws, ws.numel(), None, None, s)
+        assert st == sv.SV_OK
+
+    with torch.cuda.stream(s):
+        call()  # first call outside capture (one-time attribute and driver lookups)
+    torch.cuda.synchronize()
+    eager = [t.cpu().numpy().copy() for t in (tok, n, arg)]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        call()
+    for t in (tok, n, arg):
+        t.fill_(-9)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    for t, e in zip((tok, n, arg), eager):
+        assert np.array_equal(t.cpu().numpy(), e)
+    _check(case, drafts, ref, *eager)
