@@ -34,6 +34,10 @@ constexpr int HEAD_B_BYTES = HEAD_BN * HEAD_BK * 2;
 constexpr int HEAD_STAGE_BYTES = HEAD_A_BYTES + HEAD_B_BYTES;
 // stages, 1 KB of slack to align them to the 1,024-byte swizzle period, barriers
 constexpr int HEAD_SMEM = HEAD_STAGES * HEAD_STAGE_BYTES + 1024 + 256;
+// each CTA allocates all 512 tensor-memory columns of its SM, so no second CTA
+// may ever be resident beside it: its shared memory alone rules that out
+// (228 KB per SM, 1 KB of it reserved per CTA)
+static_assert(2 * (HEAD_SMEM + 1024) > 228 * 1024, "two projection CTAs must not fit on one SM");
 constexpr int HEAD_DECIDE_NT = 128;  // one warp per sequence
 
 // Instruction descriptor of tcgen05.mma kind::f16: fp32 accumulator (bits 4-5),
