@@ -41,6 +41,9 @@ KSAMPLES = 40  # event-bracketed launches of the streaming kernel per workload
 # sources that define the streaming kernel (the one the roofline figures describe)
 KERNEL_SOURCES = [os.path.join(ROOT, "draft_token_verification_verify_b200", "csrc", f)
                   for f in ("sv_rows.cuh", "sv_common.cuh", "sv_ptx.cuh")]
+# and the output projection kernel
+HEAD_SOURCES = [os.path.join(ROOT, "draft_token_verification_verify_b200", "csrc", f)
+                for f in ("sv_head.cuh", "sv_ptx.cuh")]
 
 WORKLOAD_ORDER = ("batched", "greedy", "large", "single", "tiny")
 GRAPH_WORKLOADS = ("single", "tiny")  # launch-bound: also timed from a CUDA-graph replay
@@ -93,18 +96,18 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(sources=None) -> str:
     h = hashlib.sha256()
-    for p in KERNEL_SOURCES:
+    for p in (KERNEL_SOURCES if sources is None else sources):
         with open(p, "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload: str):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel source (else None)."""
-    path = os.path.join(PROFILE_DIR, f"sv_rows_kernel_{workload}.md")
+def profiled_traffic(workload: str, kernel: str = "sv_rows_kernel", sources=None):
+    """DRAM bytes per launch from the committed ncu summary of `kernel` on
+    `workload`, if it was taken on the current kernel source (else None)."""
+    path = os.path.join(PROFILE_DIR, f"{kernel}_{workload}.md")
     if not os.path.exists(path):
         return None
     vals = {}
@@ -112,7 +115,7 @@ def profiled_traffic(workload: str):
         if line.startswith("- ") and ":" in line:
             k, v = line[2:].split(":", 1)
             vals[k.strip()] = v.strip().strip("`")
-    if vals.get("kernel_source_sha256_16") != kernel_source_hash():
+    if vals.get("kernel_source_sha256_16") != kernel_source_hash(sources):
         return None
     try:
         return float(vals["dram_bytes_per_launch"])
@@ -751,6 +754,7 @@ def measure_head(args, sv, dev, world, rank):
             "ms_per_step": ms / args.steps, "gpu_launches": 2 * args.steps, "clocks": clocks,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "peak_source": src, "kernel": "sv_head_kernel",
+                         "traffic": profiled_traffic("head_greedy", "sv_head_kernel", HEAD_SOURCES),
                          "kernel_ms_mean": kmean, "kernel_ms_median": statistics.median(kern_ms),
                          "kernel_samples": len(kern_ms), "flops_per_launch": flops,
                          "weight_gbs": w_bytes / (kmean / 1000.0) / 1e9, "weight_bytes": w_bytes},

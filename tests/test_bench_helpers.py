@@ -29,6 +29,7 @@ def test_profiled_traffic_only_for_the_current_source(tmp_path, monkeypatch):
 
 def test_committed_profile_matches_the_kernel_source():
     assert bench.profiled_traffic("batched") is not None
+    assert bench.profiled_traffic("head_greedy", "sv_head_kernel", bench.HEAD_SOURCES) is not None
 
 
 def test_measured_peak_fallback(tmp_path, monkeypatch):
