@@ -3,13 +3,14 @@
 // The target scores the k+1 positions of every sequence in one forward pass
 // (entry "推测解码", section "提议与核验的基本步骤", paragraph 1); greedy
 // verification needs only each position's lowest-index argmax (paragraph 4).
-// K_head computes the logits z = h . W[v] of a 128-row x 256-entry tile on the
-// tensor cores (tcgen05.mma, bf16 operands staged by 2D tensor-map copies in
-// the 128-byte-swizzled K-major layout, fp32 accumulators in tensor memory)
-// and its epilogue reduces the tile to each row's (maximum, lowest index)
-// straight out of tensor memory and folds it into the row's running best with
-// one 64-bit atomic maximum: the logits are never written.  K_decide walks
-// the chain on the rows' results.
+// K_head computes the logits z = h . W[v] in tiles of 128 rows x up to 256
+// vocabulary entries on the tensor cores (tcgen05.mma, bf16 operands staged by
+// 2D tensor-map copies in the 128-byte-swizzled K-major layout, fp32
+// accumulators in tensor memory; one persistent CTA per SM works through the
+// tiles) and its epilogue reduces each tile to each row's (maximum, lowest
+// index) straight out of tensor memory and folds it into the row's running
+// best with one 64-bit atomic maximum: the logits are never written.
+// K_decide walks the chain on the rows' results.
 #pragma once
 
 #include <cuda.h>  // CUtensorMap (the type only; the map is encoded on the host)
